@@ -1,0 +1,156 @@
+"""Gated sliding-window attention core (ZGCM-1 GatedSWA without projections) on B200.
+
+A thin ctypes binding over ``libswa.so`` (the C ABI in ``include/swa.h``).
+This module only marshals arguments: every step of the computation runs in
+the library's sm_100a kernels.  If the compiled library is missing, importing
+the binding raises, so there is no silent CPU fallback.
+
+PyTorch serves as the owner of device memory and streams: tensors are passed
+by ``data_ptr()`` and calls are enqueued on the current CUDA stream.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["fwd", "bwd", "bwd_workspace_size", "decode_step", "get_last_device_error",
+           "SwaError", "Params", "lib", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswa.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT = 0, 1, 2, 3, 4
+FLAG_FORCE_TIMEOUT = 1
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``swa_params_t``."""
+    _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("rot_dim", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("rope_base", ctypes.c_double), ("eps", ctypes.c_float), ("scale", ctypes.c_float)]
+
+
+class SwaError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {lib().swa_error_string(code).decode()} (code {code})")
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def lib():
+    """The loaded ``libswa.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m hybrid_sliding_window_gated_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(Params)
+        L.swa_fwd.argtypes = [P] + [_vp] * 9
+        L.swa_fwd.restype = ctypes.c_int
+        L.swa_bwd.argtypes = [P] + [_vp] * 15 + [ctypes.c_size_t, _vp]
+        L.swa_bwd.restype = ctypes.c_int
+        L.swa_bwd_workspace_size.argtypes = [P]
+        L.swa_bwd_workspace_size.restype = ctypes.c_size_t
+        L.swa_decode_step.argtypes = [P] + [_vp] * 11
+        L.swa_decode_step.restype = ctypes.c_int
+        L.swa_error_string.argtypes = [ctypes.c_int]
+        L.swa_error_string.restype = ctypes.c_char_p
+        L.swa_get_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int)]
+        L.swa_get_last_device_error.restype = ctypes.c_int
+        L.swa_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc, where):
+    if rc != OK:
+        raise SwaError(rc, where)
+
+
+def make_params(B, T, Hq, Hkv, *, head_dim=128, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
+                scale=0.0, flags=0):
+    return Params(B, T, Hq, Hkv, head_dim, window, rot_dim, flags, rope_base, eps, scale)
+
+
+def fwd(q, k, v, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6, scale=0.0,
+        out=None, lse=None, want_lse=False, flags=0, stream=None):
+    """o = A_SWA(RoPE(RMSNorm(q)), RoPE(RMSNorm(k)), v) * sigmoid(g).
+
+    q, g: [B,T,Hq,128] bf16; k, v: [B,T,Hkv,128] bf16; wq, wk: [128] fp32 (CUDA).
+    Returns o (and lse [B,Hq,T] fp32 when ``want_lse`` or ``lse`` is given).
+    """
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale, flags=flags)
+    rc = lib().swa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
+                       _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc, "swa_fwd")
+    return (out, lse) if lse is not None else out
+
+
+def bwd_workspace_size(B, T, Hq, Hkv, *, head_dim=128, window=128, rot_dim=42):
+    p = make_params(B, T, Hq, Hkv, head_dim=head_dim, window=window, rot_dim=rot_dim)
+    return int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
+
+
+def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
+        scale=0.0, workspace=None, grads=None, stream=None):
+    """Gradients (dq, dk, dv, dg, dwq, dwk) of sum(o * dO) for the forward above."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g),
+                 torch.zeros(D, dtype=torch.float32, device=q.device),
+                 torch.zeros(D, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dg, dwq, dwk = grads
+    nbytes = int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().swa_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
+                       _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq),
+                       _ptr(dwk), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "swa_bwd")
+    return grads
+
+
+def decode_step(pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, *, rot_dim=42, rope_base=1e7,
+                eps=1e-6, scale=0.0, out=None, stream=None):
+    """One decode step; updates the [N,Hkv,128,128] rings in place, returns o [N,Hq,128]."""
+    N, Hq, D = q.shape
+    Hkv, W = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    p = make_params(N, 1, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
+                    eps=eps, scale=scale)
+    rc = lib().swa_decode_step(ctypes.byref(p), _ptr(pos), _ptr(q), _ptr(k_new), _ptr(v_new),
+                               _ptr(g), _ptr(wq), _ptr(wk), _ptr(k_cache), _ptr(v_cache), _ptr(out),
+                               _stream(stream))
+    _check(rc, "swa_decode_step")
+    return out
+
+
+def get_last_device_error(stream=None):
+    """(code, site): SWA_OK or SWA_ERR_DEVICE_TIMEOUT with the raw site word; clears it."""
+    site = ctypes.c_int(0)
+    rc = lib().swa_get_last_device_error(_stream(stream), ctypes.byref(site))
+    return rc, site.value

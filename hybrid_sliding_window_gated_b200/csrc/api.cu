@@ -1,0 +1,232 @@
+// api.cu -- the C ABI declared in include/swa.h: argument validation, TMA
+// tensor-map construction, kernel launch and error mapping.  No entry point
+// allocates device memory or synchronises (except swa_get_last_device_error).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "swa_internal.h"
+
+namespace swa {
+
+// Sticky per-device error word written by bounded waits that ran out.
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_num_sms[kMaxDevices] = {0};
+int* g_err_ptr[kMaxDevices] = {nullptr};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int map_cuda_error(cudaError_t e) { return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA; }
+
+int current_device_info(DeviceInfo* info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SWA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return SWA_ERR_CUDA;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return SWA_ERR_UNSUPPORTED;  // built for sm_100a only
+    g_num_sms[dev] = n;
+  }
+  info->device = dev;
+  info->num_sms = g_num_sms[dev];
+  return SWA_OK;
+}
+
+int device_error_word(int** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SWA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return SWA_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  *ptr = g_err_ptr[dev];
+  return SWA_OK;
+}
+
+int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint64_t d3, uint32_t box0, uint32_t box1, uint32_t box2, uint32_t box3,
+                   CUtensorMapSwizzle swizzle) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return SWA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};  // bytes, dims 1..3
+  const cuuint32_t box[4] = {box0, box1, box2, box3};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : SWA_ERR_CUDA;
+}
+
+// Shape checks shared by every entry point.  Returns SWA_OK, INVALID_ARG or
+// UNSUPPORTED (a valid shape the tensor-core path is not built for).
+int check_params(const swa_params_t* p, bool decode) {
+  if (p == nullptr) return SWA_ERR_INVALID_ARG;
+  if (p->B < 0 || (!decode && p->T < 0) || p->Hq <= 0 || p->Hkv <= 0 || p->head_dim <= 0 ||
+      p->window <= 0 || p->rot_dim < 0 || (p->rot_dim & 1) || p->rot_dim > p->head_dim ||
+      !(p->eps >= 0.0f) || !(p->scale >= 0.0f) || (p->Hq % p->Hkv) != 0 ||
+      (p->rot_dim > 0 && !(p->rope_base > 0.0)))
+    return SWA_ERR_INVALID_ARG;
+  if (p->head_dim != kHeadDim || p->window != kWindow) return SWA_ERR_UNSUPPORTED;
+  if (!(p->rot_dim == 0 || p->rot_dim == 32 || p->rot_dim == 42 || p->rot_dim == 48))
+    return SWA_ERR_UNSUPPORTED;
+  if (p->B > (1ll << 30) || (!decode && p->T > (1ll << 30)) || p->Hq > 4096)
+    return SWA_ERR_UNSUPPORTED;
+  return SWA_OK;
+}
+
+static float score_scale(const swa_params_t* p) {
+  return p->scale > 0.0f ? p->scale : static_cast<float>(1.0 / std::sqrt((double)p->head_dim));
+}
+
+static void fill_inv_freq(const swa_params_t* p, double* out) {
+  for (int j = 0; j < kMaxPairs; ++j)
+    out[j] = (2 * j < p->rot_dim) ? std::pow(p->rope_base, -2.0 * j / p->rot_dim) : 0.0;
+}
+
+}  // namespace swa
+
+using namespace swa;
+
+extern "C" {
+
+const char* swa_version(void) { return "swa-b200 0.1 (sm_100a)"; }
+
+const char* swa_error_string(int code) {
+  switch (code) {
+    case SWA_OK: return "ok";
+    case SWA_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer or bad shape)";
+    case SWA_ERR_UNSUPPORTED: return "unsupported shape for the sm_100a tensor-core path";
+    case SWA_ERR_CUDA: return "a CUDA runtime call failed";
+    case SWA_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
+    default: return "unknown error";
+  }
+}
+
+int swa_get_last_device_error(void* stream, int* site) {
+  int* word = nullptr;
+  int rc = device_error_word(&word);
+  if (rc != SWA_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SWA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SWA_ERR_CUDA;
+  if (site) *site = v;
+  if (v == 0) return SWA_OK;
+  const int zero = 0;
+  if (cudaMemcpy(word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return SWA_ERR_CUDA;
+  return SWA_ERR_DEVICE_TIMEOUT;
+}
+
+int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
+            const swa_bf16_t* g, const float* wq, const float* wk, swa_bf16_t* o, float* lse,
+            void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  if (!q || !k || !v || !g || !wq || !wk || !o) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o) ||
+      !aligned16(wq) || !aligned16(wk) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+
+  FwdArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.tiles_per_chain = static_cast<int>((p->T + kTile - 1) / kTile);
+  a.total_tiles = static_cast<long long>(a.tiles_per_chain) * p->B * p->Hkv;
+  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.flags = p->flags;
+  a.wq = wq;
+  a.wk = wk;
+  a.g = g;
+  a.o = o;
+  a.lse = lse;
+  rc = device_error_word(&a.err);
+  if (rc != SWA_OK) return rc;
+  fill_inv_freq(p, a.inv_freq);
+
+  CUtensorMap tq, tk, tv, tg;
+  const uint64_t D = kHeadDim, T = p->T, B = p->B;
+  if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 128, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_NONE)))
+    return rc;
+  return launch_fwd(p, tq, tk, tv, tg, a, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// Entry points whose kernels live in their own translation units.
+namespace swa {
+int swa_bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                 const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                 swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream);
+size_t swa_bwd_workspace_bytes(const swa_params_t* p);
+int swa_decode_impl(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
+                    const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
+                    const float* wq, const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                    swa_bf16_t* o, cudaStream_t stream);
+}  // namespace swa
+
+extern "C" {
+
+int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
+            const swa_bf16_t* g, const float* wq, const float* wk, const float* lse,
+            const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk, swa_bf16_t* dv, swa_bf16_t* dg,
+            float* dwq, float* dwk, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  return swa_bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, workspace,
+                      workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t swa_bwd_workspace_size(const swa_params_t* p) {
+  if (check_params(p, false) != SWA_OK) return 0;
+  return swa_bwd_workspace_bytes(p);
+}
+
+int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
+                    const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
+                    const float* wq, const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                    swa_bf16_t* o, void* stream) {
+  int rc = check_params(p, true);
+  if (rc != SWA_OK) return rc;
+  return swa_decode_impl(p, pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, o,
+                         static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

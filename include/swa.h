@@ -1,0 +1,149 @@
+/*
+ * swa.h -- C ABI of the gated sliding-window attention core for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation is the GatedSWA module of ZGCM-1 without its projections:
+ *
+ *   O = A_SWA(q', k', v) (*) sigma(g),   q' = RoPE(RMSNorm(q)),  k' = RoPE(RMSNorm(k))
+ *
+ * Sources: "7.39B 오픈 모델로 256K 문맥의 수학 추론과 에이전트 검색을 겨냥한 ZGCM-1"
+ * (onedev.kr), section "어떻게 동작하나": GatedSWA(h) = o_proj(A_SWA(q,k,v) (*)
+ * sigma(g_proj(h))), 32 query heads and 8 KV heads of dim 128, a 128-token
+ * window, RMSNorm as the QK normalisation and partial RoPE with rotary
+ * fraction 0.33; and "ZGCM-1: A Fully Open and Extremely Efficient Foundation
+ * Model for Math and Agentic Search" (jaehun.me), section "How Gated SWA
+ * Behaves": norm and partial RoPE on q and k, GQA attention inside the window
+ * (a token sees the window including itself), element-wise sigmoid gate.
+ * Section "Why the KV Cache Shrinks by 6.4x" of the same page fixes that a
+ * window layer keeps only its last W tokens, which is the decode ring below.
+ *
+ * Readings taken where the pages are silent:
+ *   - RMSNorm per head over head_dim: y = x / sqrt(mean(x^2) + eps) * w, one
+ *     fp32 weight vector [head_dim] for q and one for k, shared by all heads;
+ *   - RoPE after the norm on the first rot_dim dims, rotate-half pairs
+ *     (j, j + rot_dim/2) turned by pos * rope_base^(-2j/rot_dim); the other
+ *     dims pass through; prefill positions are 0 .. T-1;
+ *   - scores scaled by `scale` (0 selects 1/sqrt(head_dim)); query i attends
+ *     keys max(0, i-window+1) .. i; q head h reads KV head h / (Hq/Hkv);
+ *   - sigma(g) = 1/(1+exp(-g)) per output element; g are gate logits.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *     row-major, 16-byte aligned.  Prefill tensors are [B, T, H, head_dim]
+ *     (H = Hq for q, g, o, dq, dg; H = Hkv for k, v, dk, dv).  bf16 data is
+ *     passed as swa_bf16_t (raw bits).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The library never synchronises and allocates no
+ *     device memory; it keeps only small per-device caches (SM count, kernel
+ *     attributes).
+ *   - The tensor-core path needs head_dim == 128, window == 128, Hq a
+ *     multiple of Hkv and rot_dim even in {0, 32, 42, 48}.  Other shapes return
+ *     SWA_ERR_UNSUPPORTED; nothing silently falls back to a slow path.
+ *   - Errors: SWA_OK on success; SWA_ERR_INVALID_ARG (null or misaligned
+ *     pointer, negative size, Hq % Hkv != 0, ...); SWA_ERR_UNSUPPORTED;
+ *     SWA_ERR_CUDA (a CUDA runtime call failed, e.g. the launch); the kernels
+ *     bound every internal wait and, when one runs out, record the site in a
+ *     sticky device word that swa_get_last_device_error() returns as
+ *     SWA_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t swa_bf16_t; /* bf16 bit pattern */
+
+enum {
+  SWA_OK = 0,
+  SWA_ERR_INVALID_ARG = 1,
+  SWA_ERR_UNSUPPORTED = 2,
+  SWA_ERR_CUDA = 3,
+  SWA_ERR_DEVICE_TIMEOUT = 4
+};
+
+/* Debug bits for swa_params_t.flags (0 in normal use).  FORCE_TIMEOUT makes
+ * the kernel wait on a barrier that nothing completes, so tests can check
+ * that the bounded wait ends the kernel and reports SWA_ERR_DEVICE_TIMEOUT. */
+enum { SWA_FLAG_FORCE_TIMEOUT = 1 };
+
+typedef struct swa_params {
+  int64_t B;        /* batch rows (prefill) or number of sequences (decode) */
+  int64_t T;        /* tokens per row (prefill); ignored by decode */
+  int32_t Hq;       /* query heads (32 in ZGCM-1) */
+  int32_t Hkv;      /* KV heads (8) */
+  int32_t head_dim; /* 128 */
+  int32_t window;   /* W: keys i-W+1 .. i (128) */
+  int32_t rot_dim;  /* rotated dims (42 = 0.33 * 128, even) */
+  int32_t flags;    /* SWA_FLAG_* debug bits, 0 normally */
+  double rope_base; /* 1e4; 1e7 at the 256K stage */
+  float eps;        /* RMSNorm epsilon (1e-6) */
+  float scale;      /* score scale; 0 selects 1/sqrt(head_dim) */
+} swa_params_t;
+
+/*
+ * Forward.  q, g: [B,T,Hq,D]; k, v: [B,T,Hkv,D] (bf16); wq, wk: [D] fp32.
+ * Writes o [B,T,Hq,D] bf16 and, when lse != NULL, lse [B,Hq,T] fp32, the
+ * natural-log softmax normaliser of each row's scaled scores (what swa_bwd
+ * reads).  o and lse must not overlap the inputs.
+ */
+int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+            const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+            swa_bf16_t* o, float* lse, void* stream);
+
+/*
+ * Backward of swa_fwd given the upstream gradient dO [B,T,Hq,D] and the lse
+ * that swa_fwd wrote.  Writes dq, dg [B,T,Hq,D] and dk, dv [B,T,Hkv,D]
+ * (bf16) and ADDS the weight gradients into dwq, dwk [D] (fp32; the caller
+ * zeroes them).  `workspace` is caller-owned device scratch of at least
+ * swa_bwd_workspace_size(p) bytes, 256-byte aligned; its contents on entry
+ * do not matter.  The chain rule covers the gate, the softmax, RoPE and the
+ * RMSNorm (the weights included).
+ */
+int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+            const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+            const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+            swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* workspace,
+            size_t workspace_bytes, void* stream);
+
+/* Bytes of scratch swa_bwd needs for these parameters (0 if unsupported). */
+size_t swa_bwd_workspace_size(const swa_params_t* p);
+
+/*
+ * One decode step for p->B sequences against their window caches.
+ * pos: [B] int64 device array, the position of each sequence's new token.
+ * q, g: [B,Hq,D]; k_new, v_new: [B,Hkv,D] (bf16).
+ * k_cache, v_cache: [B,Hkv,W,D] bf16 rings, updated in place: slot
+ * pos mod W receives RoPE(RMSNorm(k_new)) (rounded to bf16) and v_new
+ * (bit-exact copy); slot s holds the key of position pos - ((pos - s) mod W),
+ * ignored when that position is negative.  Writes o [B,Hq,D] bf16.
+ * Distinct sequences must not share ring memory.
+ */
+int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
+                    const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
+                    const float* wq, const float* wk, swa_bf16_t* k_cache,
+                    swa_bf16_t* v_cache, swa_bf16_t* o, void* stream);
+
+/* Static description of an error code. */
+const char* swa_error_string(int code);
+
+/*
+ * Waits for `stream`, then returns SWA_ERR_DEVICE_TIMEOUT if any kernel of
+ * this library on the current device recorded a timed-out wait since the
+ * last call (the raw site code goes to *site when site != NULL), else SWA_OK.
+ * Clears the record.  Returns SWA_ERR_CUDA if the stream itself failed.
+ */
+int swa_get_last_device_error(void* stream, int* site);
+
+/* Library version string. */
+const char* swa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

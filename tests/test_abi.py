@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every declared entry point and rejects bad
+arguments on the host (no GPU compute is needed for any of these checks)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import hybrid_sliding_window_gated_b200 as swa
+from hybrid_sliding_window_gated_b200 import build as swa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    swa_build.build()
+    return swa.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "swa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(swa_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"swa_fwd", "swa_bwd", "swa_decode_step", "swa_bwd_workspace_size"} <= set(names)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", swa.LIB_PATH], text=True)
+    exported = set(re.findall(r" T (swa_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(L, n)
+
+
+def test_error_strings_and_version(L):
+    for code in range(5):
+        assert L.swa_error_string(code)
+    assert b"sm_100a" in L.swa_version()
+
+
+def _params(**kw):
+    base = dict(B=1, T=256, Hq=4, Hkv=1)
+    base.update(kw)
+    B, T, Hq, Hkv = base.pop("B"), base.pop("T"), base.pop("Hq"), base.pop("Hkv")
+    return swa.make_params(B, T, Hq, Hkv, **base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=6, Hkv=4), swa.ERR_INVALID_ARG),         # Hq not a multiple of Hkv
+    (dict(rot_dim=41), swa.ERR_INVALID_ARG),          # odd rotary dims
+    (dict(rot_dim=256), swa.ERR_INVALID_ARG),         # more rotary dims than head dims
+    (dict(T=-1), swa.ERR_INVALID_ARG),
+    (dict(eps=-1.0), swa.ERR_INVALID_ARG),
+    (dict(head_dim=64), swa.ERR_UNSUPPORTED),         # tensor-core path is built for 128
+    (dict(window=64), swa.ERR_UNSUPPORTED),
+    (dict(rot_dim=40), swa.ERR_UNSUPPORTED),
+])
+def test_bad_shapes_rejected_before_any_launch(L, kw, code):
+    p = _params(**kw)
+    nul = ctypes.c_void_p(0)
+    assert L.swa_fwd(ctypes.byref(p), *([nul] * 9)) == code
+    assert L.swa_bwd(ctypes.byref(p), *([nul] * 15), 0, nul) == code
+    assert L.swa_bwd_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_null_pointers_rejected(L):
+    p = _params()
+    nul = ctypes.c_void_p(0)
+    assert L.swa_fwd(ctypes.byref(p), *([nul] * 9)) == swa.ERR_INVALID_ARG
+    assert L.swa_fwd(None, *([nul] * 9)) == swa.ERR_INVALID_ARG
+
+
+def test_empty_problem_is_a_no_op(L):
+    p = _params(T=0)
+    nul = ctypes.c_void_p(0)
+    assert L.swa_fwd(ctypes.byref(p), *([nul] * 9)) == swa.OK
+
+
+def test_misaligned_pointer_rejected(L):
+    p = _params()
+    good = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    args = [good] * 9
+    args[0] = bad
+    assert L.swa_fwd(ctypes.byref(p), *args) == swa.ERR_INVALID_ARG

@@ -1,0 +1,127 @@
+"""GPU forward parity: swa_fwd (through the C ABI) against the fp64 oracle.
+
+Small shapes are compared element by element on every output; the
+layer-shape and long-context configurations run at full size in the launch
+configuration the benchmark times and are compared on sampled query rows
+(several per batch row, across tile boundaries and the ragged tail), which the
+oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import hybrid_sliding_window_gated_b200 as swa
+import oracle
+import workloads
+from swa_testutil import assert_parity, to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+# lse is a smooth maximum of the scores, so its error is bounded by the score
+# error, which bf16 rounding of q' and k' (relative 2^-9 per element) keeps
+# well under 2e-2 for unit-RMS rows.
+LSE_ATOL = 2e-2
+
+
+def run_gpu(inp, cfg, want_lse=True):
+    return swa.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"],
+                   window=cfg.W, rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps,
+                   want_lse=want_lse)
+
+
+def oracle_full(inp, cfg):
+    f = lambda t: t.float().cpu().double().numpy()
+    return oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["g"]), f(inp["wq"]),
+                      f(inp["wk"]), W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+
+
+def check_full(cfg, device=DEV):
+    inp = workloads.prefill_inputs(cfg, device="cpu")
+    o_ref, lse_ref = oracle_full(inp, cfg)
+    dinp = {k: v.to(device) for k, v in inp.items()}
+    o, lse = run_gpu(dinp, cfg)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    assert_parity(to_f64(o), o_ref, "o")
+    # lse [B,Hq,T] vs oracle [B,T,Hq]
+    np.testing.assert_allclose(to_f64(lse), lse_ref.transpose(0, 2, 1), rtol=0, atol=LSE_ATOL)
+    return o, lse
+
+
+def test_tiny_config_full():
+    check_full(workloads.TINY)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", [
+    (1, 1, 4, 1), (1, 127, 4, 1), (1, 128, 4, 1), (1, 129, 4, 1), (2, 300, 8, 2),
+    (1, 520, 2, 2), (1, 700, 3, 1), (3, 257, 8, 8), (1, 1000, 32, 8),
+])
+def test_shapes_and_ragged_tails(B, T, Hq, Hkv):
+    check_full(workloads.custom_prefill(B, T, Hq, Hkv, base=1e4, g_std=2.0, seed=B * 1000 + T))
+
+
+@pytest.mark.parametrize("rot_dim", [0, 32, 48])
+def test_other_rot_dims(rot_dim):
+    check_full(workloads.custom_prefill(1, 300, 4, 2, base=1e4, seed=7, R=rot_dim))
+
+
+def test_large_rope_base_and_positions():
+    check_full(workloads.custom_prefill(1, 2000, 4, 1, base=1e7, seed=8))
+
+
+def test_saturated_gate_gives_zero_and_ungated():
+    cfg = workloads.custom_prefill(1, 300, 4, 1, seed=9)
+    inp = {k: v.to(DEV) for k, v in workloads.prefill_inputs(cfg).items()}
+    inp["g"] = torch.full_like(inp["g"], float("-inf"))
+    o = run_gpu(inp, cfg, want_lse=False)
+    assert torch.count_nonzero(o).item() == 0
+
+
+def _sampled_rows_check(cfg, chunks):
+    inp = workloads.prefill_inputs(cfg, device=DEV)
+    o, lse = run_gpu(inp, cfg)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    assert torch.isfinite(o).all()
+    host = {k: v.cpu() for k, v in inp.items()}
+    o_cpu, lse_cpu = o.cpu(), lse.cpu()
+    worst = (0.0, 0.0)
+    for b, t0, t1 in chunks:
+        ref, lref = oracle.fwd_rows(host["q"], host["k"], host["v"], host["g"], host["wq"],
+                                    host["wk"], b, t0, t1, W=cfg.W, R=cfg.R, base=cfg.base,
+                                    eps=cfg.eps)
+        got = to_f64(o_cpu[b:b + 1, t0:t1])
+        ma, fr = assert_parity(got, ref, f"o rows b={b} [{t0},{t1})")
+        worst = (max(worst[0], ma), max(worst[1], fr))
+        np.testing.assert_allclose(to_f64(lse_cpu[b:b + 1, :, t0:t1]), lref.transpose(0, 2, 1),
+                                   rtol=0, atol=LSE_ATOL)
+    return worst
+
+
+def test_layer_shape_sampled_rows():
+    cfg = workloads.LAYER
+    T = cfg.T
+    chunks = [(0, 0, 64), (1, 100, 260), (2, 2040, 2060), (3, T - 130, T), (0, T // 2, T // 2 + 40)]
+    _sampled_rows_check(cfg, chunks)
+
+
+def test_long_context_sampled_rows():
+    cfg = workloads.LONG
+    T = cfg.T
+    chunks = [(0, 0, 40), (0, 127, 200), (0, 131000, 131100), (0, 200000, 200050),
+              (0, T - 140, T)]
+    _sampled_rows_check(cfg, chunks)
+
+
+def test_forced_timeout_is_reported_and_context_survives():
+    cfg = workloads.TINY
+    inp = {k: v.to(DEV) for k, v in workloads.prefill_inputs(cfg).items()}
+    assert swa.get_last_device_error()[0] == swa.OK
+    swa.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"], rope_base=cfg.base,
+            flags=swa.FLAG_FORCE_TIMEOUT)
+    code, site = swa.get_last_device_error()
+    assert code == swa.ERR_DEVICE_TIMEOUT and site >= 0x100
+    assert swa.get_last_device_error()[0] == swa.OK  # cleared
+    check_full(cfg)  # the context is still usable and results are right
