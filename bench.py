@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the gated sliding-window attention core on B200.
+
+One step = one pass of the hot path over one batch of synthetic input held in
+HBM.  The headline line times swa_fwd on the ZGCM-1 layer-shape prefill
+workload (B=4, T=4096, 32 query / 8 KV heads, head_dim 128, window 128,
+rot_dim 42): norm, RoPE, windowed GQA attention and the gate all run inside
+the one fused kernel launch that forms the step.  Secondary workloads (the
+long-context forward, training forward+backward and the 27-layer decode step)
+are timed the same way and reported under "secondary".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl swa|reference]
+
+For N > 1 launch with torchrun: each rank runs its own batch (the batch rows
+are independent problems, so there is no data-path collective; scaling is
+weak) and the reported time is the maximum over ranks.  `--impl reference`
+times the fp64 CPU oracle on bounded samples of the same workload (rank 0
+only).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+
+def FWD_BYTES_PER_TOKEN(c):
+    """Algorithmic HBM bytes per token of the forward: read q, g, k, v; write o."""
+    return (3 * c.Hq + 2 * c.Hkv) * c.D * 2
+
+
+def BWD_BYTES_PER_TOKEN(c):
+    """Backward: read q, g, dO, k, v and lse; write dq, dg, dk, dv."""
+    return (3 * c.Hq + 2 * c.Hkv) * c.D * 2 + c.Hq * 4 + (2 * c.Hq + 2 * c.Hkv) * c.D * 2
+
+
+def band_keys(T, W):
+    """sum_i min(i+1, W) for one sequence of T tokens."""
+    full = max(T - W + 1, 0)
+    ramp = min(T, W - 1)
+    return full * W + ramp * (ramp + 1) // 2
+
+
+def fwd_flops(c):
+    return 4 * c.D * c.Hq * band_keys(c.T, c.W) * c.B
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured (MEASURED_PEAKS.json)"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback (profiling recipe)"}
+
+
+def kernel_source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "hybrid_sliding_window_gated_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(profile_name, files):
+    """dram bytes per launch from a committed ncu summary, or None if the kernel
+    sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = (s.strip() for s in line.split("=", 1))
+                vals[k] = v
+    if vals.get("kernel_sources_sha256_16") != kernel_source_digest(files):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a thread."""
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == str(uuid).replace("GPU-", ""):
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than fail
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        nv = self.nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "applications_clocks_setting": getattr(nv, "nvmlClocksEventReasonApplicationsClocksSetting", 0x2),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sync_boost": getattr(nv, "nvmlClocksEventReasonSyncBoost", 0x10),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if not inside:  # timed region shorter than one sampling period
+            inside = self.samples[-5:]
+            window = "last samples after the timed region"
+        mhz = [s[1] for s in inside]
+        active = set()
+        for s in inside:
+            for n, bit in names.items():
+                if s[2] & bit and n != "gpu_idle":
+                    active.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(active), "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------- timing
+
+def timed_loop(step_fns, steps, warmup, stream, world, sampler=None, per_launch=None):
+    """Run warmup steps, then time `steps` steps between barriers on `stream`.
+
+    step_fns: list of callables, one per rotating input set.  Returns
+    (total_ms max over ranks, per-launch mean ms of the measured kernel, t0, t1).
+    """
+    for i in range(warmup):
+        step_fns[i % len(step_fns)]()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launch_evs = []
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(steps):
+            if per_launch is not None:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                step_fns[i % len(step_fns)]()
+                b.record(stream)
+                launch_evs.append((a, b))
+            else:
+                step_fns[i % len(step_fns)]()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    per = None
+    if launch_evs:
+        per = sum(a.elapsed_time(b) for a, b in launch_evs) / len(launch_evs)
+    return ms, per, t0, t1
+
+
+# ------------------------------------------------------------- workloads
+
+def fwd_workload(swa, cfg, device, n_sets=2, lse=False):
+    sets = []
+    for s in range(n_sets):
+        inp = workloads.prefill_inputs(cfg, device=device, seed=cfg.seed + 100 * s,
+                                       with_grad_out=False)
+        inp["o"] = torch.empty_like(inp["q"])
+        inp["lse"] = torch.empty((cfg.B, cfg.Hq, cfg.T), dtype=torch.float32, device=device) \
+            if lse else None
+        sets.append(inp)
+
+    def mk(inp):
+        def step():
+            swa.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"], window=cfg.W,
+                    rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps, out=inp["o"], lse=inp["lse"])
+        return step
+    return [mk(x) for x in sets], sets
+
+
+def e2e_fwd(swa, cfg, device, steps, warmup, stream, world):
+    """Same metric through the public call with pinned host buffers: H2D of the
+    step's inputs, swa_fwd, D2H of the output, all inside the timed region."""
+    host = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=False)
+    host = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(host["q"].shape, dtype=torch.bfloat16).pin_memory()
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    o = torch.empty_like(dev["q"])
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        swa.fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["wq"], dev["wk"], window=cfg.W,
+                rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps, out=o)
+        out_host.copy_(o, non_blocking=True)
+    ms, _, _, _ = timed_loop([step], steps, warmup, stream, world)
+    return ms, h2d, d2h
+
+
+def cpu_baseline_fwd(cfg, target_s=10.0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload
+    (query rows of batch row 0 with all their heads), on this host's cores."""
+    import oracle
+    inp = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=False)
+    n = 64
+    t_first = None
+    while True:
+        t0 = time.perf_counter()
+        oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"], 0, 1024,
+                        1024 + n, W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= cfg.T - 1024:
+            break
+        n = min(cfg.T - 1024, max(2 * n, int(n * target_s / max(dt, 1e-3) * 1.1)))
+        t_first = dt
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} query tokens x {cfg.Hq} heads of batch row 0 (rows 1024..{1024 + n}) "
+                      f"of the {cfg.name} workload, fp64, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- main
+
+def run_swa(args, rank, world, device):
+    import hybrid_sliding_window_gated_b200 as swa
+    from hybrid_sliding_window_gated_b200 import build as swa_build
+    if rank == 0:
+        swa_build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    swa.lib()
+    peaks = load_peaks()
+    cfg = workloads.LAYER
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(torch.cuda.current_device())
+
+    steps_fns, _ = fwd_workload(swa, cfg, device)
+    # per-launch timing pass (events around each launch) for the roofline figure
+    _, per_launch_ms, _, _ = timed_loop(steps_fns, max(args.steps, 10), args.warmup, stream,
+                                        world, per_launch=True)
+    sampler.start()
+    ms, _, t0, t1 = timed_loop(steps_fns, args.steps, args.warmup, stream, world)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    tokens_per_rank = cfg.B * cfg.T
+    total_tokens = tokens_per_rank * world * args.steps
+    value = total_tokens / (ms / 1e3)
+    bytes_launch = FWD_BYTES_PER_TOKEN(cfg) * tokens_per_rank
+    achieved = bytes_launch / (per_launch_ms / 1e3) / 1e9
+    traffic = committed_traffic("swa_fwd_kernel_layer_shape.txt", ["fwd.cu", "ptx.cuh"])
+
+    e2e_ms, h2d, d2h = e2e_fwd(swa, cfg, device, max(3, min(args.steps, 10)), 2, stream, world)
+    e2e_value = tokens_per_rank * world / (e2e_ms / max(3, min(args.steps, 10)) / 1e3)
+
+    line = {
+        "metric": "gated-SWA forward tokens/s (layer-shape prefill)",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded randn, ZGCM-1 layer shapes)",
+        "config": {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                   "head_dim": cfg.D, "window": cfg.W, "rot_dim": cfg.R, "rope_base": cfg.base,
+                   "parallelism": f"independent batches x{world}",
+                   "l2": "two rotating input sets of 470 MB each (> 126 MB L2)"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": traffic, "kernel": "swa_fwd_kernel",
+                     "algorithmic_bytes_per_launch": bytes_launch,
+                     "launch_ms": round(per_launch_ms, 5),
+                     "peak_source": peaks["source"] + ", hbm_gbs (burst copy)"},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if not args.no_secondary:
+        line["secondary"] = secondary(swa, args, world, device, stream, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_fwd(cfg)
+    return line
+
+
+def secondary(swa, args, world, device, stream, peaks):
+    out = {}
+    cfg = workloads.LONG
+    fns, sets = fwd_workload(swa, cfg, device, n_sets=1)
+    steps = max(3, min(args.steps, 10))
+    ms, per, _, _ = timed_loop(fns, steps, 2, stream, world, per_launch=True)
+    b = FWD_BYTES_PER_TOKEN(cfg) * cfg.B * cfg.T
+    out["long_context_fwd"] = {
+        "workload": cfg.name, "tokens_per_s": round(cfg.B * cfg.T * world / (ms / steps / 1e3), 1),
+        "ms_per_step": round(ms / steps, 4),
+        "achieved_GBps": round(b / (per / 1e3) / 1e9, 1),
+        "frac_of_measured_hbm": round(b / (per / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "l2": "7.5 GB per step (> L2)"}
+    del fns, sets
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_profile(args, device):
+    """Warmup + steps launches of swa_fwd on the layer-shape workload, nothing
+    else, so that a profiler sees a short, predictable launch list."""
+    import hybrid_sliding_window_gated_b200 as swa
+    cfg = workloads.LAYER
+    fns, _ = fwd_workload(swa, cfg, device)
+    for i in range(args.warmup + args.steps):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    code, site = swa.get_last_device_error()
+    return {"profile": cfg.name, "launches": args.warmup + args.steps, "device_error": code}
+
+
+def run_reference(args, rank, world):
+    """The fp64 oracle on bounded samples, as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    cfg = workloads.LAYER
+    inp = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=False)
+    n = 128  # query tokens (x 32 heads) per step
+
+    def step(i):
+        t0 = 1024 + (i * n) % (cfg.T - 1024 - n)
+        oracle.fwd_rows(inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"], i % cfg.B,
+                        t0, t0 + n, W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    return {
+        "metric": "gated-SWA forward tokens/s (layer-shape prefill)", "impl": "reference",
+        "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded randn, ZGCM-1 layer shapes)",
+        "config": {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                   "head_dim": cfg.D, "window": cfg.W, "rot_dim": cfg.R, "rope_base": cfg.base,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": oracle.threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} query tokens x {cfg.Hq} heads per step of the "
+                                   f"{cfg.name} workload, fp64"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only warmup + steps launches of the headline kernel (for ncu)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=device)
+    if args.profile:
+        line = run_profile(args, device)
+    else:
+        line = run_swa(args, rank, world, device)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

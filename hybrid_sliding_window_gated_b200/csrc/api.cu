@@ -176,14 +176,18 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
   if (rc != SWA_OK) return rc;
   fill_inv_freq(p, a.inv_freq);
 
-  CUtensorMap tq, tk, tv, tg;
+  // Every tensor moves in boxes of 128 rows x 64 dims (128-byte rows, 128B
+  // swizzle): the MMA operand layout for q, k, v, and the same layout for the
+  // gate and output tiles that pass through a Q slot.
+  CUtensorMap tq, tk, tv, tg, to;
   const uint64_t D = kHeadDim, T = p->T, B = p->B;
   if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 128, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_NONE)))
+      (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&to, o, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
-  return launch_fwd(p, tq, tk, tv, tg, a, static_cast<cudaStream_t>(stream));
+  return launch_fwd(p, tq, tk, tv, tg, to, a, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

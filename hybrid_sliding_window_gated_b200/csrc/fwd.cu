@@ -1,7 +1,7 @@
 // fwd.cu -- fused prefill forward of the gated sliding-window attention core
-// for sm_100a: TMA loads, QK-RMSNorm and partial RoPE in shared memory,
-// tcgen05 QK^T and PV with TMEM accumulators, single-pass softmax over the
-// 256-key band, and the sigmoid-gate epilogue.
+// for sm_100a: TMA loads and stores, QK-RMSNorm and partial RoPE in shared
+// memory, tcgen05 QK^T and PV with TMEM accumulators, single-pass softmax over
+// the 256-key band, and the sigmoid-gate epilogue.
 //
 // Definition (ZGCM-1 pages: onedev.kr summary, "어떻게 동작하나"; jaehun.me
 // review, "How Gated SWA Behaves"): for query token i and head h,
@@ -16,19 +16,52 @@
 // rotated once per range and shared by the G = Hq/Hkv query heads of its
 // group and by two query tiles.
 //
-// Roles (512 threads):
-//   warp 0      TMA producer (one lane)
+// Roles (384 threads, three warpgroups; registers rebalanced with setmaxnreg):
+//   warp 0      K/V producer (lane 0 issues TMA; all lanes compute each K
+//               tile's rotation table)
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one lane)
-//   warps 4-7   "transform": RMSNorm + RoPE of Q and K rows, in place in the
-//               128-byte-swizzled tiles, one row per thread
-//   warps 8-11  softmax + epilogue for TMEM region 0 (even head slots)
-//   warps 12-15 softmax + epilogue for TMEM region 1 (odd head slots)
+//   warps 4-7   region 0 (even head slots), warps 8-11 region 1 (odd).  For
+//               each of its heads a region warpgroup normalises and rotates
+//               the Q rows (and the K rows of a tile whose first head it owns)
+//               in place in the 128-byte-swizzled tiles, runs the softmax, and
+//               finally the epilogue: it copies O out of TMEM (freeing the
+//               region for the next QK^T) and writes o = O/l * sigmoid(g).
+//               One thread per row throughout, so 1/rms(q) and 1/l stay in
+//               registers.
+//
+// Q slot reuse.  Region r owns Q slot r.  Once QK^T(n) has read Q(n), the slot
+// receives the gate tile g(n) by TMA (it lands while the softmax runs); the
+// epilogue overwrites it in place with o(n), which leaves by TMA store; then
+// Q(n+2) is loaded into the slot.  All bulk global traffic (q, k, v, g in; o
+// out) thus moves by TMA: the load/store unit touches only shared memory,
+// since a row-per-thread pattern on global memory touches 32 cache lines per
+// warp instruction.
 //
 // TMEM (512 columns) holds two regions of 256 columns.  For a head in region
 // r: S = Q [K_{t-1} K_t]^T fills all 256 columns (fp32); the softmax writes P
 // as packed bf16 over the first 128 columns; PV accumulates O (fp32) into the
 // last 128 columns; the epilogue reads O.  Regions alternate between heads so
 // the tensor core works on one head while the softmax runs on the other.
+//
+// Scores without the q norm.  s = scale * q'.k' with q' = RoPE(q/rms(q) * wq).
+// The MMA multiplies q'' = [RoPE(q * wq) on the rotated dims; raw q elsewhere]
+// by k'' = [RoPE(k/rms(k) * wk); k/rms(k) * wk * wq elsewhere] (wq folded into
+// the unrotated dims of K, where it commutes), and the softmax applies the
+// per-row factor 1/rms(q).  So Q rows only need their sum of squares and the
+// rotation of the first rot_dim dims.
+//
+// Softmax without a max pass.  After RMSNorm every row has sum(xhat^2) <= D,
+// so |q'| <= sqrt(D) max|wq| and |k'| <= sqrt(D) max|wk| (RoPE keeps norms),
+// hence every score s <= M = scale * D * max|wq| * max|wk|.  exp2((s - M) log2e)
+// then never overflows, and it cannot underflow while 2 M log2e <= 120 (the
+// smallest possible score is -M); softmax is invariant to the subtracted
+// constant, so the result equals the max-subtracted form.  Weights outside
+// that range fall back to an exact two-pass (row max first) softmax.
+//
+// Rotation angles.  Position p = 128 j + 16 a + b: the rotation by p w is the
+// product of a per-tile table rot((128 j + 16 a) w), a in 0..7, computed by the
+// producer's lanes for each K tile (fp64 range reduction, then sincosf), and a
+// per-CTA table rot(b w), b in 0..15.
 #include "ptx.cuh"
 #include "swa_internal.h"
 
@@ -36,7 +69,14 @@ namespace swa {
 
 namespace fwd {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
+// Launch budget is 384 x 168 registers; the split below sums to at most that.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 56;   // producer + MMA warpgroup
+constexpr int kRegsRegion = 224;   // each region warpgroup
+static_assert(kRegsControl + 2 * kRegsRegion <= 3 * kRegsLaunch,
+              "register split exceeds the launch budget");
+
 constexpr int kHalfBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = 16 KiB (one TMA box)
 constexpr int kTileBytes = 2 * kHalfBytes;  // a full 128 x 128 bf16 tile
 
@@ -44,56 +84,74 @@ struct alignas(1024) Smem {
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
   uint8_t q[2][kTileBytes];
-  float2 cs[kMaxPairs * kTile];  // per-row (cos, sin), laid out [pair][row]
+  float2 rot_lo[kMaxPairs][16];        // rot(b * w_p), b = 0..15
+  float2 rot_hi[2][kMaxPairs][8];      // rot((128 j + 16 a) * w_p) per K slot
   float wq[kHeadDim];
   float wk[kHeadDim];
+  float wkq[kHeadDim];    // wk * wq, for the K dims that RoPE leaves alone
   uint64_t kfull[2], kready[2], kempty[2];
   uint64_t vfull[2], vempty[2];
-  uint64_t qfull[2], qready[2], qempty[2];
+  uint64_t qfull[2], qready[2];
   uint64_t sfull[2], pfull[2], ofull[2], tfree[2];
-  uint64_t drain, never;
+  uint64_t gfull[2], ostore[2];  // gate tile landed / o written, per region
+  uint64_t tables, drain, never;
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory over the 227 KiB per-CTA limit");
 
 // Wait-site ids reported through the device error word.
 enum Site {
-  kSiteKEmpty = 1, kSiteVEmpty, kSiteQEmpty, kSiteKFull, kSiteQFull, kSiteKReady,
-  kSiteQReady, kSiteTFree, kSiteVFull, kSitePFull, kSiteSFull, kSiteOFull, kSiteForced
+  kSiteKEmpty = 1, kSiteVEmpty, kSiteOStore, kSiteKFull, kSiteQFull, kSiteKReady,
+  kSiteQReady, kSiteTFree, kSiteVFull, kSitePFull, kSiteSFull, kSiteOFull, kSiteForced,
+  kSiteTables, kSiteGFull
 };
 
-struct Tile {
-  int b, kvh, t;
-  bool has_prev;   // key tile t-1 exists (t > 0)
-  bool need_prev;  // ... and must be loaded here (first tile of a segment)
-  bool seg_last;   // last tile of this CTA's run on the chain
+// Position inside a CTA's contiguous run of tiles, advanced without division.
+struct Cursor {
+  int b, kvh, t;  // chain (batch row, KV head) and tile index in the chain
+  int h;          // query head within the GQA group
+  int u;          // tiles advanced since the start of the run
 };
 
-__device__ __forceinline__ Tile tile_at(const FwdArgs& a, long long u, long long u0,
-                                        long long u1) {
-  Tile x;
-  long long chain = u / a.tiles_per_chain;
-  x.t = static_cast<int>(u - chain * a.tiles_per_chain);
-  x.b = static_cast<int>(chain / a.Hkv);
-  x.kvh = static_cast<int>(chain - static_cast<long long>(x.b) * a.Hkv);
-  x.has_prev = x.t > 0;
-  x.need_prev = x.has_prev && (u == u0);
-  x.seg_last = (u == u1 - 1) || (x.t == a.tiles_per_chain - 1);
-  return x;
+__device__ __forceinline__ Cursor cursor_at(const FwdArgs& a, int u0) {
+  Cursor c;
+  const int chain = u0 / a.tiles_per_chain;
+  c.t = u0 - chain * a.tiles_per_chain;
+  c.b = chain / a.Hkv;
+  c.kvh = chain - c.b * a.Hkv;
+  c.h = 0;
+  c.u = 0;
+  return c;
+}
+__device__ __forceinline__ void next_tile(Cursor& c, const FwdArgs& a) {
+  ++c.u;
+  if (++c.t == a.tiles_per_chain) {
+    c.t = 0;
+    if (++c.kvh == a.Hkv) {
+      c.kvh = 0;
+      ++c.b;
+    }
+  }
+}
+__device__ __forceinline__ void next_head(Cursor& c, const FwdArgs& a) {
+  if (++c.h == a.G) {
+    c.h = 0;
+    next_tile(c, a);
+  }
+}
+// Key tile t-1 exists / must be loaded at this tile (first tile of a run).
+__device__ __forceinline__ bool has_prev(const Cursor& c) { return c.t > 0; }
+__device__ __forceinline__ bool need_prev(const Cursor& c) { return c.t > 0 && c.u == 0; }
+// Last tile of the run on its chain: its K/V tile is released after use.
+__device__ __forceinline__ bool seg_last(const Cursor& c, const FwdArgs& a, int n_tiles) {
+  return c.u == n_tiles - 1 || c.t == a.tiles_per_chain - 1;
 }
 
-// Offset of element d of row `row` inside a tile stored as two 128B-swizzled
-// halves (the layout TMA SWIZZLE_128B writes): 16-byte chunk c of a 128-byte
-// row lands at chunk c ^ (row & 7).
+// Offset of 16-byte chunk `chunk16` of row `row` inside one 128B-swizzled
+// half tile (the layout TMA SWIZZLE_128B writes): chunk c lands at c ^ (row & 7).
 __device__ __forceinline__ uint32_t sw_off(int row, int chunk16) {
   return static_cast<uint32_t>(row * 128 + ((chunk16 ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ void unpack8(const uint4& u, float* x) {
-  x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x);
-  x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
-  x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z);
-  x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
 }
 
 __device__ __forceinline__ uint4 pack8(const float* x) {
@@ -105,70 +163,119 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
   return u;
 }
 
-// Fill this thread's (cos, sin) row for tile j (position j*128 + row).
-template <int kPairs>
-__device__ __forceinline__ void fill_cos_sin(Smem& sm, const FwdArgs& a, int j, int row) {
-  const double pos = static_cast<double>(j) * kTile + row;
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) {
+  return make_float2(bf16_lo(u), bf16_hi(u));
+}
+
+__device__ __forceinline__ float2 cmul(float2 x, float2 y) {
+  return make_float2(x.x * y.x - x.y * y.y, x.x * y.y + x.y * y.x);
+}
+
+// Rotation (cos, sin) of position 128 j + row for pair p, from the tables.
+__device__ __forceinline__ float2 rot_at(const Smem& sm, int kslot, int p, int row) {
+  return cmul(sm.rot_hi[kslot][p][row >> 4], sm.rot_lo[p][row & 15]);
+}
+
+// Sum of squares of a 128-element bf16 row held in two swizzled halves.
+__device__ __forceinline__ float row_sumsq(const uint8_t* h0, const uint8_t* h1, int row) {
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};  // independent chains for ILP
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 x = *reinterpret_cast<const uint4*>(h0 + sw_off(row, c));
+    const uint4 y = *reinterpret_cast<const uint4*>(h1 + sw_off(row, c));
+    const uint32_t w[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = bf16x2_to_f2(w[i]);
+      acc[i & 3] = __ffma2_rn(f, f, acc[i & 3]);
+    }
+  }
+  const float2 s2 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return s2.x + s2.y;
+}
+
+// Rotate the first 2*kPairs dims of a row in place: y = R(x * scale * wr),
+// rotate-half pairs (p, p + kPairs).  Dims of the rotated chunks beyond
+// 2*kPairs are multiplied by scale * wo, or left as they are (kKeepOthers).
+template <int kPairs, bool kKeepOthers>
+__device__ __forceinline__ void rope_chunks(uint8_t* h0, int row, float scale, const float* wr,
+                                            const float* wo, const Smem& sm, int kslot) {
+  constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
+  float x[kRopeChunks * 8];
+#pragma unroll
+  for (int c = 0; c < kRopeChunks; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(h0 + sw_off(row, c));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * c + 2 * e] = bf16_lo(w4[e]);
+      x[8 * c + 2 * e + 1] = bf16_hi(w4[e]);
+    }
+  }
+#pragma unroll
+  for (int d = 2 * kPairs; d < kRopeChunks * 8; ++d)
+    if (!kKeepOthers) x[d] = x[d] * scale * wo[d];
 #pragma unroll
   for (int p = 0; p < kPairs; ++p) {
-    float c, s;
-    rope_cos_sin(pos, a.inv_freq[p], &c, &s);
-    sm.cs[p * kTile + row] = make_float2(c, s);
+    const float2 t = rot_at(sm, kslot, p, row);
+    const float u = x[p] * scale * wr[p];
+    const float v = x[p + kPairs] * scale * wr[p + kPairs];
+    x[p] = u * t.x - v * t.y;            // x_p cos - x_{p+P} sin
+    x[p + kPairs] = v * t.x + u * t.y;   // x_{p+P} cos + x_p sin
+  }
+#pragma unroll
+  for (int c = 0; c < kRopeChunks; ++c)
+    *reinterpret_cast<uint4*>(h0 + sw_off(row, c)) = pack8(x + 8 * c);
+}
+
+// Scale dims [8*c0, 128) of a row in place by scale * w[d] (f32x2 math).
+__device__ __forceinline__ void scale_chunks(uint8_t* h0, uint8_t* h1, int row, int c0,
+                                             float scale, const float* w) {
+  const float2 sc = make_float2(scale, scale);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    if (c < c0) continue;
+    uint8_t* p = (c < 8 ? h0 : h1) + sw_off(row, c & 7);
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const float4 wa = *reinterpret_cast<const float4*>(w + 8 * c);
+    const float4 wb = *reinterpret_cast<const float4*>(w + 8 * c + 4);
+    const float2 y0 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.x), make_float2(wa.x, wa.y)), sc);
+    const float2 y1 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.y), make_float2(wa.z, wa.w)), sc);
+    const float2 y2 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.z), make_float2(wb.x, wb.y)), sc);
+    const float2 y3 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.w), make_float2(wb.z, wb.w)), sc);
+    uint4 o;
+    o.x = pack_bf16x2(y0.x, y0.y);
+    o.y = pack_bf16x2(y1.x, y1.y);
+    o.z = pack_bf16x2(y2.x, y2.y);
+    o.w = pack_bf16x2(y3.x, y3.y);
+    *reinterpret_cast<uint4*>(p) = o;
   }
 }
 
-// RMSNorm (weight w) and partial RoPE of row `row` of a tile, in place.
+// K row: k'' = [RoPE(k / rms(k) * wk) on the rotated dims; k / rms(k) * wk * wq
+// elsewhere].
 template <int kPairs>
-__device__ __forceinline__ void transform_row(uint8_t* tile, int row, const float* w,
-                                              const float2* cs, float eps) {
+__device__ __forceinline__ void transform_k_row(uint8_t* tile, int row, const Smem& sm, int kslot,
+                                                float eps) {
   uint8_t* h0 = tile;
   uint8_t* h1 = tile + kHalfBytes;
-  float ss = 0.f;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    float x[8], y[8];
-    unpack8(*reinterpret_cast<const uint4*>(h0 + sw_off(row, c)), x);
-    unpack8(*reinterpret_cast<const uint4*>(h1 + sw_off(row, c)), y);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], fmaf(y[i], y[i], ss));
-  }
-  const float rinv = rsqrtf(ss * (1.0f / kHeadDim) + eps);
-
+  const float rinv = rsqrtf(row_sumsq(h0, h1, row) * (1.0f / kHeadDim) + eps);
   constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
-  if constexpr (kRopeChunks > 0) {
-    float x[kRopeChunks * 8];
-#pragma unroll
-    for (int c = 0; c < kRopeChunks; ++c)
-      unpack8(*reinterpret_cast<const uint4*>(h0 + sw_off(row, c)), x + 8 * c);
-#pragma unroll
-    for (int d = 0; d < kRopeChunks * 8; ++d) x[d] = x[d] * rinv * w[d];
-#pragma unroll
-    for (int p = 0; p < kPairs; ++p) {
-      const float2 t = cs[p * kTile + row];
-      const float u = x[p], v = x[p + kPairs];
-      x[p] = u * t.x - v * t.y;
-      x[p + kPairs] = v * t.x + u * t.y;
-    }
-#pragma unroll
-    for (int c = 0; c < kRopeChunks; ++c)
-      *reinterpret_cast<uint4*>(h0 + sw_off(row, c)) = pack8(x + 8 * c);
-  }
-#pragma unroll
-  for (int c = kRopeChunks; c < 8; ++c) {
-    float x[8];
-    unpack8(*reinterpret_cast<const uint4*>(h0 + sw_off(row, c)), x);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = x[i] * rinv * w[8 * c + i];
-    *reinterpret_cast<uint4*>(h0 + sw_off(row, c)) = pack8(x);
-  }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    float x[8];
-    unpack8(*reinterpret_cast<const uint4*>(h1 + sw_off(row, c)), x);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = x[i] * rinv * w[64 + 8 * c + i];
-    *reinterpret_cast<uint4*>(h1 + sw_off(row, c)) = pack8(x);
-  }
+  if constexpr (kRopeChunks > 0)
+    rope_chunks<kPairs, false>(h0, row, rinv, sm.wk, sm.wkq, sm, kslot);
+  scale_chunks(h0, h1, row, kRopeChunks, rinv, sm.wkq);
+}
+
+// Q row: q'' = [RoPE(q * wq) on the rotated dims; q unchanged elsewhere].
+// Returns 1/rms(q), which the softmax applies to the scores.
+template <int kPairs>
+__device__ __forceinline__ float transform_q_row(uint8_t* tile, int row, const Smem& sm,
+                                                 int kslot, float eps) {
+  const float rinv = rsqrtf(row_sumsq(tile, tile + kHalfBytes, row) * (1.0f / kHeadDim) + eps);
+  constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
+  if constexpr (kRopeChunks > 0) rope_chunks<kPairs, true>(tile, row, 1.0f, sm.wq, sm.wq, sm, kslot);
+  return rinv;
 }
 
 // K-major operand descriptor for k-step kk (16 elements) of a 128 x 128 tile.
@@ -183,11 +290,23 @@ __device__ __forceinline__ uint64_t desc_v(const uint8_t* tile, int kk) {
 constexpr uint32_t kIdescQK = make_idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 128, false, true);
 
+// Phase bookkeeping for a 2-slot ring: bit s of `par` is the parity of the
+// next use of slot s; bit s of `used` says whether slot s was used before.
+struct Ring {
+  uint32_t par = 0, used = 0;
+  __device__ __forceinline__ uint32_t parity(int s) const { return (par >> s) & 1u; }
+  __device__ __forceinline__ bool was_used(int s) const { return (used >> s) & 1u; }
+  __device__ __forceinline__ void advance(int s) {
+    par ^= 1u << s;
+    used |= 1u << s;
+  }
+};
+
 template <int kPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const FwdArgs a) {
+                   const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~static_cast<uintptr_t>(1023));
@@ -195,29 +314,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  const long long u0 = a.total_tiles * blockIdx.x / gridDim.x;
-  const long long u1 = a.total_tiles * (blockIdx.x + 1) / gridDim.x;
-  const long long n_heads = (u1 - u0) * a.G;
+  const int u0 = static_cast<int>(a.total_tiles * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
+  const int n_tiles = u1 - u0;
+  const int n_heads = n_tiles * a.G;
 
   if (tid < kHeadDim) {
-    sm.wq[tid] = a.wq[tid];
-    sm.wk[tid] = a.wk[tid];
+    const float wq = a.wq[tid], wk = a.wk[tid];
+    sm.wq[tid] = wq;
+    sm.wk[tid] = wk;
+    sm.wkq[tid] = wk * wq;
   }
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.kfull[i], 1);
+      mbar_init(&sm.kfull[i], 2);  // the copy's expect_tx arrive + the rotation table
       mbar_init(&sm.kready[i], 128);
       mbar_init(&sm.kempty[i], 1);
       mbar_init(&sm.vfull[i], 1);
       mbar_init(&sm.vempty[i], 1);
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qready[i], 128);
-      mbar_init(&sm.qempty[i], 1);
       mbar_init(&sm.sfull[i], 1);
       mbar_init(&sm.pfull[i], 128);
       mbar_init(&sm.ofull[i], 1);
       mbar_init(&sm.tfree[i], 128);
+      mbar_init(&sm.gfull[i], 1);
+      mbar_init(&sm.ostore[i], 128);
     }
+    mbar_init(&sm.tables, 128);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.never, 1);
     sm.abort = 0;
@@ -228,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_g);
+    prefetch_tensormap(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -239,138 +364,127 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t nk[2] = {0, 0}, nv[2] = {0, 0}, nq[2] = {0, 0};
+  if (warp < 4) {
+    regs_dec<kRegsControl>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      Ring kr, vr;
       bool ok = true;
-      auto load_kv = [&](const CUtensorMap* map, uint8_t (*buf)[kTileBytes], uint64_t* full,
-                         uint64_t* empty, uint32_t* cnt, int j, const Tile& x, int site) {
+      auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+        return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+      };
+      auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {
         const int s = j & 1;
-        if (cnt[s] > 0 && !mbar_wait(&empty[s], (cnt[s] - 1) & 1, abort, a.err, site)) return false;
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
-        tma_load_4d(buf[s], map, &full[s], 0, x.kvh, j * kTile, x.b);
-        tma_load_4d(buf[s] + kHalfBytes, map, &full[s], 64, x.kvh, j * kTile, x.b);
-        ++cnt[s];
+        Ring& ring = is_k ? kr : vr;
+        uint64_t* full = is_k ? &sm.kfull[s] : &sm.vfull[s];
+        uint64_t* empty = is_k ? &sm.kempty[s] : &sm.vempty[s];
+        if (ring.was_used(s) && !wait0(empty, ring.parity(s) ^ 1u, is_k ? kSiteKEmpty : kSiteVEmpty))
+          return false;
+        if (lane == 0) {
+          uint8_t* dst = is_k ? sm.k[s] : sm.v[s];
+          const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+          mbar_arrive_expect_tx(full, kTileBytes);
+          tma_load_4d(dst, map, full, 0, c.kvh, j * kTile, c.b);
+          tma_load_4d(dst + kHalfBytes, map, full, 64, c.kvh, j * kTile, c.b);
+        }
+        if (is_k) {
+          // rot((128 j + 16 a) w_p) for this tile, then the second arrive on kfull.
+          for (int e = lane; e < kPairs * 8; e += 32) {
+            const int p = e >> 3, ai = e & 7;
+            float cv, sv;
+            rope_cos_sin(static_cast<double>(j) * kTile + 16.0 * ai, a.inv_freq[p], &cv, &sv);
+            sm.rot_hi[s][p][ai] = make_float2(cv, sv);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full);
+        }
+        ring.advance(s);
         return true;
       };
-      long long n = 0;  // head slots issued so far; Q slot = n & 1
-      for (long long u = u0; u < u1 && ok; ++u) {
-        const Tile x = tile_at(a, u, u0, u1);
-        if (x.need_prev) {
-          ok = ok && load_kv(&tm_k, sm.k, sm.kfull, sm.kempty, nk, x.t - 1, x, kSiteKEmpty);
-          ok = ok && load_kv(&tm_v, sm.v, sm.vfull, sm.vempty, nv, x.t - 1, x, kSiteVEmpty);
-        }
-        ok = ok && load_kv(&tm_k, sm.k, sm.kfull, sm.kempty, nk, x.t, x, kSiteKEmpty);
-        for (int h = 0; h < a.G && ok; ++h) {
-          const int s = static_cast<int>(n & 1);
-          if (nq[s] > 0 && !mbar_wait(&sm.qempty[s], (nq[s] - 1) & 1, abort, a.err, kSiteQEmpty)) {
-            ok = false;
-            break;
-          }
-          const int hq = x.kvh * a.G + h;
-          mbar_arrive_expect_tx(&sm.qfull[s], kTileBytes);
-          tma_load_4d(sm.q[s], &tm_q, &sm.qfull[s], 0, hq, x.t * kTile, x.b);
-          tma_load_4d(sm.q[s] + kHalfBytes, &tm_q, &sm.qfull[s], 64, hq, x.t * kTile, x.b);
-          tma_prefetch_4d(&tm_g, 0, hq, x.t * kTile, x.b);
-          ++nq[s];
-          ++n;
-          if (h == 0) ok = load_kv(&tm_v, sm.v, sm.vfull, sm.vempty, nv, x.t, x, kSiteVEmpty);
-        }
+      Cursor c = cursor_at(a, u0);
+      for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+        if (need_prev(c))  // first tile of a run: key tile t-1 as well
+          ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
+        ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
       }
-      if (!ok) {
-        // Drain the loads this thread issued before the CTA releases its memory.
+      if (!ok && lane == 0) {
+        // Drain the loads this warp issued before the CTA releases its memory.
         for (int s = 0; s < 2; ++s) {
-          if (nk[s]) mbar_wait_drain(&sm.kfull[s], (nk[s] - 1) & 1);
-          if (nv[s]) mbar_wait_drain(&sm.vfull[s], (nv[s] - 1) & 1);
-          if (nq[s]) mbar_wait_drain(&sm.qfull[s], (nq[s] - 1) & 1);
+          if (kr.was_used(s)) mbar_wait_drain(&sm.kfull[s], kr.parity(s) ^ 1u);
+          if (vr.was_used(s)) mbar_wait_drain(&sm.vfull[s], vr.parity(s) ^ 1u);
         }
       }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      uint32_t nkr[2] = {0, 0}, nvr[2] = {0, 0};
+    } else if (warp == 1 && lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      Ring kr, vr;  // readiness of K (after the transform) and V slots
       bool ok = true;
       if (a.flags & SWA_FLAG_FORCE_TIMEOUT) ok = mbar_wait(&sm.never, 0, abort, a.err, kSiteForced);
-
-      auto do_qk = [&](long long n) -> bool {
-        const long long u = u0 + n / a.G;
-        const int h = static_cast<int>(n % a.G);
-        const Tile x = tile_at(a, u, u0, u1);
-        const int sp = (x.t + 1) & 1, sc = x.t & 1;
-        if (h == 0) {
-          if (x.need_prev) {
-            if (!mbar_wait(&sm.kready[sp], nkr[sp] & 1, abort, a.err, kSiteKReady)) return false;
-            ++nkr[sp];
+      Cursor cq = cursor_at(a, u0), cp = cq;
+      for (int n = 0; n < n_heads && ok; n += 2) {
+        // QK^T for heads n and n+1, then PV for both (regions n&1 alternate).
+        for (int i = 0; i < 2 && n + i < n_heads && ok; ++i, next_head(cq, a)) {
+          const int m = n + i, r = m & 1;
+          const uint32_t cnt = static_cast<uint32_t>(m >> 1);
+          const int sp = (cq.t + 1) & 1, sc = cq.t & 1;
+          if (cq.h == 0) {
+            if (need_prev(cq)) {
+              if (!mbar_wait(&sm.kready[sp], kr.parity(sp), abort, a.err, kSiteKReady)) { ok = false; break; }
+              kr.advance(sp);
+            }
+            if (!mbar_wait(&sm.kready[sc], kr.parity(sc), abort, a.err, kSiteKReady)) { ok = false; break; }
+            kr.advance(sc);
           }
-          if (!mbar_wait(&sm.kready[sc], nkr[sc] & 1, abort, a.err, kSiteKReady)) return false;
-          ++nkr[sc];
-        }
-        const int r = static_cast<int>(n & 1);
-        const uint32_t c = static_cast<uint32_t>(n >> 1);
-        if (!mbar_wait(&sm.qready[r], c & 1, abort, a.err, kSiteQReady)) return false;
-        if (c > 0 && !mbar_wait(&sm.tfree[r], (c - 1) & 1, abort, a.err, kSiteTFree)) return false;
-        tc_fence_after();
-        const uint32_t s_base = tmem + r * 256;
-        for (int blk = x.has_prev ? 0 : 1; blk < 2; ++blk) {
-          const uint8_t* kt = sm.k[blk == 0 ? sp : sc];
+          if (!mbar_wait(&sm.qready[r], cnt & 1, abort, a.err, kSiteQReady)) { ok = false; break; }
+          if (cnt > 0 && !mbar_wait(&sm.tfree[r], (cnt - 1) & 1, abort, a.err, kSiteTFree)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t s_base = tmem + r * 256;
+          const bool hp = has_prev(cq);
+          for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+            const uint8_t* kt = sm.k[blk == 0 ? sp : sc];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(s_base + blk * 128, desc_kmajor(sm.q[r], kk), desc_kmajor(kt, kk), kIdescQK,
-                   kk > 0);
-        }
-        mma_commit(&sm.sfull[r]);
-        mma_commit(&sm.qempty[r]);
-        if (h == a.G - 1) {
-          if (x.has_prev) mma_commit(&sm.kempty[sp]);
-          if (x.seg_last) mma_commit(&sm.kempty[sc]);
-        }
-        return true;
-      };
-
-      auto do_pv = [&](long long n) -> bool {
-        const long long u = u0 + n / a.G;
-        const int h = static_cast<int>(n % a.G);
-        const Tile x = tile_at(a, u, u0, u1);
-        const int sp = (x.t + 1) & 1, sc = x.t & 1;
-        if (h == 0) {
-          if (x.need_prev) {
-            if (!mbar_wait(&sm.vfull[sp], nvr[sp] & 1, abort, a.err, kSiteVFull)) return false;
-            ++nvr[sp];
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(s_base + blk * 128, desc_kmajor(sm.q[r], kk), desc_kmajor(kt, kk), kIdescQK,
+                     kk > 0);
           }
-          if (!mbar_wait(&sm.vfull[sc], nvr[sc] & 1, abort, a.err, kSiteVFull)) return false;
-          ++nvr[sc];
+          mma_commit(&sm.sfull[r]);
+          if (cq.h == a.G - 1) {
+            if (hp) mma_commit(&sm.kempty[sp]);
+            if (seg_last(cq, a, n_tiles)) mma_commit(&sm.kempty[sc]);
+          }
         }
-        const int r = static_cast<int>(n & 1);
-        const uint32_t c = static_cast<uint32_t>(n >> 1);
-        if (!mbar_wait(&sm.pfull[r], c & 1, abort, a.err, kSitePFull)) return false;
-        tc_fence_after();
-        const uint32_t p_base = tmem + r * 256;
-        const uint32_t o_base = p_base + 128;
-        bool first = true;
-        for (int blk = x.has_prev ? 0 : 1; blk < 2; ++blk) {
-          const uint8_t* vt = sm.v[blk == 0 ? sp : sc];
+        for (int i = 0; i < 2 && n + i < n_heads && ok; ++i, next_head(cp, a)) {
+          const int m = n + i, r = m & 1;
+          const uint32_t cnt = static_cast<uint32_t>(m >> 1);
+          const int sp = (cp.t + 1) & 1, sc = cp.t & 1;
+          if (cp.h == 0) {
+            if (need_prev(cp)) {
+              if (!mbar_wait(&sm.vfull[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
+              vr.advance(sp);
+            }
+            if (!mbar_wait(&sm.vfull[sc], vr.parity(sc), abort, a.err, kSiteVFull)) { ok = false; break; }
+            vr.advance(sc);
+          }
+          if (!mbar_wait(&sm.pfull[r], cnt & 1, abort, a.err, kSitePFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t p_base = tmem + r * 256;
+          const bool hp = has_prev(cp);
+          uint32_t acc = 0;
+          for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+            const uint8_t* vt = sm.v[blk == 0 ? sp : sc];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_ts(o_base, p_base + blk * 64 + kk * 8, desc_v(vt, kk), kIdescPV, first ? 0u : 1u);
-            first = false;
+            for (int kk = 0; kk < 8; ++kk) {
+              mma_ts(p_base + 128, p_base + blk * 64 + kk * 8, desc_v(vt, kk), kIdescPV, acc);
+              acc = 1;
+            }
+          }
+          mma_commit(&sm.ofull[r]);
+          if (cp.h == a.G - 1) {
+            if (hp) mma_commit(&sm.vempty[sp]);
+            if (seg_last(cp, a, n_tiles)) mma_commit(&sm.vempty[sc]);
           }
         }
-        mma_commit(&sm.ofull[r]);
-        if (h == a.G - 1) {
-          if (x.has_prev) mma_commit(&sm.vempty[sp]);
-          if (x.seg_last) mma_commit(&sm.vempty[sc]);
-        }
-        return true;
-      };
-
-      for (long long n = 0; n < n_heads && ok; n += 2) {
-        ok = do_qk(n);
-        if (ok && n + 1 < n_heads) ok = do_qk(n + 1);
-        if (ok) ok = do_pv(n);
-        if (ok && n + 1 < n_heads) ok = do_pv(n + 1);
       }
       if (!ok) {
         // No tcgen05.mma may still be running when TMEM is released.
@@ -379,172 +493,266 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------------------------------------------------- transform
-    const int row = tid - 128;
-    uint32_t nk[2] = {0, 0};
-    long long n = 0;
-    bool ok = true;
-    auto do_k = [&](int j) -> bool {
-      const int s = j & 1;
-      if (!mbar_wait(&sm.kfull[s], nk[s] & 1, abort, a.err, kSiteKFull)) return false;
-      fill_cos_sin<kPairs>(sm, a, j, row);
-      transform_row<kPairs>(sm.k[s], row, sm.wk, sm.cs, a.eps);
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.kready[s]);
-      ++nk[s];
+  } else {
+    // --------------------------------------------------------------- region
+    // Warpgroup r serves TMEM region r: heads n = r, r+2, ...  Per head:
+    // softmax S(n) once QK^T(n) is done, then the transform T(n+2) of the
+    // next Q (overlapping PV(n)), then the epilogue E(n).
+    regs_inc<kRegsRegion>();
+    const int r = (warp - 4) >> 2;
+    const int wq4 = warp & 3;  // TMEM lane quarter
+    const int row = wq4 * 32 + lane;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16) + r * 256;
+    // rot(b w_p), b = 0..15, filled once by warpgroup 0.
+    if (r == 0) {
+      for (int e = row; e < kPairs * 16; e += 128) {
+        const int p = e >> 4, bi = e & 15;
+        float cv, sv;
+        rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
+        sm.rot_lo[p][bi] = make_float2(cv, sv);
+      }
+      mbar_arrive(&sm.tables);
+    }
+    const float sl2 = a.scale_log2;
+    float wmq = 0.f, wmk = 0.f;
+    for (int d = 0; d < kHeadDim; ++d) {
+      wmq = fmaxf(wmq, fabsf(sm.wq[d]));
+      wmk = fmaxf(wmk, fabsf(sm.wk[d]));
+    }
+    // Score bound in log2 units, with a 1/64 margin for the bf16 rounding of q', k'.
+    const float bound = sl2 * kHeadDim * wmq * wmk * (1.0f + 1.0f / 64.0f);
+    const bool exact = !(2.0f * bound <= 120.0f);
+    bool ok = mbar_wait(&sm.tables, 0, abort, a.err, kSiteTables);
+
+    // K loads are accounted in order by both warpgroups (the same sequence the
+    // producer issues); the warpgroup that owns the first head of a tile
+    // transforms that tile's K loads, right before its Q.
+    Ring kr;
+    int acct = 0;  // tiles accounted so far
+    Cursor kc = cursor_at(a, u0);
+    auto account = [&](int upto, bool transform_last) -> bool {
+      while (acct <= upto) {
+        for (int j = need_prev(kc) ? kc.t - 1 : kc.t; j <= kc.t; ++j) {
+          const int s = j & 1;
+          if (transform_last && acct == upto) {
+            if (!mbar_wait(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
+            transform_k_row<kPairs>(sm.k[s], row, sm, s, a.eps);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.kready[s]);
+          } else if (acct == upto && j == kc.t) {
+            // The Q rows of this tile use its rotation table, which the
+            // producer publishes with kfull.  The slot cannot be refilled
+            // before every QK^T of tile t+1, which waits for this warpgroup,
+            // so the phase seen here is the current one.
+            if (!mbar_wait(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
+          }
+          kr.advance(s);
+        }
+        next_tile(kc, a);
+        ++acct;
+      }
       return true;
     };
-    for (long long u = u0; u < u1 && ok; ++u) {
-      const Tile x = tile_at(a, u, u0, u1);
-      if (x.need_prev) ok = do_k(x.t - 1);
-      if (ok) ok = do_k(x.t);  // leaves the cos/sin rows of tile t for the Q heads
-      for (int h = 0; h < a.G && ok; ++h, ++n) {
-        const int s = static_cast<int>(n & 1);
-        if (!mbar_wait(&sm.qfull[s], static_cast<uint32_t>(n >> 1) & 1, abort, a.err, kSiteQFull)) {
-          ok = false;
-          break;
-        }
-        transform_row<kPairs>(sm.q[s], row, sm.wq, sm.cs, a.eps);
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.qready[s]);
-      }
-    }
-  } else if (warp >= 8) {
-    // ------------------------------------------------ softmax + epilogue
-    const int r = (warp - 8) >> 2;  // TMEM region served by this warpgroup
-    const int wq4 = warp & 3;       // TMEM lane quarter
-    const int row = wq4 * 32 + lane;
-    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16);
-    const uint32_t s_cols = t_row + r * 256;
-    const float sl2 = a.scale_log2;
-    bool ok = true;
-    for (long long n = r; n < n_heads && ok; n += 2) {
-      const long long u = u0 + n / a.G;
-      const int h = static_cast<int>(n % a.G);
-      const Tile x = tile_at(a, u, u0, u1);
-      const uint32_t c = static_cast<uint32_t>(n >> 1);
-      const int hq = x.kvh * a.G + h;
-      const long long pos = static_cast<long long>(x.t) * kTile + row;
-      const bool valid = pos < a.T;
-      const long long elem = ((static_cast<long long>(x.b) * a.T + (valid ? pos : 0)) * a.Hq + hq) *
-                             kHeadDim;
-      const uint4* gp = reinterpret_cast<const uint4*>(a.g + elem);
+    // Row 0 of the warpgroup issues the warpgroup's own copies: Q(n) and g(n)
+    // into Q slot r, o(n) out of it.
+    const bool elected = row == 0;
+    int q_issued = 0, g_issued = 0;  // copies issued by this thread, for the drain
+    auto issue_q = [&](const Cursor& cn) {
+      const int hq = cn.kvh * a.G + cn.h;
+      mbar_arrive_expect_tx(&sm.qfull[r], kTileBytes);
+      tma_load_4d(sm.q[r], &tm_q, &sm.qfull[r], 0, hq, cn.t * kTile, cn.b);
+      tma_load_4d(sm.q[r] + kHalfBytes, &tm_q, &sm.qfull[r], 64, hq, cn.t * kTile, cn.b);
+      tma_prefetch_4d(&tm_g, 0, hq, cn.t * kTile, cn.b);  // warm L2 for the gate tile
+      tma_prefetch_4d(&tm_g, 64, hq, cn.t * kTile, cn.b);
+      ++q_issued;
+    };
 
-      if (!mbar_wait(&sm.sfull[r], c & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
+    Cursor c = cursor_at(a, u0);
+    if (r == 1) next_head(c, a);
+    if (elected && r < n_heads) issue_q(c);
+    for (int n = r; n < n_heads && ok; n += 2) {
+      const uint32_t cnt = static_cast<uint32_t>(n >> 1);
+      const int hq = c.kvh * a.G + c.h;
+      const long long pos = static_cast<long long>(c.t) * kTile + row;
+
+      // ---- transform T(n): the K tiles of a tile whose first head this is,
+      // then Q(n).  rot_hi of slot t&1 stays valid until K_{t+2} is loaded,
+      // after every QK^T of tile t+1.
+      if (!account(c.u, c.h == 0)) { ok = false; break; }
+      if (!mbar_wait(&sm.qfull[r], cnt & 1, abort, a.err, kSiteQFull)) { ok = false; break; }
+      const float rinv = transform_q_row<kPairs>(sm.q[r], row, sm, c.t & 1, a.eps);
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.qready[r]);
+
+      // ---- softmax S(n)
+      if (!mbar_wait(&sm.sfull[r], cnt & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
-
-      // Pass 1: row maximum over the band.  Key tile t-1 contributes columns
-      // c > row, key tile t columns c <= row; 32-column chunks entirely
-      // outside the band are skipped.
-      float m = -INFINITY;
-      uint32_t v[32];
-      if (x.has_prev) {
-        for (int ch = wq4; ch < 4; ++ch) {
-          tmem_ld32(s_cols + ch * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i > row) m = fmaxf(m, __uint_as_float(v[i]));
-        }
+      if (elected) {  // QK^T(n) has read Q(n): the slot takes the gate tile now
+        mbar_arrive_expect_tx(&sm.gfull[r], kTileBytes);
+        tma_load_4d(sm.q[r], &tm_g, &sm.gfull[r], 0, hq, c.t * kTile, c.b);
+        tma_load_4d(sm.q[r] + kHalfBytes, &tm_g, &sm.gfull[r], 64, hq, c.t * kTile, c.b);
+        ++g_issued;
       }
-      for (int ch = 0; ch <= wq4; ++ch) {
-        tmem_ld32(s_cols + 128 + ch * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (ch * 32 + i <= row) m = fmaxf(m, __uint_as_float(v[i]));
-      }
-      const float ms = m * sl2;
-
-      // Pass 2: P = exp2(s*scale*log2e - max), packed bf16 over the first 128
-      // columns of the region; row sum in fp32.
-      float l = 0.f;
-      uint32_t pk[16];
-      if (x.has_prev) {
-        for (int ch = 0; ch < 4; ++ch) {
-          if (ch < wq4) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = 0u;
-          } else {
-            tmem_ld32(s_cols + ch * 32, v);
+      // The MMA saw unnormalised q rows; 1/rms(q) enters with the softmax scale.
+      const float rs = sl2 * rinv;
+      const bool hp = has_prev(c);
+      float ms = bound;
+      if (exact) {
+        // Row maximum over the band: key tile t-1 gives columns c > row, key
+        // tile t columns c <= row; pieces entirely outside the band are skipped.
+        float m = -INFINITY;
+        for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+          for (int pc = 0; pc < 4; ++pc) {
+            const bool none = blk == 0 ? (pc < wq4) : (pc > wq4);
+            if (none) continue;
+            uint32_t v[32];
+            tmem_ld32(t_row + blk * 128 + pc * 32, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = (ch * 32 + 2 * i > row)
-                                   ? ex2_approx(fmaf(__uint_as_float(v[2 * i]), sl2, -ms)) : 0.f;
-              const float p1 = (ch * 32 + 2 * i + 1 > row)
-                                   ? ex2_approx(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -ms)) : 0.f;
-              l += p0 + p1;
-              pk[i] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 32; ++i) {
+              const bool in = blk == 0 ? (pc * 32 + i > row) : (pc * 32 + i <= row);
+              if (in) m = fmaxf(m, __uint_as_float(v[i]));
             }
           }
-          tmem_st16(s_cols + ch * 16, pk);
         }
+        ms = m * rs;
       }
-      for (int ch = 0; ch < 4; ++ch) {
-        if (ch > wq4) {
+      // P = exp2(s * rs - ms), packed bf16 over the first 128 columns of the
+      // region; fp32 row sum.  Key tile t-1 (columns 0..127) keeps columns
+      // c > row, key tile t (128..255) columns c <= row.  For this warp's 32
+      // rows, 32-column chunk pc of key tile t-1 is empty for pc < wq4 and
+      // full for pc > wq4; of key tile t full for pc < wq4 and empty for
+      // pc > wq4; only pc == wq4 straddles the band edge.
+      const int na = hp ? 4 - wq4 : 0;  // chunks of key tile t-1 in the band
+      const int nch = na + wq4 + 1;     // plus those of key tile t
+      float2 l2 = make_float2(0.f, 0.f);
+      const float2 rs2 = make_float2(rs, rs), nms2 = make_float2(-ms, -ms);
+      {
+        uint32_t v[2][32];
+        tmem_ld32(t_row + (na > 0 ? wq4 * 32 : 128), v[0]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = 0u;
-        } else {
-          tmem_ld32(s_cols + 128 + ch * 32, v);
-          tmem_wait_ld();
+        for (int i = 0; i < 5; ++i) {
+          if (i < nch) {
+            const int blk = i < na ? 0 : 1;
+            const int pc = blk == 0 ? wq4 + i : i - na;
+            tmem_wait_ld();
+            if (i + 1 < nch) {  // next chunk's load overlaps this one's math
+              const int blk1 = i + 1 < na ? 0 : 1;
+              const int pc1 = blk1 == 0 ? wq4 + i + 1 : i + 1 - na;
+              tmem_ld32(t_row + blk1 * 128 + pc1 * 32, v[(i + 1) & 1]);
+            }
+            const uint32_t(&x)[32] = v[i & 1];
+            uint32_t pk[16];
+            if (pc != wq4) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = (ch * 32 + 2 * i <= row)
-                                 ? ex2_approx(fmaf(__uint_as_float(v[2 * i]), sl2, -ms)) : 0.f;
-            const float p1 = (ch * 32 + 2 * i + 1 <= row)
-                                 ? ex2_approx(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -ms)) : 0.f;
-            l += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+              for (int e = 0; e < 16; ++e) {
+                const float2 z = __ffma2_rn(
+                    make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
+                const float2 p = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+                l2 = __fadd2_rn(l2, p);
+                pk[e] = pack_bf16x2(p.x, p.y);
+              }
+            } else {  // the diagonal chunk: mask per column
+              const int c0 = pc * 32;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int cc = c0 + 2 * e;
+                const bool in0 = blk == 0 ? (cc > row) : (cc <= row);
+                const bool in1 = blk == 0 ? (cc + 1 > row) : (cc + 1 <= row);
+                const float2 z = __ffma2_rn(
+                    make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
+                const float2 p =
+                    make_float2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
+                l2 = __fadd2_rn(l2, p);
+                pk[e] = pack_bf16x2(p.x, p.y);
+              }
+            }
+            tmem_st16(t_row + blk * 64 + pc * 16, pk);
           }
         }
-        tmem_st16(s_cols + 64 + ch * 16, pk);
       }
+      {
+        // Zero the empty chunks last: P columns alias S columns that the
+        // chunks above still had to read.
+        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        for (int pc = 0; pc < 4; ++pc) {
+          if (hp && pc < wq4) tmem_st16(t_row + pc * 16, zero16);
+          if (pc > wq4) tmem_st16(t_row + 64 + pc * 16, zero16);
+        }
+      }
+      const float l = l2.x + l2.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.pfull[r]);
-
-      if (a.lse != nullptr && valid)
-        a.lse[(static_cast<long long>(x.b) * a.Hq + hq) * a.T + pos] =
+      if (a.lse != nullptr && pos < a.T)
+        a.lse[(static_cast<long long>(c.b) * a.Hq + hq) * a.T + pos] =
             (ms + __log2f(l)) * 0.6931471805599453f;
-      const float inv_l = 1.0f / l;
 
-      // Epilogue: O / l * sigmoid(g), bf16, 16-byte stores of this row.
-      uint4 gv[4];
-      if (valid) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) gv[i] = __ldg(gp + i);
-      }
-      if (!mbar_wait(&sm.ofull[r], c & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
+      // ---- epilogue E(n): o = A/l * sigmoid(g) = (A * l^-1/2) * (1 + tanh(g/2)),
+      // written over g(n) in Q slot r, 32 columns per step.
+      if (!mbar_wait(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
+      if (!mbar_wait(&sm.gfull[r], cnt & 1, abort, a.err, kSiteGFull)) { ok = false; break; }
       tc_fence_after();
-      uint4* op = reinterpret_cast<uint4*>(a.o + elem);
-      for (int ch = 0; ch < 4; ++ch) {
-        tmem_ld32(s_cols + 128 + ch * 32, v);
-        tmem_wait_ld();
-        if (ch == 3) {
-          tc_fence_before();
-          mbar_arrive(&sm.tfree[r]);
-        }
-        uint4 gn[4];
-        if (valid && ch < 3) {
+      const float2 hl2 = make_float2(0.5f / l, 0.5f / l);
+      {
+        uint32_t ov[2][32];
+        tmem_ld32(t_row + 128, ov[0]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) gn[i] = __ldg(gp + 4 * (ch + 1) + i);
-        }
-        if (valid) {
+        for (int ch = 0; ch < kHeadDim / 32; ++ch) {
+          tmem_wait_ld();
+          if (ch + 1 < kHeadDim / 32) {
+            tmem_ld32(t_row + 128 + (ch + 1) * 32, ov[(ch + 1) & 1]);
+          } else {
+            tc_fence_before();
+            mbar_arrive(&sm.tfree[r]);  // region r may take the next QK^T now
+          }
+          uint8_t* half = sm.q[r] + (ch >> 1) * kHalfBytes;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float gf[8], of[8];
-            unpack8(gv[i], gf);
+          for (int i = 0; i < 4; ++i) {  // four 16-byte pieces of this chunk
+            uint4* gp = reinterpret_cast<uint4*>(half + sw_off(row, (ch & 1) * 4 + i));
+            const uint4 gv = *gp;
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t ow[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              of[e] = __uint_as_float(v[8 * i + e]) * inv_l * sigmoid_fast(gf[e]);
-            __stcs(op + 4 * ch + i, pack8(of));
+            for (int e = 0; e < 4; ++e) {
+              const float2 t =
+                  tanh2_f16(__fmul2_rn(bf16x2_to_f2(gw[e]), make_float2(0.5f, 0.5f)));
+              const float2 acc = __fmul2_rn(make_float2(__uint_as_float(ov[ch & 1][8 * i + 2 * e]),
+                                                        __uint_as_float(ov[ch & 1][8 * i + 2 * e + 1])),
+                                            hl2);
+              const float2 o2 = __ffma2_rn(acc, t, acc);
+              ow[e] = pack_bf16x2(o2.x, o2.y);
+            }
+            *gp = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) gv[i] = gn[i];
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.ostore[r]);
+
+      Cursor cn = c;
+      next_head(cn, a);
+      next_head(cn, a);
+      if (elected) {
+        // o(n) out of the slot (rows past T are clipped by the copy), then
+        // Q(n+2) in once the store has read it.
+        if (!mbar_wait(&sm.ostore[r], cnt & 1, abort, a.err, kSiteOStore)) { ok = false; break; }
+        tma_store_4d(&tm_o, sm.q[r], 0, hq, c.t * kTile, c.b);
+        tma_store_4d(&tm_o, sm.q[r] + kHalfBytes, 64, hq, c.t * kTile, c.b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        if (n + 2 < n_heads) issue_q(cn);
+      }
+      c = cn;
+    }
+    if (elected) {
+      if (!ok) {
+        // Drain this thread's loads before the CTA releases its memory.
+        if (q_issued > 0) mbar_wait_drain(&sm.qfull[r], static_cast<uint32_t>(q_issued - 1) & 1);
+        if (g_issued > 0) mbar_wait_drain(&sm.gfull[r], static_cast<uint32_t>(g_issued - 1) & 1);
+      }
+      bulk_wait_all();  // every store complete before the CTA exits
     }
   }
 
@@ -558,37 +766,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int kPairs>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& tg, const FwdArgs& a, int num_sms, cudaStream_t stream) {
+                const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
+                cudaStream_t stream) {
   const size_t smem = sizeof(Smem) + 1024;
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(swa_fwd_kernel<kPairs>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    // The register split (setmaxnreg) assumes the kernel was built with the
+    // full launch budget per thread; refuse to launch otherwise.
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, swa_fwd_kernel<kPairs>);
+    if (e != cudaSuccess) return map_cuda_error(e);
+    if (attr.numRegs != kRegsLaunch) return SWA_ERR_UNSUPPORTED;
+    e = cudaFuncSetAttribute(swa_fwd_kernel<kPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
     if (e != cudaSuccess) return map_cuda_error(e);
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
   swa_fwd_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, tg,
-                                                                                 a);
+                                                                                 to, a);
   return map_cuda_error(cudaGetLastError());
 }
 
 }  // namespace fwd
 
 int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tg, const FwdArgs& a,
-               cudaStream_t stream) {
+               const CUtensorMap& tv, const CUtensorMap& tg, const CUtensorMap& to,
+               const FwdArgs& a, cudaStream_t stream) {
   DeviceInfo di;
   int rc = current_device_info(&di);
   if (rc != SWA_OK) return rc;
+  if (a.total_tiles > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
   switch (p->rot_dim) {
-    case 0: return fwd::launch_impl<0>(tq, tk, tv, tg, a, di.num_sms, stream);
-    case 32: return fwd::launch_impl<16>(tq, tk, tv, tg, a, di.num_sms, stream);
-    case 42: return fwd::launch_impl<21>(tq, tk, tv, tg, a, di.num_sms, stream);
-    case 48: return fwd::launch_impl<24>(tq, tk, tv, tg, a, di.num_sms, stream);
+    case 0: return fwd::launch_impl<0>(tq, tk, tv, tg, to, a, di.num_sms, stream);
+    case 32: return fwd::launch_impl<16>(tq, tk, tv, tg, to, a, di.num_sms, stream);
+    case 42: return fwd::launch_impl<21>(tq, tk, tv, tg, to, a, di.num_sms, stream);
+    case 48: return fwd::launch_impl<24>(tq, tk, tv, tg, to, a, di.num_sms, stream);
     default: return SWA_ERR_UNSUPPORTED;
   }
 }

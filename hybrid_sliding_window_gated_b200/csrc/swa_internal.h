@@ -43,8 +43,8 @@ int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                    CUtensorMapSwizzle swizzle);
 
 int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tg, const FwdArgs& a,
-               cudaStream_t stream);
+               const CUtensorMap& tv, const CUtensorMap& tg, const CUtensorMap& to,
+               const FwdArgs& a, cudaStream_t stream);
 
 int map_cuda_error(cudaError_t e);
 
