@@ -373,7 +373,43 @@ def secondary(swa, args, world, device, stream, peaks):
         "l2": "7.5 GB per step (> L2)"}
     del fns, sets
     torch.cuda.empty_cache()
+    out["decode_step"] = decode_bench(swa, args, world, device, stream, peaks)
     return out
+
+
+def DECODE_BYTES_PER_SEQ_LAYER(c):
+    """Algorithmic HBM bytes of one (sequence, layer) decode: the W-1 older ring
+    slots of K and V, the new k and v, their slot writes, and q, g, o."""
+    kv_row = c.Hkv * c.D * 2
+    return (c.W - 1) * kv_row * 2 + 2 * kv_row + 2 * kv_row + 3 * c.Hq * c.D * 2
+
+
+def decode_bench(swa, args, world, device, stream, peaks):
+    """A decode step of the whole model's window layers: one swa_decode_step per
+    layer, each over its own [N, Hkv, 128, 128] K and V rings (3.5 GB > L2)."""
+    cfg = workloads.DECODE
+    layers = [workloads.decode_layer_inputs(cfg, l, device=device) for l in range(cfg.layers)]
+    outs = [torch.empty_like(x["q"]) for x in layers]
+
+    def step():
+        for x, o in zip(layers, outs):
+            swa.decode_step(x["pos"], x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"],
+                            x["k_cache"], x["v_cache"], rot_dim=cfg.R, rope_base=cfg.base,
+                            eps=cfg.eps, out=o)
+    steps = max(5, min(args.steps, 20))
+    ms, per, _, _ = timed_loop([step], steps, 3, stream, world, per_launch=True)
+    b = DECODE_BYTES_PER_SEQ_LAYER(cfg) * cfg.N * cfg.layers
+    res = {"workload": cfg.name,
+           "tokens_per_s": round(cfg.N * world / (ms / steps / 1e3), 1),
+           "ms_per_step": round(ms / steps, 4),
+           "algorithmic_bytes_per_step": b,
+           "achieved_GBps": round(b / (per / 1e3) / 1e9, 1),
+           "frac_of_measured_hbm": round(b / (per / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+           "launches_per_step": cfg.layers,
+           "note": "positions fixed across steps: each step rewrites the same ring slots"}
+    del layers, outs
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_profile(args, device):

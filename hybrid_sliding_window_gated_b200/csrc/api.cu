@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "decode_internal.h"
 #include "swa_internal.h"
 
 namespace swa {
@@ -142,7 +143,7 @@ int swa_get_last_device_error(void* stream, int* site) {
   const int zero = 0;
   if (cudaMemcpy(word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return SWA_ERR_CUDA;
-  return SWA_ERR_DEVICE_TIMEOUT;
+  return v == kDevErrBadPosition ? SWA_ERR_INVALID_ARG : SWA_ERR_DEVICE_TIMEOUT;
 }
 
 int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
@@ -200,10 +201,6 @@ int swa_bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k
                  swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* workspace,
                  size_t workspace_bytes, cudaStream_t stream);
 size_t swa_bwd_workspace_bytes(const swa_params_t* p);
-int swa_decode_impl(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
-                    const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
-                    const float* wq, const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
-                    swa_bf16_t* o, cudaStream_t stream);
 }  // namespace swa
 
 extern "C" {
@@ -229,8 +226,47 @@ int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t*
                     swa_bf16_t* o, void* stream) {
   int rc = check_params(p, true);
   if (rc != SWA_OK) return rc;
-  return swa_decode_impl(p, pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, o,
-                         static_cast<cudaStream_t>(stream));
+  if (p->Hq / p->Hkv > kDecMaxGroup) return SWA_ERR_UNSUPPORTED;
+  if (p->B == 0) return SWA_OK;
+  if (!pos || !q || !k_new || !v_new || !g || !wq || !wk || !k_cache || !v_cache || !o)
+    return SWA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) || !aligned16(q) || !aligned16(k_new) ||
+      !aligned16(v_new) || !aligned16(g) || !aligned16(wq) || !aligned16(wk) ||
+      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+    return SWA_ERR_INVALID_ARG;
+
+  DecArgs a{};
+  a.N = static_cast<int>(p->B);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.half_rot = p->rot_dim / 2;
+  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.pos = pos;
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.g = g;
+  a.wq = wq;
+  a.wk = wk;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.o = o;
+  rc = device_error_word(&a.err);
+  if (rc != SWA_OK) return rc;
+  fill_inv_freq(p, a.inv_freq);
+
+  // Each (sequence, KV head) ring [W, D] arrives as two 128-slot x 64-dim
+  // boxes with 128B swizzle.
+  CUtensorMap tk, tv;
+  const uint64_t D = kHeadDim, W = kWindow, N = p->B;
+  if ((rc = encode_tmap_4d(&tk, k_cache, D, W, p->Hkv, N, 64, kWindow, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tv, v_cache, D, W, p->Hkv, N, 64, kWindow, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  return launch_decode(tk, tv, a, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

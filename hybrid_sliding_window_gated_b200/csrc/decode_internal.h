@@ -1,0 +1,34 @@
+// decode_internal.h -- arguments of the decode-step kernel (host and device).
+#pragma once
+#include "swa_internal.h"
+
+namespace swa {
+
+constexpr int kDecMaxGroup = 8;  // query heads per KV head the decode kernel takes
+
+struct DecArgs {
+  int N, Hq, Hkv, G;
+  int half_rot;      // rot_dim / 2 rotated pairs
+  float scale_log2;  // softmax scale * log2(e)
+  float eps;
+  const int64_t* pos;
+  const uint16_t* q;      // [N, Hq, D]
+  const uint16_t* k_new;  // [N, Hkv, D]
+  const uint16_t* v_new;  // [N, Hkv, D]
+  const uint16_t* g;      // [N, Hq, D]
+  const float* wq;
+  const float* wk;
+  uint16_t* k_cache;  // [N, Hkv, W, D]
+  uint16_t* v_cache;
+  uint16_t* o;        // [N, Hq, D]
+  int* err;
+  double inv_freq[kMaxPairs];
+};
+
+// Device error codes beyond the wait timeouts: a decode position below 0.
+constexpr int kDevErrBadPosition = 0x200;
+
+int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a,
+                  cudaStream_t stream);
+
+}  // namespace swa

@@ -9,9 +9,4 @@ int swa_bwd_impl(const swa_params_t*, const swa_bf16_t*, const swa_bf16_t*, cons
   return SWA_ERR_UNSUPPORTED;
 }
 size_t swa_bwd_workspace_bytes(const swa_params_t*) { return 0; }
-int swa_decode_impl(const swa_params_t*, const int64_t*, const swa_bf16_t*, const swa_bf16_t*,
-                    const swa_bf16_t*, const swa_bf16_t*, const float*, const float*, swa_bf16_t*,
-                    swa_bf16_t*, swa_bf16_t*, cudaStream_t) {
-  return SWA_ERR_UNSUPPORTED;
-}
 }  // namespace swa

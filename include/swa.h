@@ -44,7 +44,9 @@
  *     SWA_ERR_CUDA (a CUDA runtime call failed, e.g. the launch); the kernels
  *     bound every internal wait and, when one runs out, record the site in a
  *     sticky device word that swa_get_last_device_error() returns as
- *     SWA_ERR_DEVICE_TIMEOUT.
+ *     SWA_ERR_DEVICE_TIMEOUT.  Arguments that live in device memory (decode
+ *     positions) are checked by the kernel, which records a bad one in the same
+ *     word, returned as SWA_ERR_INVALID_ARG.
  */
 #ifndef SWA_H_
 #define SWA_H_
@@ -115,13 +117,18 @@ size_t swa_bwd_workspace_size(const swa_params_t* p);
 
 /*
  * One decode step for p->B sequences against their window caches.
- * pos: [B] int64 device array, the position of each sequence's new token.
- * q, g: [B,Hq,D]; k_new, v_new: [B,Hkv,D] (bf16).
+ * pos: [B] int64 device array (8-byte aligned), the position of each
+ * sequence's new token, >= 0 (a negative one leaves that sequence's o and ring
+ * untouched and is reported by swa_get_last_device_error as
+ * SWA_ERR_INVALID_ARG).  q, g: [B,Hq,D]; k_new, v_new: [B,Hkv,D] (bf16).
  * k_cache, v_cache: [B,Hkv,W,D] bf16 rings, updated in place: slot
  * pos mod W receives RoPE(RMSNorm(k_new)) (rounded to bf16) and v_new
  * (bit-exact copy); slot s holds the key of position pos - ((pos - s) mod W),
  * ignored when that position is negative.  Writes o [B,Hq,D] bf16.
- * Distinct sequences must not share ring memory.
+ * Distinct sequences must not share ring memory.  Hq / Hkv <= 8 (else
+ * SWA_ERR_UNSUPPORTED).  Source: the window layers keep only their last W
+ * tokens (jaehun.me review, "Why the KV Cache Shrinks by 6.4x"); decoding is
+ * memory-bandwidth bound (onedev.kr summary, "어떻게 동작하나").
  */
 int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
                     const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,

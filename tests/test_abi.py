@@ -87,3 +87,21 @@ def test_misaligned_pointer_rejected(L):
     args = [good] * 9
     args[0] = bad
     assert L.swa_fwd(ctypes.byref(p), *args) == swa.ERR_INVALID_ARG
+
+
+def test_decode_host_checks(L):
+    nul = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(1 << 20)
+    # more than 8 query heads per KV head: the decode kernel's row budget
+    assert L.swa_decode_step(ctypes.byref(_params(Hq=16, Hkv=1)), *([good] * 11)) == \
+        swa.ERR_UNSUPPORTED
+    assert L.swa_decode_step(ctypes.byref(_params(window=64)), *([good] * 11)) == \
+        swa.ERR_UNSUPPORTED
+    assert L.swa_decode_step(ctypes.byref(_params()), *([nul] * 11)) == swa.ERR_INVALID_ARG
+    assert L.swa_decode_step(ctypes.byref(_params(B=0)), *([nul] * 11)) == swa.OK
+    args = [good] * 11
+    args[0] = ctypes.c_void_p((1 << 20) + 4)  # positions must be 8-byte aligned
+    assert L.swa_decode_step(ctypes.byref(_params()), *args) == swa.ERR_INVALID_ARG
+    args = [good] * 11
+    args[7] = ctypes.c_void_p((1 << 20) + 8)  # ring must be 16-byte aligned
+    assert L.swa_decode_step(ctypes.byref(_params()), *args) == swa.ERR_INVALID_ARG

@@ -1,0 +1,128 @@
+"""GPU parity of the decode step (swa_decode_step through the C ABI) against
+the fp64 oracle: attention output within the bf16 tolerances, ring writes
+bit-exact (slot index, the untouched slots, the V slot) and the K slot equal
+to the oracle's bf16-rounded k' up to one rounding step."""
+import numpy as np
+import pytest
+import torch
+
+import hybrid_sliding_window_gated_b200 as swa
+import oracle
+import workloads
+from swa_testutil import assert_parity, to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def bits(t):
+    return t.detach().cpu().view(torch.int16).numpy().astype(np.uint16)
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def run_both(inp, R, base, eps=1e-6):
+    """Decode on the GPU (copies of the rings) and in the oracle."""
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    kc, vc = d["k_cache"].clone(), d["v_cache"].clone()
+    o = swa.decode_step(d["pos"], d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], kc, vc,
+                        rot_dim=R, rope_base=base, eps=eps)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    o_ref, kc_ref, vc_ref = oracle.decode(
+        inp["pos"].numpy(), f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+        f64(inp["wq"]), f64(inp["wk"]), bits(inp["k_cache"]), bits(inp["v_cache"]), R=R,
+        base=base, eps=eps)
+    return o, kc, vc, o_ref, kc_ref, vc_ref
+
+
+def check_rings(pos, kc_in, vc_in, kc, vc, kc_ref, vc_ref):
+    kc_in, vc_in, kc, vc = bits(kc_in), bits(vc_in), bits(kc), bits(vc)
+    W = kc.shape[2]
+    for n, p in enumerate(pos.tolist()):
+        s = p % W
+        others = [i for i in range(W) if i != s]
+        assert np.array_equal(kc[n][:, others], kc_in[n][:, others]), f"seq {n}: K slots touched"
+        assert np.array_equal(vc[n][:, others], vc_in[n][:, others]), f"seq {n}: V slots touched"
+        assert np.array_equal(vc[n][:, s], vc_ref[n][:, s]), f"seq {n}: V slot is not v_new"
+        # k' computed in fp32 vs fp64 may round to the neighbouring bf16 value
+        got = oracle.bf16_bits_to_f64(kc[n][:, s])
+        ref = oracle.bf16_bits_to_f64(kc_ref[n][:, s])
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-30), f"seq {n}: K slot"
+        assert np.mean(kc[n][:, s] == kc_ref[n][:, s]) > 0.95
+
+
+def test_decode_config_one_layer():
+    cfg = workloads.DECODE
+    inp = workloads.decode_layer_inputs(cfg, layer=0)
+    o, kc, vc, o_ref, kc_ref, vc_ref = run_both(inp, cfg.R, cfg.base)
+    assert_parity(to_f64(o), o_ref, "decode o")
+    check_rings(inp["pos"], inp["k_cache"], inp["v_cache"], kc, vc, kc_ref, vc_ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv,R", [(4, 1, 42), (8, 8, 42), (16, 2, 42), (8, 2, 0), (8, 2, 32),
+                                      (8, 2, 48)])
+def test_decode_group_sizes_and_rot_dims(Hq, Hkv, R):
+    cfg = workloads.Decode("decode test", N=7, layers=1, Hq=Hq, Hkv=Hkv, base=1e4, seed=11, R=R)
+    inp = workloads.decode_layer_inputs(cfg, layer=3)
+    inp["pos"] = torch.tensor([0, 1, 64, 126, 127, 128, 262143], dtype=torch.int64)
+    o, kc, vc, o_ref, kc_ref, vc_ref = run_both(inp, R, cfg.base)
+    assert_parity(to_f64(o), o_ref, f"decode o {Hq}/{Hkv} R={R}")
+    check_rings(inp["pos"], inp["k_cache"], inp["v_cache"], kc, vc, kc_ref, vc_ref)
+
+
+def test_sequential_decode_reproduces_prefill():
+    """Decoding tokens 0..T-1 one by one, starting from rings full of garbage,
+    gives the prefill rows: the ring keeps exactly the last 128 tokens."""
+    cfg = workloads.custom_prefill(2, 300, 8, 2, base=1e4, g_std=1.0, seed=21)
+    inp = workloads.prefill_inputs(cfg)
+    o_ref, _ = oracle.fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                          f64(inp["wq"]), f64(inp["wk"]), W=cfg.W, R=cfg.R, base=cfg.base,
+                          eps=cfg.eps)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    kc = (torch.randn((2, 2, 128, 128), generator=gen) * 50).to(torch.bfloat16).to(DEV)
+    vc = (torch.randn((2, 2, 128, 128), generator=gen) * 50).to(torch.bfloat16).to(DEV)
+    outs = []
+    for t in range(cfg.T):
+        pos = torch.full((2,), t, dtype=torch.int64, device=DEV)
+        outs.append(swa.decode_step(pos, d["q"][:, t].contiguous(), d["k"][:, t].contiguous(),
+                                    d["v"][:, t].contiguous(), d["g"][:, t].contiguous(), d["wq"],
+                                    d["wk"], kc, vc, rot_dim=cfg.R, rope_base=cfg.base))
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    o = torch.stack(outs, dim=1)
+    assert_parity(to_f64(o), o_ref, "sequential decode vs prefill")
+
+
+def test_negative_position_is_reported_and_skipped():
+    cfg = workloads.Decode("decode test", N=3, layers=1, Hq=8, Hkv=2, base=1e4, seed=12)
+    inp = workloads.decode_layer_inputs(cfg, layer=0)
+    inp["pos"] = torch.tensor([300, -1, 7], dtype=torch.int64)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    kc, vc = d["k_cache"].clone(), d["v_cache"].clone()
+    o = torch.full_like(d["q"], 3.0)
+    swa.decode_step(d["pos"], d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], kc, vc,
+                    rope_base=cfg.base, out=o)
+    code, site = swa.get_last_device_error()
+    assert code == swa.ERR_INVALID_ARG
+    assert swa.get_last_device_error()[0] == swa.OK
+    assert torch.all(o[1] == 3.0)
+    assert torch.equal(kc[1], d["k_cache"][1]) and torch.equal(vc[1], d["v_cache"][1])
+    keep = [0, 2]
+    o_ref, _, _ = oracle.decode(inp["pos"].numpy()[keep], f64(inp["q"])[keep], f64(inp["k"])[keep],
+                                f64(inp["v"])[keep], f64(inp["g"])[keep], f64(inp["wq"]),
+                                f64(inp["wk"]), bits(inp["k_cache"])[keep],
+                                bits(inp["v_cache"])[keep], R=42, base=cfg.base, eps=1e-6)
+    assert_parity(to_f64(o[keep]), o_ref, "decode o beside a bad position")
+
+
+def test_saturated_gate_gives_zero():
+    cfg = workloads.Decode("decode test", N=4, layers=1, Hq=8, Hkv=2, base=1e4, seed=13)
+    inp = {k: v.to(DEV) for k, v in workloads.decode_layer_inputs(cfg, layer=0).items()}
+    inp["g"] = torch.full_like(inp["g"], float("-inf"))
+    o = swa.decode_step(inp["pos"], inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"],
+                        inp["k_cache"], inp["v_cache"], rope_base=cfg.base)
+    assert torch.count_nonzero(o).item() == 0
