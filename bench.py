@@ -373,8 +373,54 @@ def secondary(swa, args, world, device, stream, peaks):
         "l2": "7.5 GB per step (> L2)"}
     del fns, sets
     torch.cuda.empty_cache()
+    out["train_fwd_bwd"] = train_bench(swa, args, world, device, stream, peaks)
     out["decode_step"] = decode_bench(swa, args, world, device, stream, peaks)
     return out
+
+
+def train_bench(swa, args, world, device, stream, peaks):
+    """Training step of the layer core on the training shape: swa_fwd (with
+    lse) then swa_bwd; inputs 1x16384 are above L2 (2.1 GB live)."""
+    cfg = workloads.TRAIN
+    d = workloads.prefill_inputs(cfg, device=device, with_grad_out=True)
+    o = torch.empty_like(d["q"])
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.T), dtype=torch.float32, device=device)
+    grads = (torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"]),
+             torch.empty_like(d["g"]), torch.zeros(cfg.D, device=device),
+             torch.zeros(cfg.D, device=device))
+    ws = torch.empty(swa.bwd_workspace_size(cfg.B, cfg.T, cfg.Hq, cfg.Hkv), dtype=torch.uint8,
+                     device=device)
+
+    def fwd():
+        swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], rope_base=cfg.base,
+                out=o, lse=lse)
+
+    def bwd():
+        swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"],
+                rope_base=cfg.base, workspace=ws, grads=grads)
+
+    def step():
+        fwd()
+        bwd()
+    steps = max(3, min(args.steps, 10))
+    ms, _, _, _ = timed_loop([step], steps, 3, stream, world)
+    ms_b, _, _, _ = timed_loop([bwd], steps, 3, stream, world)
+    tok = cfg.B * cfg.T
+    b_fb = (FWD_BYTES_PER_TOKEN(cfg) + cfg.Hq * 4 + BWD_BYTES_PER_TOKEN(cfg)) * tok
+    b_b = BWD_BYTES_PER_TOKEN(cfg) * tok
+    res = {"workload": cfg.name,
+           "tokens_per_s": round(tok * world / (ms / steps / 1e3), 1),
+           "ms_per_step": round(ms / steps, 4),
+           "algorithmic_bytes_per_step": b_fb,
+           "achieved_GBps": round(b_fb / (ms / steps / 1e3) / 1e9, 1),
+           "frac_of_measured_hbm": round(b_fb / (ms / steps / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+           "bwd_ms": round(ms_b / steps, 4),
+           "bwd_frac_of_measured_hbm":
+               round(b_b / (ms_b / steps / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+           "launches_per_step": 3}
+    del d, o, lse, grads, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def DECODE_BYTES_PER_SEQ_LAYER(c):

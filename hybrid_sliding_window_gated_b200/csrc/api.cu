@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "bwd_internal.h"
 #include "decode_internal.h"
 #include "swa_internal.h"
 
@@ -143,7 +144,8 @@ int swa_get_last_device_error(void* stream, int* site) {
   const int zero = 0;
   if (cudaMemcpy(word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return SWA_ERR_CUDA;
-  return v == kDevErrBadPosition ? SWA_ERR_INVALID_ARG : SWA_ERR_DEVICE_TIMEOUT;
+  // 0x100 + site: a wait ran out; 0x200 and up: an argument the kernel checked
+  return v >= kDevErrBadPosition ? SWA_ERR_INVALID_ARG : SWA_ERR_DEVICE_TIMEOUT;
 }
 
 int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
@@ -193,16 +195,6 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
 
 }  // extern "C"
 
-// Entry points whose kernels live in their own translation units.
-namespace swa {
-int swa_bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
-                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
-                 const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
-                 swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* workspace,
-                 size_t workspace_bytes, cudaStream_t stream);
-size_t swa_bwd_workspace_bytes(const swa_params_t* p);
-}  // namespace swa
-
 extern "C" {
 
 int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
@@ -211,13 +203,66 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
             float* dwq, float* dwk, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_params(p, false);
   if (rc != SWA_OK) return rc;
-  return swa_bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, workspace,
-                      workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  if (!q || !k || !v || !g || !wq || !wk || !lse || !dO || !dq || !dk || !dv || !dg || !dwq ||
+      !dwk || !workspace)
+    return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(wq) ||
+      !aligned16(wk) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(dg) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dwq) & 3u) || (reinterpret_cast<uintptr_t>(dwk) & 3u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SWA_ERR_INVALID_ARG;
+  const size_t da_bytes = bwd_ws_da_bytes(p->B, p->T, p->Hq);
+  const size_t d_bytes = bwd_ws_d_bytes(p->B, p->T, p->Hq);
+  if (workspace_bytes < da_bytes + 2 * d_bytes) return SWA_ERR_INVALID_ARG;
+
+  BwdArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.tiles_per_chain = static_cast<int>((p->T + kTile - 1) / kTile);
+  a.total_tiles = static_cast<long long>(a.tiles_per_chain) * p->B * p->Hkv;
+  a.scale = score_scale(p);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.q = q;
+  a.k = k;
+  a.g = g;
+  a.dO = dO;
+  a.lse = lse;
+  a.wq = wq;
+  a.wk = wk;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dg = dg;
+  a.dwq = dwq;
+  a.dwk = dwk;
+  a.ws_da = static_cast<uint16_t*>(workspace);
+  a.ws_d = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + da_bytes);
+  a.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + da_bytes + d_bytes);
+  rc = device_error_word(&a.err);
+  if (rc != SWA_OK) return rc;
+  fill_inv_freq(p, a.inv_freq);
+  if (a.total_tiles > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv, tda;
+  const uint64_t D = kHeadDim, T = p->T, B = p->B;
+  if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tda, a.ws_da, D, p->Hq, T, B, 64, 1, kTile, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  return launch_bwd(p, tq, tk, tv, tda, a, static_cast<cudaStream_t>(stream));
 }
 
 size_t swa_bwd_workspace_size(const swa_params_t* p) {
   if (check_params(p, false) != SWA_OK) return 0;
-  return swa_bwd_workspace_bytes(p);
+  return bwd_ws_da_bytes(p->B, p->T, p->Hq) + 2 * bwd_ws_d_bytes(p->B, p->T, p->Hq);
 }
 
 int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,

@@ -1,0 +1,1146 @@
+// bwd.cu -- backward of the gated sliding-window attention core for sm_100a.
+//
+// Forward (ZGCM-1 pages: onedev.kr summary, "어떻게 동작하나"; jaehun.me review,
+// "How Gated SWA Behaves"): q' = RoPE(RMSNorm(q; wq)), k' = RoPE(RMSNorm(k; wk)),
+// s_ij = scale q'_i.k'_j on the band j in [i-127, i], P = softmax(s), A = P V,
+// O = A (*) sigmoid(g).  Given dO and the forward's lse, the chain rule gives
+//   dg = dO (*) A (*) sig (1 - sig),   dA = dO (*) sig,   D_i = dA_i . A_i,
+//   dP = dA V^T,   dS = scale P (*) (dP - D),
+//   dq' = dS k',   dk' = dS^T q',   dv = P^T dA,
+// then RoPE^-1 (rotation by -theta) and the RMSNorm Jacobian
+//   dx = (w (*) dy - xhat mean(xhat (*) w (*) dy)) / r,   dw += dy (*) xhat.
+//
+// Two kernels, both on the tensor cores with TMEM accumulators:
+//   swa_bwd_q_kernel (query-major, one 128-row query tile and head at a time,
+//     key tiles t-1 and t resident): recomputes S and P (from lse) and
+//     A = P V, writes dg and the workspace rows dA (fp16) and D (fp32), then
+//     dP = dA V^T, dS per key tile into shared memory, dQ = dS K' and dq.
+//   swa_bwd_kv_kernel (key-major, one key tile at a time, query tiles j and
+//     j+1 and every head of the group): S^T = K' Q'^T and dP^T = V dA^T,
+//     P^T and dS^T packed in TMEM, dV += P^T dA and dK += dS^T Q' accumulated
+//     in TMEM across the 2G (query tile, head) pairs, then dk and dv.
+// Every dq row and every dk/dv row is complete inside one CTA: no atomics
+// except the per-CTA sums of dwq and dwk.
+//
+// Roles (256 threads): warp 0 TMA producer (its lanes also compute rotation
+// tables), warp 1 TMEM allocator and MMA issuer, warps 4-7 the compute
+// warpgroup (one thread per tile row).  Waits are bounded as in the forward.
+#include <cuda_fp16.h>
+
+#include "bwd_internal.h"
+#include "ptx.cuh"
+
+namespace swa {
+namespace bwd {
+
+constexpr int kThreads = 256;
+constexpr int kHalfBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 (one TMA box)
+constexpr int kTileBytes = 2 * kHalfBytes;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum Site {
+  kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
+  kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
+  kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged
+};
+
+// ---------------------------------------------------------------- helpers
+
+// Offset of 16-byte chunk `c` (0..7) of row `row` in a 128B-swizzled half tile.
+__device__ __forceinline__ uint32_t sw_off(int row, int c) {
+  return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ float2 bf2(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 f16x2(uint32_t u) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&u));
+}
+// Largest magnitude the fp16 staging of V and dA carries (the fp16 maximum).
+constexpr float kF16Max = 65504.0f;
+
+// Row `row` of a [128 x 128] bf16 tile (two 128-byte-row halves) converted to
+// fp16 in place: every backward contraction runs fp16 x fp16, three more
+// mantissa bits than bf16.  Returns false if a value is beyond the fp16 range.
+__device__ __forceinline__ bool row_to_f16(uint8_t* tile, int row) {
+  bool ok = true;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint4* p = reinterpret_cast<uint4*>(tile + h * kHalfBytes + row * 128);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 u = p[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = bf2(w[e]);
+        ok &= fabsf(f.x) <= kF16Max && fabsf(f.y) <= kF16Max;
+        o[e] = pack_f16x2(f.x, f.y);
+      }
+      p[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  return ok;
+}
+__device__ __forceinline__ float2 cmul(float2 x, float2 y) {
+  return make_float2(x.x * y.x - x.y * y.y, x.x * y.y + x.y * y.x);
+}
+
+// A bounded wait whose outcome is the same on every lane of the warp, so the
+// warp-collective tcgen05 loads and stores that follow never run divergent.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* err, int site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, site));
+}
+
+struct RotTables {
+  float2 lo[kMaxPairs][16];  // rot(b w_p), b = 0..15
+};
+
+// Rotation of position 128 j + row for pair p: hi[p][row/16] is rot((128 j +
+// 16 a) w_p) for the tile, lo the per-CTA table.
+__device__ __forceinline__ float2 rot_at(const float2 (*hi)[8], const RotTables& t, int p, int row) {
+  return cmul(hi[p][row >> 4], t.lo[p][row & 15]);
+}
+
+__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 x = *reinterpret_cast<const uint4*>(tile + sw_off(row, c));
+    const uint4 y = *reinterpret_cast<const uint4*>(tile + kHalfBytes + sw_off(row, c));
+    const uint32_t w[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = bf2(w[i]);
+      acc[i & 3] = __ffma2_rn(f, f, acc[i & 3]);
+    }
+  }
+  const float2 s = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return s.x + s.y;
+}
+
+// In place: bf16 row <- RoPE(row / rms(row) * w) as fp16 (the true normalised,
+// rotated operand; fp16 keeps 3 more mantissa bits than bf16 for the score and
+// gradient contractions whose operands are all computed here).  Returns 1/rms.
+template <int kPairs>
+__device__ __forceinline__ float norm_rope_row(uint8_t* tile, int row, const float* w,
+                                               const float2 (*hi)[8], const RotTables& t,
+                                               float eps) {
+  const float rinv = rsqrtf(row_sumsq(tile, row) * (1.0f / kHeadDim) + eps);
+  float x[kHeadDim / 2];  // the first half (dims 0..63): it holds every rotated pair
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(tile + sw_off(row, c));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * c + 2 * e] = bf16_lo(w4[e]) * rinv * w[8 * c + 2 * e];
+      x[8 * c + 2 * e + 1] = bf16_hi(w4[e]) * rinv * w[8 * c + 2 * e + 1];
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < kPairs; ++p) {
+    const float2 r = rot_at(hi, t, p, row);
+    const float a = x[p], b = x[p + kPairs];
+    x[p] = a * r.x - b * r.y;
+    x[p + kPairs] = b * r.x + a * r.y;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 u;
+    u.x = pack_f16x2(x[8 * c], x[8 * c + 1]);
+    u.y = pack_f16x2(x[8 * c + 2], x[8 * c + 3]);
+    u.z = pack_f16x2(x[8 * c + 4], x[8 * c + 5]);
+    u.w = pack_f16x2(x[8 * c + 6], x[8 * c + 7]);
+    *reinterpret_cast<uint4*>(tile + sw_off(row, c)) = u;
+  }
+  uint8_t* h1 = tile + kHalfBytes;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(h1 + sw_off(row, c));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int d = 64 + 8 * c + 2 * e;
+      o4[e] = pack_f16x2(bf16_lo(w4[e]) * rinv * w[d], bf16_hi(w4[e]) * rinv * w[d + 1]);
+    }
+    *reinterpret_cast<uint4*>(h1 + sw_off(row, c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+  }
+  return rinv;
+}
+
+// Sum a 64-value per-thread vector over the warp; lane l gets dims 2l, 2l+1.
+__device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane) {
+#pragma unroll
+  for (int m = 16, n = 32; m >= 1; m >>= 1, n >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float keep = up ? v[n + i] : v[i];
+      const float send = up ? v[i] : v[n + i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  return make_float2(v[0], v[1]);
+}
+
+// Gradient of one row through RoPE and RMSNorm.  dz: the gradient w.r.t. the
+// rotated, normalised row, read from TMEM columns [col, col+128) of this
+// thread's lane; x: the raw row (bf16 pairs); returns dx (bf16 pairs) and adds
+// dy (*) xhat into dw (shared, summed over the warp first).
+template <int kPairs>
+__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint32_t (&x)[64],
+                                               float rinv, const float* w, const float2 (*hi)[8],
+                                               const RotTables& t, int row, int lane, float* dw,
+                                               uint32_t (&dx)[64]) {
+  // Pass 1: dy (RoPE^-1 of dz), then dot = mean(xhat (*) w (*) dy) and dw.
+  float dot = 0.f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float y[64];
+    uint32_t r[32];
+    tmem_ld32(t_lane_col + half * 64, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+    tmem_ld32(t_lane_col + half * 64 + 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
+    if (half == 0) {
+#pragma unroll
+      for (int p = 0; p < kPairs; ++p) {
+        const float2 c = rot_at(hi, t, p, row);
+        const float a = y[p], b = y[p + kPairs];
+        y[p] = a * c.x + b * c.y;            // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
+        y[p + kPairs] = b * c.x - a * c.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 xh = bf2(x[half * 32 + i]);
+      const int d = half * 64 + 2 * i;
+      dot += y[2 * i] * w[d] * xh.x + y[2 * i + 1] * w[d + 1] * xh.y;
+      y[2 * i] *= xh.x * rinv;  // dw contribution dy * xhat
+      y[2 * i + 1] *= xh.y * rinv;
+    }
+    const float2 s = warp_reduce_scatter64(y, lane);
+    atomicAdd(dw + half * 64 + 2 * lane, s.x);
+    atomicAdd(dw + half * 64 + 2 * lane + 1, s.y);
+  }
+  dot *= rinv * (1.0f / kHeadDim);  // x = raw, so xhat = x * rinv
+  // Pass 2: dx = rinv (w dy - xhat dot).
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float y[64];
+    uint32_t r[32];
+    tmem_ld32(t_lane_col + half * 64, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+    tmem_ld32(t_lane_col + half * 64 + 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
+    if (half == 0) {
+#pragma unroll
+      for (int p = 0; p < kPairs; ++p) {
+        const float2 c = rot_at(hi, t, p, row);
+        const float a = y[p], b = y[p + kPairs];
+        y[p] = a * c.x + b * c.y;
+        y[p + kPairs] = b * c.x - a * c.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 xh = bf2(x[half * 32 + i]);
+      const int d = half * 64 + 2 * i;
+      const float g0 = rinv * (y[2 * i] * w[d] - xh.x * rinv * dot);
+      const float g1 = rinv * (y[2 * i + 1] * w[d + 1] - xh.y * rinv * dot);
+      dx[half * 32 + i] = pack_bf16x2(g0, g1);
+    }
+  }
+}
+
+// One 256-byte row per thread, in 16-byte pieces (rows are 16-byte aligned).
+__device__ __forceinline__ void load_row(const uint16_t* p, uint32_t (&x)[64]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + i);
+    x[4 * i] = u.x;
+    x[4 * i + 1] = u.y;
+    x[4 * i + 2] = u.z;
+    x[4 * i + 3] = u.w;
+  }
+}
+__device__ __forceinline__ void zero_row(uint32_t (&x)[64]) {
+#pragma unroll
+  for (int i = 0; i < 64; ++i) x[i] = 0u;
+}
+__device__ __forceinline__ void store_row(uint16_t* p, const uint32_t (&x)[64]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    reinterpret_cast<uint4*>(p)[i] = make_uint4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
+__device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
+  return make_desc_sw128(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mn(const uint8_t* tile, int kk) {
+  return make_desc_sw128(smem_u32(tile) + kk * 2048, kHalfBytes, 1024);
+}
+constexpr uint32_t kIdescKK = make_idesc_bf16(128, 128, false, false);  // A, B K-major
+constexpr uint32_t kIdescKM = make_idesc_bf16(128, 128, false, true);   // B MN-major
+// The same shapes with fp16 A and B (format fields 0): Q', K' and dS operands.
+constexpr uint32_t kF16 = ~((1u << 7) | (1u << 10));
+constexpr uint32_t kIdescKK16 = kIdescKK & kF16;
+constexpr uint32_t kIdescKM16 = kIdescKM & kF16;
+// fp16 holds the normalised operands while max|w| * sqrt(head_dim) stays well
+// inside its range; larger weights are refused (device error code below).
+constexpr float kMaxWeight = 4096.0f;
+
+// Contiguous per-CTA ranges of tiles over (batch row, KV head, tile).
+struct Cursor {
+  int b, kvh, t, u;
+};
+__device__ __forceinline__ Cursor cursor_at(const BwdArgs& a, int u0) {
+  Cursor c;
+  const int chain = u0 / a.tiles_per_chain;
+  c.t = u0 - chain * a.tiles_per_chain;
+  c.b = chain / a.Hkv;
+  c.kvh = chain - c.b * a.Hkv;
+  c.u = 0;
+  return c;
+}
+__device__ __forceinline__ void next_tile(Cursor& c, const BwdArgs& a) {
+  ++c.u;
+  if (++c.t == a.tiles_per_chain) {
+    c.t = 0;
+    if (++c.kvh == a.Hkv) {
+      c.kvh = 0;
+      ++c.b;
+    }
+  }
+}
+
+// Rotation table rot((128 j + 16 a) w_p), a = 0..7, computed by a warp.
+template <int kPairs>
+__device__ __forceinline__ void fill_rot_hi(float2 (*hi)[8], int j, const BwdArgs& a, int lane) {
+  for (int e = lane; e < kPairs * 8; e += 32) {
+    const int p = e >> 3, ai = e & 7;
+    float cv, sv;
+    rope_cos_sin(static_cast<double>(j) * kTile + 16.0 * ai, a.inv_freq[p], &cv, &sv);
+    hi[p][ai] = make_float2(cv, sv);
+  }
+}
+
+// ===================================================== pass 1: query-major
+
+struct alignas(1024) SmemQ {
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
+  uint8_t q[kTileBytes];   // Q' of the current head, then dS of one key tile
+  uint8_t da[kTileBytes];  // dA of the current head (MMA operand)
+  RotTables rot;
+  float2 rot_hi[2][kMaxPairs][8];  // per K slot
+  float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
+  uint64_t kfull[2], kready[2], kempty[2], vfull[2], vready[2], vempty[2];
+  uint64_t qfull, qempty, qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
+  uint64_t tables, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SmemQ) + 1024 <= 232448, "pass 1 shared memory");
+
+template <int kPairs>
+__global__ void __launch_bounds__(kThreads, 1)
+    swa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemQ& sm = *reinterpret_cast<SmemQ*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u0 = static_cast<int>(a.total_tiles * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
+  int n_tiles = u1 - u0;
+
+  if (tid < kHeadDim) {
+    sm.wq[tid] = a.wq[tid];
+    sm.wk[tid] = a.wk[tid];
+    sm.dw[tid] = 0.f;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.kfull[i], 2);
+      mbar_init(&sm.kready[i], 128);
+      mbar_init(&sm.kempty[i], 1);
+      mbar_init(&sm.vfull[i], 1);
+      mbar_init(&sm.vready[i], 128);
+      mbar_init(&sm.vempty[i], 1);
+    }
+    mbar_init(&sm.qfull, 1);
+    mbar_init(&sm.qempty, 1);
+    mbar_init(&sm.qready, 128);
+    mbar_init(&sm.sfull, 1);
+    mbar_init(&sm.pfull, 128);
+    mbar_init(&sm.afull, 1);
+    mbar_init(&sm.dafull, 128);
+    mbar_init(&sm.dpfull, 1);
+    mbar_init(&sm.dsfull, 128);
+    mbar_init(&sm.dq0, 1);
+    mbar_init(&sm.dqfull, 1);
+    mbar_init(&sm.tfree, 128);
+    mbar_init(&sm.tables, 128);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  // Weights whose normalised operands could leave the fp16 range are refused
+  // (uniformly: every thread sees the same shared copy).
+  {
+    bool wbad = false;
+    for (int d = 0; d < kHeadDim; ++d)
+      wbad |= !(fabsf(sm.wq[d]) <= kMaxWeight && fabsf(sm.wk[d]) <= kMaxWeight);
+    if (wbad) {
+      if (tid == 0 && blockIdx.x == 0) atomicCAS(a.err, 0, kDevErrBadWeights);
+      n_tiles = 0;
+    }
+  }
+  const int n_heads = n_tiles * a.G;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kpar = 0, vpar = 0, kused = 0, vused = 0;  // per-slot parity / used bits
+    bool ok = true;
+    int nq = 0;
+    auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
+      bool w = true;
+      if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+      return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+    };
+    auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {
+      const int s = j & 1;
+      uint32_t& par = is_k ? kpar : vpar;
+      uint32_t& used = is_k ? kused : vused;
+      uint64_t* full = is_k ? &sm.kfull[s] : &sm.vfull[s];
+      uint64_t* empty = is_k ? &sm.kempty[s] : &sm.vempty[s];
+      if (((used >> s) & 1u) &&
+          !wait0(empty, ((par >> s) & 1u) ^ 1u, is_k ? kSiteKEmpty : kSiteVEmpty))
+        return false;
+      if (lane == 0) {
+        uint8_t* dst = is_k ? sm.k[s] : sm.v[s];
+        const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+        mbar_arrive_expect_tx(full, kTileBytes);
+        tma_load_4d(dst, map, full, 0, c.kvh, j * kTile, c.b);
+        tma_load_4d(dst + kHalfBytes, map, full, 64, c.kvh, j * kTile, c.b);
+      }
+      if (is_k) {
+        fill_rot_hi<kPairs>(sm.rot_hi[s], j, a, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full);
+      }
+      par ^= 1u << s;
+      used |= 1u << s;
+      return true;
+    };
+    Cursor c = cursor_at(a, u0);
+    for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+      if (c.t > 0 && c.u == 0)
+        ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
+      ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
+      for (int h = 0; h < a.G && ok; ++h, ++nq) {
+        if (nq > 0 && !wait0(&sm.qempty, (nq - 1) & 1, kSiteQEmpty)) { ok = false; break; }
+        if (lane == 0) {
+          const int hq = c.kvh * a.G + h;
+          mbar_arrive_expect_tx(&sm.qfull, kTileBytes);
+          tma_load_4d(sm.q, &tm_q, &sm.qfull, 0, hq, c.t * kTile, c.b);
+          tma_load_4d(sm.q + kHalfBytes, &tm_q, &sm.qfull, 64, hq, c.t * kTile, c.b);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < 2; ++s) {
+        if ((kused >> s) & 1u) mbar_wait_drain(&sm.kfull[s], ((kpar >> s) & 1u) ^ 1u);
+        if ((vused >> s) & 1u) mbar_wait_drain(&sm.vfull[s], ((vpar >> s) & 1u) ^ 1u);
+      }
+      if (nq > 0) mbar_wait_drain(&sm.qfull, (nq - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t kpar = 0, vpar = 0;
+      bool ok = true;
+      int nds = 0;  // dS tiles consumed so far
+      Cursor c = cursor_at(a, u0);
+      int h = 0;
+      auto W = [&](uint64_t* bar, uint32_t par, int site) {
+        if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
+        return ok;
+      };
+      for (int n = 0; n < n_heads && ok; ++n) {
+        const uint32_t ph = n & 1;
+        const bool hp = c.t > 0;
+        const int sp = (c.t + 1) & 1, sc = c.t & 1;
+        if (h == 0) {
+          if (c.t > 0 && c.u == 0) {
+            if (!W(&sm.kready[sp], (kpar >> sp) & 1u, kSiteKReady)) break;
+            kpar ^= 1u << sp;
+          }
+          if (!W(&sm.kready[sc], (kpar >> sc) & 1u, kSiteKReady)) break;
+          kpar ^= 1u << sc;
+        }
+        if (!W(&sm.qready, ph, kSiteQReady)) break;
+        if (n > 0 && !W(&sm.tfree, ph ^ 1u, kSiteTFree)) break;
+        tc_fence_after();
+        // S = Q' [K'_{t-1} K'_t]^T into columns 0..255
+        for (int blk = hp ? 0 : 1; blk < 2; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + blk * 128, desc_kmajor(sm.q, kk), desc_kmajor(sm.k[blk ? sc : sp], kk),
+                   kIdescKK16, kk > 0);
+        mma_commit(&sm.sfull);
+        if (h == 0) {
+          if (c.t > 0 && c.u == 0) {
+            if (!W(&sm.vready[sp], (vpar >> sp) & 1u, kSiteVFull)) break;
+            vpar ^= 1u << sp;
+          }
+          if (!W(&sm.vready[sc], (vpar >> sc) & 1u, kSiteVFull)) break;
+          vpar ^= 1u << sc;
+        }
+        // A = P V into columns 256..383 (P packed in columns 0..127)
+        if (!W(&sm.pfull, ph, kSitePFull)) break;
+        tc_fence_after();
+        {
+          uint32_t acc = 0;
+          for (int blk = hp ? 0 : 1; blk < 2; ++blk)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              mma_ts(tmem + 256, tmem + blk * 64 + kk * 8, desc_mn(sm.v[blk ? sc : sp], kk),
+                     kIdescKM16, acc);
+              acc = 1;
+            }
+        }
+        mma_commit(&sm.afull);
+        // dP = dA [V_{t-1} V_t]^T into columns 256..511
+        if (!W(&sm.dafull, ph, kSiteDAFull)) break;
+        tc_fence_after();
+        for (int blk = hp ? 0 : 1; blk < 2; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 256 + blk * 128, desc_kmajor(sm.da, kk),
+                   desc_kmajor(sm.v[blk ? sc : sp], kk), kIdescKK16, kk > 0);
+        mma_commit(&sm.dpfull);
+        // dQ = sum over key tiles of dS K' into columns 128..255
+        {
+          uint32_t acc = 0;
+          for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+            if (!W(&sm.dsfull, nds & 1, kSiteDSFull)) break;
+            ++nds;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              mma_ss(tmem + 128, desc_kmajor(sm.q, kk), desc_mn(sm.k[blk ? sc : sp], kk),
+                     kIdescKM16, acc);
+              acc = 1;
+            }
+            mma_commit(blk == 0 ? &sm.dq0 : &sm.dqfull);
+          }
+          if (!ok) break;
+        }
+        mma_commit(&sm.qempty);
+        if (h == a.G - 1) {
+          if (hp) {
+            mma_commit(&sm.kempty[sp]);
+            mma_commit(&sm.vempty[sp]);
+          }
+          if (c.u == n_tiles - 1 || c.t == a.tiles_per_chain - 1) {
+            mma_commit(&sm.kempty[sc]);
+            mma_commit(&sm.vempty[sc]);
+          }
+        }
+        if (++h == a.G) {
+          h = 0;
+          next_tile(c, a);
+        }
+      }
+      if (!ok) {
+        mma_commit(&sm.drain);
+        mbar_wait_drain(&sm.drain, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------- compute warpgroup
+    const int row = tid - 128;
+    const int wq4 = warp & 3;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16);
+    for (int e = row; e < kPairs * 16; e += 128) {
+      const int p = e >> 4, bi = e & 15;
+      float cv, sv;
+      rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
+      sm.rot.lo[p][bi] = make_float2(cv, sv);
+    }
+    mbar_arrive(&sm.tables);
+    bool ok = warp_wait(&sm.tables, 0, abort, a.err, kSiteTables);
+    uint32_t kpar = 0, vpar = 0;
+    bool in_range = true;  // v and dO within the fp16 staging range
+    int nds = 0, ndq0 = 0;
+    Cursor c = cursor_at(a, u0);
+    int h = 0;
+    for (int n = 0; n < n_heads && ok; ++n) {
+      const uint32_t ph = n & 1;
+      const bool hp = c.t > 0;
+      const int sc = c.t & 1;
+      const int hq = c.kvh * a.G + h;
+      const long long pos = static_cast<long long>(c.t) * kTile + row;
+      const bool valid_row = pos < a.T;
+      const long long tok = (static_cast<long long>(c.b) * a.T + pos) * a.Hq + hq;  // row of q/g/dO
+      const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + pos;  // lse / D
+
+      // ---- K' of this tile's new key tiles (first head of the tile)
+      if (h == 0) {
+        for (int j = (c.t > 0 && c.u == 0) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+          const int s = j & 1;
+          ok = warp_wait(&sm.kfull[s], (kpar >> s) & 1u, abort, a.err, kSiteKFull);
+          if (!ok) break;
+          norm_rope_row<kPairs>(sm.k[s], row, sm.wk, sm.rot_hi[s], sm.rot, a.eps);
+          fence_proxy_async_smem();
+          mbar_arrive(&sm.kready[s]);
+          kpar ^= 1u << s;
+          ok = warp_wait(&sm.vfull[s], (vpar >> s) & 1u, abort, a.err, kSiteVFull);
+          if (!ok) break;
+          in_range &= row_to_f16(sm.v[s], row);
+          fence_proxy_async_smem();
+          mbar_arrive(&sm.vready[s]);
+          vpar ^= 1u << s;
+        }
+        if (!ok) break;
+      }
+      // ---- Q'
+      if (!(ok = warp_wait(&sm.qfull, ph, abort, a.err, kSiteQFull))) break;
+      const float rinv_q = norm_rope_row<kPairs>(sm.q, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.qready);
+      const float lse2 = valid_row ? a.lse[lrow] * kLog2e : 0.f;
+      float lsum = 0.f;
+
+      // ---- P = exp(s - lse) on the band, packed over columns 0..127
+      if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
+      tc_fence_after();
+      for (int blk = 0; blk < 2; ++blk) {
+        for (int pc = 0; pc < 4; ++pc) {
+          // key tile t-1 keeps columns > row, key tile t columns <= row
+          // Warp-uniform (tcgen05.ld is warp-collective); row validity is in the mask.
+          const bool any = blk == 0 ? (hp && pc >= wq4) : (pc <= wq4);
+          uint32_t pk[16];
+          if (any) {
+            uint32_t x[32];
+            tmem_ld32(t_row + blk * 128 + pc * 32, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = pc * 32 + 2 * e;
+              const bool in0 = valid_row && (blk == 0 ? c0 > row : c0 <= row);
+              const bool in1 = valid_row && (blk == 0 ? c0 + 1 > row : c0 + 1 <= row);
+              const float p0 = in0 ? ex2_approx(__uint_as_float(x[2 * e]) * a.scale_log2 - lse2) : 0.f;
+              const float p1 =
+                  in1 ? ex2_approx(__uint_as_float(x[2 * e + 1]) * a.scale_log2 - lse2) : 0.f;
+              pk[e] = pack_f16x2(p0, p1);
+              const float2 pr = f16x2(pk[e]);  // the values the MMAs see
+              lsum += pr.x + pr.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          }
+          tmem_st16(t_row + blk * 64 + pc * 16, pk);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.pfull);
+      // The forward's lse came from its own rounding of the scores; these rows
+      // are renormalised to sum to exactly 1 under this pass's scores, and the
+      // corrected normaliser goes to the key-major pass.
+      const float inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
+      if (valid_row) a.ws_lse[lrow] = a.lse[lrow] + __logf(lsum);
+
+      // ---- A: dg, dA (smem and workspace), D
+      uint32_t gw[64], dow[64];
+      if (valid_row) {
+        load_row(a.g + tok * kHeadDim, gw);
+        load_row(a.dO + tok * kHeadDim, dow);
+      } else {
+        zero_row(gw);
+        zero_row(dow);
+      }
+      if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
+      tc_fence_after();
+      float dsum = 0.f;
+      {
+        uint32_t dgw[64], daw[64];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t x[32];
+          tmem_ld32(t_row + 256 + ch * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int wi = ch * 16 + e;
+            const float2 gg = bf2(gw[wi]), dd = bf2(dow[wi]);
+            const float a0 = __uint_as_float(x[2 * e]) * inv_l;
+            const float a1 = __uint_as_float(x[2 * e + 1]) * inv_l;
+            const float s0 = 1.0f / (1.0f + __expf(-gg.x)), s1 = 1.0f / (1.0f + __expf(-gg.y));
+            dgw[wi] = pack_bf16x2(dd.x * a0 * s0 * (1.0f - s0), dd.y * a1 * s1 * (1.0f - s1));
+            in_range &= fabsf(dd.x) <= kF16Max && fabsf(dd.y) <= kF16Max;
+            daw[wi] = pack_f16x2(dd.x * s0, dd.y * s1);
+            const float2 dr = f16x2(daw[wi]);  // D uses the rounded dA the MMAs see
+            dsum += dr.x * a0 + dr.y * a1;
+          }
+        }
+        // dA into the MMA operand tile (row-major over dims, 128B swizzle)
+#pragma unroll
+        for (int c16 = 0; c16 < 16; ++c16)
+          *reinterpret_cast<uint4*>(sm.da + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) =
+              make_uint4(daw[4 * c16], daw[4 * c16 + 1], daw[4 * c16 + 2], daw[4 * c16 + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.dafull);
+        if (valid_row) {
+          store_row(a.dg + tok * kHeadDim, dgw);
+          store_row(a.ws_da + tok * kHeadDim, daw);
+          a.ws_d[lrow] = dsum;
+        }
+      }
+
+      // ---- dS = scale P (dP - D) per key tile into the Q slot, then dQ
+      if (!(ok = warp_wait(&sm.dpfull, ph, abort, a.err, kSiteDPFull))) break;
+      tc_fence_after();
+      for (int blk = hp ? 0 : 1; blk < 2 && ok; ++blk) {
+        if (blk == 1 && hp) {  // the MMA has read dS of key tile t-1 from the slot
+          if (!(ok = warp_wait(&sm.dq0, ndq0 & 1, abort, a.err, kSiteDQ0))) break;
+          ++ndq0;
+        }
+        for (int pc = 0; pc < 4; ++pc) {
+          uint32_t pk[16], dp[32];
+          tmem_ld16(t_row + blk * 64 + pc * 16, pk);
+          tmem_ld32(t_row + 256 + blk * 128 + pc * 32, dp);
+          tmem_wait_ld();
+          uint32_t ds[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 pp = f16x2(pk[e]);
+            const float d0 = a.scale * inv_l * pp.x * (__uint_as_float(dp[2 * e]) - dsum);
+            const float d1 = a.scale * inv_l * pp.y * (__uint_as_float(dp[2 * e + 1]) - dsum);
+            ds[e] = pack_f16x2(d0, d1);
+          }
+          uint8_t* half = sm.q + (pc >> 1) * kHalfBytes;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(half + sw_off(row, (pc & 1) * 4 + i)) =
+                make_uint4(ds[4 * i], ds[4 * i + 1], ds[4 * i + 2], ds[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.dsfull);
+        ++nds;
+      }
+      if (!ok) break;
+
+      // ---- dq through RoPE^-1 and the RMSNorm Jacobian
+      uint32_t xq[64];
+      if (valid_row) {
+        load_row(a.q + tok * kHeadDim, xq);
+      } else {
+        zero_row(xq);
+      }
+      if (!(ok = warp_wait(&sm.dqfull, ph, abort, a.err, kSiteDQFull))) break;
+      tc_fence_after();
+      {
+        uint32_t dx[64];
+        norm_rope_grad<kPairs>(t_row + 128, xq, rinv_q, sm.wq, sm.rot_hi[sc], sm.rot, row, lane,
+                               sm.dw, dx);
+        if (valid_row) store_row(a.dq + tok * kHeadDim, dx);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.tfree);
+      if (++h == a.G) {
+        h = 0;
+        next_tile(c, a);
+      }
+    }
+    if (!in_range) atomicCAS(a.err, 0, kDevErrRange);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  // per-CTA dwq into the caller's accumulator
+  if (tid >= 128 && !*abort) atomicAdd(a.dwq + (tid - 128), sm.dw[tid - 128]);
+}
+
+// ======================================================= pass 2: key-major
+
+struct alignas(1024) SmemKV {
+  uint8_t k[kTileBytes];   // K'_j
+  uint8_t v[kTileBytes];   // V_j
+  uint8_t q[kTileBytes];   // Q'_i of the current (query tile, head)
+  uint8_t da[kTileBytes];  // dA_i
+  RotTables rot;
+  float2 rot_hi[2][2][kMaxPairs][8];  // [key tile parity][tile j, j+1]
+  float lse2[2][kTile], dd[2][kTile];  // per query column, double-buffered
+  float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
+  uint64_t kfull, vfull, kvempty, qfull, qempty, qready, staged, sfull, pfull, dkvfull, tfree;
+  uint64_t tables, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SmemKV) + 1024 <= 232448, "pass 2 shared memory");
+
+template <int kPairs>
+__global__ void __launch_bounds__(kThreads, 1)
+    swa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
+                      const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                          ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u0 = static_cast<int>(a.total_tiles * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
+  int n_tiles = u1 - u0;
+
+  if (tid < kHeadDim) {
+    sm.wq[tid] = a.wq[tid];
+    sm.wk[tid] = a.wk[tid];
+    sm.dw[tid] = 0.f;
+  }
+  if (tid == 0) {
+    mbar_init(&sm.kfull, 2);
+    mbar_init(&sm.vfull, 1);
+    mbar_init(&sm.kvempty, 1);
+    mbar_init(&sm.qfull, 1);
+    mbar_init(&sm.qempty, 1);
+    mbar_init(&sm.qready, 128);
+    mbar_init(&sm.staged, 128);
+    mbar_init(&sm.sfull, 1);
+    mbar_init(&sm.pfull, 128);
+    mbar_init(&sm.dkvfull, 1);
+    mbar_init(&sm.tfree, 128);
+    mbar_init(&sm.tables, 128);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  // Weights whose normalised operands could leave the fp16 range are refused
+  // (uniformly: every thread sees the same shared copy).
+  {
+    bool wbad = false;
+    for (int d = 0; d < kHeadDim; ++d)
+      wbad |= !(fabsf(sm.wq[d]) <= kMaxWeight && fabsf(sm.wk[d]) <= kMaxWeight);
+    if (wbad) {
+      if (tid == 0 && blockIdx.x == 0) atomicCAS(a.err, 0, kDevErrBadWeights);
+      n_tiles = 0;
+    }
+  }
+  // (query tiles, heads) a key tile meets: tiles j and j+1 (if it exists) x G
+  auto n_iters = [&](const Cursor& c) { return (c.t + 1 < a.tiles_per_chain ? 2 : 1) * a.G; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    bool ok = true;
+    int nq = 0, nkv = 0;
+    auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
+      bool w = true;
+      if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+      return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+    };
+    Cursor c = cursor_at(a, u0);
+    for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+      if (it > 0 && !(ok = wait0(&sm.kvempty, (it - 1) & 1, kSiteKVEmpty))) break;
+      ++nkv;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.kfull, kTileBytes);
+        tma_load_4d(sm.k, &tm_k, &sm.kfull, 0, c.kvh, c.t * kTile, c.b);
+        tma_load_4d(sm.k + kHalfBytes, &tm_k, &sm.kfull, 64, c.kvh, c.t * kTile, c.b);
+        mbar_arrive_expect_tx(&sm.vfull, kTileBytes);
+        tma_load_4d(sm.v, &tm_v, &sm.vfull, 0, c.kvh, c.t * kTile, c.b);
+        tma_load_4d(sm.v + kHalfBytes, &tm_v, &sm.vfull, 64, c.kvh, c.t * kTile, c.b);
+      }
+      fill_rot_hi<kPairs>(sm.rot_hi[it & 1][0], c.t, a, lane);
+      fill_rot_hi<kPairs>(sm.rot_hi[it & 1][1], c.t + 1, a, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.kfull);
+      const int ni = n_iters(c);
+      for (int i = 0; i < ni && ok; ++i, ++nq) {
+        if (nq > 0 && !(ok = wait0(&sm.qempty, (nq - 1) & 1, kSiteQEmpty))) break;
+        if (lane == 0) {
+          const int qt = c.t + i / a.G, hq = c.kvh * a.G + i % a.G;
+          mbar_arrive_expect_tx(&sm.qfull, 2 * kTileBytes);
+          tma_load_4d(sm.q, &tm_q, &sm.qfull, 0, hq, qt * kTile, c.b);
+          tma_load_4d(sm.q + kHalfBytes, &tm_q, &sm.qfull, 64, hq, qt * kTile, c.b);
+          tma_load_4d(sm.da, &tm_da, &sm.qfull, 0, hq, qt * kTile, c.b);
+          tma_load_4d(sm.da + kHalfBytes, &tm_da, &sm.qfull, 64, hq, qt * kTile, c.b);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // every copy issued so far has completed or is drained here
+      if (nkv > 0) {
+        mbar_wait_drain(&sm.kfull, (nkv - 1) & 1);
+        mbar_wait_drain(&sm.vfull, (nkv - 1) & 1);
+      }
+      if (nq > 0) mbar_wait_drain(&sm.qfull, (nq - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int nq = 0;
+      auto W = [&](uint64_t* bar, uint32_t par, int site) {
+        if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
+        return ok;
+      };
+      Cursor c = cursor_at(a, u0);
+      for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+        const int ni = n_iters(c);
+        for (int i = 0; i < ni && ok; ++i, ++nq) {
+          if (!W(&sm.qready, nq & 1, kSiteQReady)) break;
+          if (i == 0) {
+            if (!W(&sm.vfull, it & 1, kSiteVFull)) break;
+            if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
+          }
+          tc_fence_after();
+          // S^T = K' Q'^T (columns 256..383), dP^T = V dA^T (384..511)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 256, desc_kmajor(sm.k, kk), desc_kmajor(sm.q, kk), kIdescKK16, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 384, desc_kmajor(sm.v, kk), desc_kmajor(sm.da, kk), kIdescKK16, kk > 0);
+          mma_commit(&sm.sfull);
+          if (!W(&sm.pfull, nq & 1, kSitePFull)) break;
+          tc_fence_after();
+          // dV += P^T dA (0..127), dK += dS^T Q' (128..255)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem, tmem + 256 + kk * 8, desc_mn(sm.da, kk), kIdescKM16, (i > 0 || kk > 0));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 128, tmem + 384 + kk * 8, desc_mn(sm.q, kk), kIdescKM16,
+                   (i > 0 || kk > 0));
+          mma_commit(&sm.qempty);
+        }
+        if (!ok) break;
+        mma_commit(&sm.dkvfull);
+        mma_commit(&sm.kvempty);
+      }
+      if (!ok) {
+        mma_commit(&sm.drain);
+        mbar_wait_drain(&sm.drain, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------- compute warpgroup
+    const int row = tid - 128;
+    const int wq4 = warp & 3;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16);
+    for (int e = row; e < kPairs * 16; e += 128) {
+      const int p = e >> 4, bi = e & 15;
+      float cv, sv;
+      rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
+      sm.rot.lo[p][bi] = make_float2(cv, sv);
+    }
+    mbar_arrive(&sm.tables);
+    bool ok = warp_wait(&sm.tables, 0, abort, a.err, kSiteTables);
+    bool in_range = true;  // v within the fp16 staging range
+    int nq = 0;
+    Cursor c = cursor_at(a, u0);
+    for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+      const long long kpos = static_cast<long long>(c.t) * kTile + row;  // this thread's key
+      // ---- K'_j
+      if (!(ok = warp_wait(&sm.kfull, it & 1, abort, a.err, kSiteKFull))) break;
+      const float rinv_k =
+          norm_rope_row<kPairs>(sm.k, row, sm.wk, sm.rot_hi[it & 1][0], sm.rot, a.eps);
+      if (!(ok = warp_wait(&sm.vfull, it & 1, abort, a.err, kSiteVFull))) break;
+      in_range &= row_to_f16(sm.v, row);
+      // (published to the MMA with the first qready below)
+      const int ni = n_iters(c);
+      for (int i = 0; i < ni && ok; ++i, ++nq) {
+        const int dt = i / a.G;  // query tile j + dt
+        const int hq = c.kvh * a.G + i % a.G;
+        const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // this thread's query row
+        // ---- Q'_i, and lse / D of its rows for the column-wise softmax
+        if (!(ok = warp_wait(&sm.qfull, nq & 1, abort, a.err, kSiteQFull))) break;
+        norm_rope_row<kPairs>(sm.q, row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
+        const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + qpos;
+        sm.lse2[nq & 1][row] = qpos < a.T ? a.ws_lse[lrow] * kLog2e : 0.f;
+        sm.dd[nq & 1][row] = qpos < a.T ? a.ws_d[lrow] : 0.f;
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.qready);
+        mbar_arrive(&sm.staged);  // lse2 / dd of this pair visible to the warpgroup
+        if (!(ok = warp_wait(&sm.staged, nq & 1, abort, a.err, kSiteStaged))) break;
+        // ---- P^T and dS^T for key row `row` against the 128 query columns
+        if (!(ok = warp_wait(&sm.sfull, nq & 1, abort, a.err, kSiteSFull))) break;
+        tc_fence_after();
+        const float* l2 = sm.lse2[nq & 1];
+        const float* dd = sm.dd[nq & 1];
+        for (int pc = 0; pc < 4; ++pc) {
+          // query tile j keeps columns >= row, tile j+1 columns < row
+          // Warp-uniform (tcgen05.ld is warp-collective); key validity is in the mask.
+          const bool any = dt == 0 ? (pc >= wq4) : (pc <= wq4);
+          uint32_t pk[16], dk[16];
+          if (any) {
+            uint32_t s[32], dp[32];
+            tmem_ld32(t_row + 256 + pc * 32, s);
+            tmem_ld32(t_row + 384 + pc * 32, dp);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float pv[2], dv[2];
+#pragma unroll
+              for (int f = 0; f < 2; ++f) {
+                const int col = pc * 32 + 2 * e + f;
+                const long long q_abs = static_cast<long long>(c.t + dt) * kTile + col;
+                const bool in = kpos < a.T && q_abs < a.T && (dt == 0 ? col >= row : col < row);
+                const float p =
+                    in ? ex2_approx(__uint_as_float(s[2 * e + f]) * a.scale_log2 - l2[col]) : 0.f;
+                pv[f] = p;
+                dv[f] = a.scale * p * (__uint_as_float(dp[2 * e + f]) - dd[col]);
+              }
+              pk[e] = pack_f16x2(pv[0], pv[1]);
+              dk[e] = pack_f16x2(dv[0], dv[1]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
+          }
+          tmem_st16(t_row + 256 + pc * 16, pk);
+          tmem_st16(t_row + 384 + pc * 16, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sm.pfull);
+      }
+      if (!ok) break;
+      // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j
+      const long long krow = (static_cast<long long>(c.b) * a.T + kpos) * a.Hkv + c.kvh;
+      uint32_t xk[64];
+      if (kpos < a.T) {
+        load_row(a.k + krow * kHeadDim, xk);
+      } else {
+        zero_row(xk);
+      }
+      if (!(ok = warp_wait(&sm.dkvfull, it & 1, abort, a.err, kSiteDKVFull))) break;
+      tc_fence_after();
+      {
+        uint32_t dx[64];
+        norm_rope_grad<kPairs>(t_row + 128, xk, rinv_k, sm.wk, sm.rot_hi[it & 1][0], sm.rot, row,
+                               lane, sm.dw, dx);
+        if (kpos < a.T) store_row(a.dk + krow * kHeadDim, dx);
+      }
+      {
+        uint32_t dv[64];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t x[32];
+          tmem_ld32(t_row + ch * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            dv[ch * 16 + e] = pack_bf16x2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+        }
+        if (kpos < a.T) store_row(a.dv + krow * kHeadDim, dv);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.tfree);
+    }
+    if (!in_range) atomicCAS(a.err, 0, kDevErrRange);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (tid >= 128 && !*abort) atomicAdd(a.dwk + (tid - 128), sm.dw[tid - 128]);
+}
+
+template <int kPairs>
+int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const CUtensorMap& tda, const BwdArgs& a, int num_sms, cudaStream_t stream) {
+  const size_t smem_q = sizeof(SmemQ) + 1024, smem_kv = sizeof(SmemKV) + 1024;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(swa_bwd_q_kernel<kPairs>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_q));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(swa_bwd_kv_kernel<kPairs>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_kv));
+    if (e != cudaSuccess) return map_cuda_error(e);
+    configured_device = dev;
+  }
+  const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
+  swa_bwd_q_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem_q, stream>>>(tq, tk, tv, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return map_cuda_error(e);
+  swa_bwd_kv_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem_kv, stream>>>(tq, tk, tv,
+                                                                                     tda, a);
+  return map_cuda_error(cudaGetLastError());
+}
+
+}  // namespace bwd
+
+int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
+               const CUtensorMap& tv, const CUtensorMap& tda, const BwdArgs& a,
+               cudaStream_t stream) {
+  DeviceInfo di;
+  int rc = current_device_info(&di);
+  if (rc != SWA_OK) return rc;
+  switch (p->rot_dim) {
+    case 0: return bwd::launch_impl<0>(tq, tk, tv, tda, a, di.num_sms, stream);
+    case 32: return bwd::launch_impl<16>(tq, tk, tv, tda, a, di.num_sms, stream);
+    case 42: return bwd::launch_impl<21>(tq, tk, tv, tda, a, di.num_sms, stream);
+    case 48: return bwd::launch_impl<24>(tq, tk, tv, tda, a, di.num_sms, stream);
+    default: return SWA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace swa

@@ -105,3 +105,16 @@ def test_decode_host_checks(L):
     args = [good] * 11
     args[7] = ctypes.c_void_p((1 << 20) + 8)  # ring must be 16-byte aligned
     assert L.swa_decode_step(ctypes.byref(_params()), *args) == swa.ERR_INVALID_ARG
+
+
+def test_bwd_host_checks(L):
+    p = _params(B=1, T=256, Hq=4, Hkv=1)
+    need = L.swa_bwd_workspace_size(ctypes.byref(p))
+    assert need >= 256 * 4 * 128 * 2 + 256 * 4 * 4
+    good = ctypes.c_void_p(1 << 20)
+    args = [good] * 15
+    assert L.swa_bwd(ctypes.byref(p), *args, need - 1, None) == swa.ERR_INVALID_ARG
+    args[14] = ctypes.c_void_p((1 << 20) + 16)  # workspace must be 256-byte aligned
+    assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
+    nul = ctypes.c_void_p(0)
+    assert L.swa_bwd(ctypes.byref(_params(T=0)), *([nul] * 15), 0, nul) == swa.OK
