@@ -13,7 +13,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "bwd", "bwd_workspace_size", "decode_step", "get_last_device_error",
+__all__ = ["fwd", "bwd", "bwd_noalloc", "bwd_workspace_size", "decode_step", "get_last_device_error",
            "SwaError", "Params", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswa.so")
@@ -53,6 +53,8 @@ def lib():
         L.swa_fwd.restype = ctypes.c_int
         L.swa_bwd.argtypes = [P] + [_vp] * 15 + [ctypes.c_size_t, _vp]
         L.swa_bwd.restype = ctypes.c_int
+        L.swa_bwd_noalloc.argtypes = [P] + [_vp] * 15
+        L.swa_bwd_noalloc.restype = ctypes.c_int
         L.swa_bwd_workspace_size.argtypes = [P]
         L.swa_bwd_workspace_size.restype = ctypes.c_size_t
         L.swa_decode_step.argtypes = [P] + [_vp] * 11
@@ -130,6 +132,25 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, e
                        _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq),
                        _ptr(dwk), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "swa_bwd")
+    return grads
+
+
+def bwd_noalloc(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4,
+                eps=1e-6, scale=0.0, grads=None, stream=None):
+    """As :func:`bwd`, with the library's fixed device scratch instead of a workspace."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g),
+                 torch.zeros(D, dtype=torch.float32, device=q.device),
+                 torch.zeros(D, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dg, dwq, dwk = grads
+    rc = lib().swa_bwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
+                               _ptr(wk), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(dg), _ptr(dwq), _ptr(dwk), _stream(stream))
+    _check(rc, "swa_bwd_noalloc")
     return grads
 
 

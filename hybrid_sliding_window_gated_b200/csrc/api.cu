@@ -16,6 +16,12 @@ namespace swa {
 // Sticky per-device error word written by bounded waits that ran out.
 __device__ int g_device_error = 0;
 
+// Device scratch of swa_bwd_noalloc: a fixed file-scope array, so that entry
+// point needs no allocation at all.  Calls that use it must not overlap on
+// one device.
+constexpr size_t kStaticScratchBytes = 64ull << 20;
+static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -46,6 +52,18 @@ int current_device_info(DeviceInfo* info) {
   }
   info->device = dev;
   info->num_sms = g_num_sms[dev];
+  return SWA_OK;
+}
+
+// Address of the static backward scratch on the current device (cached).
+static int static_scratch(void** ptr) {
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SWA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (addr[dev] == nullptr && cudaGetSymbolAddress(&addr[dev], g_bwd_scratch) != cudaSuccess)
+    return SWA_ERR_CUDA;
+  *ptr = addr[dev];
   return SWA_OK;
 }
 
@@ -258,6 +276,22 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
                            CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
   return launch_bwd(p, tq, tk, tv, tda, a, static_cast<cudaStream_t>(stream));
+}
+
+int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                    const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                    const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                    swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  const size_t need =
+      bwd_ws_da_bytes(p->B, p->T, p->Hq) + 2 * bwd_ws_d_bytes(p->B, p->T, p->Hq);
+  if (need > kStaticScratchBytes) return SWA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((rc = static_scratch(&scratch)) != SWA_OK) return rc;
+  return swa_bwd(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, scratch,
+                 kStaticScratchBytes, stream);
 }
 
 size_t swa_bwd_workspace_size(const swa_params_t* p) {

@@ -119,6 +119,19 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
 size_t swa_bwd_workspace_size(const swa_params_t* p);
 
 /*
+ * swa_bwd without a caller workspace (no paper counterpart: a library
+ * convenience).  The scratch is a fixed 64 MiB array inside the library's
+ * device image, so the call allocates nothing; problems whose
+ * swa_bwd_workspace_size exceeds 64 MiB return SWA_ERR_UNSUPPORTED.  Calls
+ * share that array: two of them must not run concurrently on one device
+ * (calls on one stream are fine).  Arguments and results are those of swa_bwd.
+ */
+int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                    const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                    const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                    swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* stream);
+
+/*
  * One decode step for p->B sequences against their window caches.
  * pos: [B] int64 device array (8-byte aligned), the position of each
  * sequence's new token, >= 0 (a negative one leaves that sequence's o and ring
