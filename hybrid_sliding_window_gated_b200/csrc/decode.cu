@@ -9,14 +9,18 @@
 //   q' = RoPE_p(RMSNorm(q)) attends over the W slots, slot s holding position
 //   p - ((p - s) mod W) (ignored when negative);  o = A * sigmoid(g).
 //
-// One CTA per (sequence, KV head): the 32 KiB K ring and 32 KiB V ring arrive
-// by TMA (128-byte swizzle) while the warps normalise and rotate q and k_new.
-// Warp w takes slots 32w .. 32w+31: S = q' K^T and the partial P V run on the
-// tensor cores with mma.sync (the G <= 8 query heads of the group are the M
-// rows, zero-padded to 16), with a per-warp maximum; the four partial results
-// are combined in shared memory (split-K softmax), scaled by 1/l and gated.
-// The warp owning slot p mod W patches that row, in shared memory and in the
-// ring, with k' (rounded to bf16) and v_new before reading it.
+// A unit is one (sequence, KV head): 64 KiB of ring plus 2.5 KiB of new-token
+// rows.  The kernel is persistent (one CTA per SM, a contiguous range of units
+// each) and streams: a producer warp keeps a 3-stage ring of units in flight
+// (the K and V rings by TMA with 128-byte swizzle, q, g, k_new, v_new by bulk
+// copies, the position by a plain load), while two consumer groups of four
+// warps take alternate units.  In a group, warp w takes slots 32w .. 32w+31:
+// S = q' K^T and the partial P V run on the tensor cores with mma.sync (the
+// G <= 8 query heads of the group are the M rows, zero-padded to 16), with a
+// per-warp maximum; the four partials are combined in shared memory (split-K
+// softmax), scaled by 1/l and gated.  The warp owning slot p mod W patches that
+// row, in shared memory and in the ring, with k' (rounded to bf16) and v_new
+// before reading it.
 #include "decode_internal.h"
 #include "ptx.cuh"
 #include "warp_mma.cuh"
@@ -24,32 +28,72 @@
 namespace swa {
 namespace dec {
 
-constexpr int kThreads = 128;
+constexpr int kGroups = 2;                       // consumer groups of 4 warps
+constexpr int kThreads = 32 * (1 + 4 * kGroups);  // producer warp + consumers
+constexpr int kStages = 3;
 constexpr int kHalfBytes = kWindow * 64 * 2;  // 128 slots x 64 dims of bf16 (one TMA box)
 constexpr int kQStride = 68;                  // words per packed q' row (bank-conflict padding)
 constexpr int kOStride = 136;                 // floats per partial-O row (padding)
 
-struct alignas(1024) Smem {
+struct alignas(1024) Stage {
   uint8_t k[2][kHalfBytes];  // K ring, dims 0..63 and 64..127, 128B-swizzled
   uint8_t v[2][kHalfBytes];  // V ring
+  uint16_t q[kDecMaxGroup][kHeadDim];  // the group's query rows
+  uint16_t g[kDecMaxGroup][kHeadDim];  // gate logits
+  uint16_t kn[kHeadDim], vn[kHeadDim];  // new token's k and v
+  long long pos;
+};
+
+struct Group {
   uint32_t qa[kDecMaxGroup][kQStride];  // q' as packed bf16 pairs
   float scratch[4][kHeadDim];           // per-warp norm / RoPE staging
   float mw[4][kDecMaxGroup];            // per-warp row maxima (log2 units)
   float lw[4][kDecMaxGroup];            // per-warp row sums
-  uint64_t kfull, vfull;
+};
+
+struct alignas(1024) Smem {
+  Stage st[kStages];
+  Group grp[kGroups];
+  uint64_t full[kStages], empty[kStages];
   int abort;
 };
-// The partial outputs [4 warps][G heads][kOStride] reuse the K ring once the
-// scores are done.
+// The partial outputs [4 warps][G heads][kOStride] reuse a stage's K ring once
+// the scores are done.
 static_assert(4 * kDecMaxGroup * kOStride * 4 <= 2 * kHalfBytes, "partial O does not fit");
-static_assert(sizeof(Smem) + 1024 <= 113 * 1024, "decode smem should allow two CTAs per SM");
+static_assert(sizeof(Smem) + 1024 <= 232448, "decode shared memory");
 
-enum Site { kSiteKFull = 0x40, kSiteVFull };
+enum Site { kSiteFull = 0x40, kSiteEmpty, kSiteGroup };
 
 // Byte offset of 16-byte chunk c (0..15) of slot row s in a [half][slot][64]
 // 128B-swizzled ring tile.
 __device__ __forceinline__ uint32_t ring_off(int s, int c) {
   return static_cast<uint32_t>((c >> 3) * kHalfBytes + s * 128 + (((c & 7) ^ (s & 7)) << 4));
+}
+
+// 1-D bulk copy global -> shared, completing on `bar` (16-byte aligned, size a
+// multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Barrier over the 128 threads of consumer group `id` that also ANDs `v`
+// across them: every decision taken after it is the same on the whole group.
+__device__ __forceinline__ bool group_and(bool v, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id)
+      : "memory");
+  return r != 0;
 }
 
 // x (4 dims 4*lane .. 4*lane+3 of one head) -> RoPE_p(x / rms(x) * w) in
@@ -92,85 +136,46 @@ __device__ __forceinline__ void load4(const uint16_t* p, float (&x)[4]) {
   x[3] = bf16_hi(u.y);
 }
 
-__global__ void __launch_bounds__(kThreads)
-    swa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const DecArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                      ~static_cast<uintptr_t>(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x / a.Hkv, kvh = blockIdx.x - n * a.Hkv;
-  const long long p = a.pos[n];
-  if (p < 0) {
-    if (tid == 0) atomicCAS(a.err, 0, kDevErrBadPosition);
+// One (sequence n, KV head kvh) unit, by the 128 threads of consumer group
+// `gi` (local warp lw).  The stage holds the unit's rings and new-token rows.
+__device__ __forceinline__ void process_unit(Stage& st, Group& gp, const DecArgs& a, int n,
+                                             int kvh, int gi, int lw, int lane) {
+  const int bar_id = 1 + gi;
+  const long long p = st.pos;
+  if (p < 0) {  // the same value for the whole group
+    if (lw == 0 && lane == 0) atomicCAS(a.err, 0, kDevErrBadPosition);
     return;
   }
   const int s0 = static_cast<int>(p & (kWindow - 1));  // slot of the new token
   const int owner = s0 >> 5;                           // warp whose slots hold it
 
-  if (tid == 0) {
-    mbar_init(&sm.kfull, 1);
-    mbar_init(&sm.vfull, 1);
-    sm.abort = 0;
-    fence_barrier_init();
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
-    mbar_arrive_expect_tx(&sm.kfull, 2 * kHalfBytes);
-    tma_load_4d(sm.k[0], &tm_k, &sm.kfull, 0, 0, kvh, n);
-    tma_load_4d(sm.k[1], &tm_k, &sm.kfull, 64, 0, kvh, n);
-    mbar_arrive_expect_tx(&sm.vfull, 2 * kHalfBytes);
-    tma_load_4d(sm.v[0], &tm_v, &sm.vfull, 0, 0, kvh, n);
-    tma_load_4d(sm.v[1], &tm_v, &sm.vfull, 64, 0, kvh, n);
-  }
-
-  // ---- while the rings load: q' for heads warp, warp+4; k' and v_new on the
-  // owner warp; the gate values this thread will apply.
+  // ---- q' for heads lw, lw+4; k' and v_new on the owner warp
   float cs = 1.0f, sn = 0.0f;
   if (lane < a.half_rot) rope_cos_sin(static_cast<double>(p), a.inv_freq[lane], &cs, &sn);
-  for (int h = warp; h < a.G; h += 4) {
+  for (int h = lw; h < a.G; h += 4) {
     float x[4];
-    load4(a.q + ((static_cast<long long>(n) * a.Hq + kvh * a.G + h) * kHeadDim + 4 * lane), x);
-    norm_rope_row(x, a.wq, a.eps, sm.scratch[warp], lane, a.half_rot, cs, sn);
-    sm.qa[h][2 * lane] = pack_bf16x2(x[0], x[1]);
-    sm.qa[h][2 * lane + 1] = pack_bf16x2(x[2], x[3]);
+    load4(st.q[h] + 4 * lane, x);
+    norm_rope_row(x, a.wq, a.eps, gp.scratch[lw], lane, a.half_rot, cs, sn);
+    gp.qa[h][2 * lane] = pack_bf16x2(x[0], x[1]);
+    gp.qa[h][2 * lane + 1] = pack_bf16x2(x[2], x[3]);
   }
-  uint2 kp = make_uint2(0u, 0u), vp = make_uint2(0u, 0u);
-  const long long kv_row = (static_cast<long long>(n) * a.Hkv + kvh) * kHeadDim;
-  if (warp == owner) {
+  if (lw == owner) {
     float x[4];
-    load4(a.k_new + kv_row + 4 * lane, x);
-    norm_rope_row(x, a.wk, a.eps, sm.scratch[warp], lane, a.half_rot, cs, sn);
-    kp = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-    vp = *reinterpret_cast<const uint2*>(a.v_new + kv_row + 4 * lane);
-  }
-  uint2 gv[kDecMaxGroup / 4];
-#pragma unroll
-  for (int i = 0; i < kDecMaxGroup / 4; ++i) {
-    const int h = warp + 4 * i;
-    if (h < a.G)
-      gv[i] = *reinterpret_cast<const uint2*>(
-          a.g + (static_cast<long long>(n) * a.Hq + kvh * a.G + h) * kHeadDim + 4 * lane);
-  }
-  __syncthreads();  // barrier init and q' visible
-
-  // Ring row offset of this sequence's slot s0 and the chunk this lane patches.
-  const long long ring_row = ((static_cast<long long>(n) * a.Hkv + kvh) * kWindow + s0) * kHeadDim;
-  const uint32_t patch_off = ring_off(s0, lane >> 1) + (lane & 1) * 8;
-
-  mbar_wait(&sm.kfull, 0, &sm.abort, a.err, kSiteKFull);
-  __syncthreads();
-  if (sm.abort) {
-    if (tid == 0) {
-      mbar_wait_drain(&sm.kfull, 0);
-      mbar_wait_drain(&sm.vfull, 0);
-    }
-    return;
-  }
-  if (warp == owner) {
-    *reinterpret_cast<uint2*>(&sm.k[0][0] + patch_off) = kp;
+    load4(st.kn + 4 * lane, x);
+    norm_rope_row(x, a.wk, a.eps, gp.scratch[lw], lane, a.half_rot, cs, sn);
+    const uint2 kp = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+    const uint2 vp = *reinterpret_cast<const uint2*>(st.vn + 4 * lane);
+    // Slot s0 of the rings: this lane's 4 dims, in shared memory and in HBM
+    // (the ring copy in shared memory has landed, so the global row is free).
+    const uint32_t off = ring_off(s0, lane >> 1) + (lane & 1) * 8;
+    *reinterpret_cast<uint2*>(&st.k[0][0] + off) = kp;
+    *reinterpret_cast<uint2*>(&st.v[0][0] + off) = vp;
+    const long long ring_row =
+        ((static_cast<long long>(n) * a.Hkv + kvh) * kWindow + s0) * kHeadDim;
     *reinterpret_cast<uint2*>(a.k_cache + ring_row + 4 * lane) = kp;
-    __syncwarp();
+    *reinterpret_cast<uint2*>(a.v_cache + ring_row + 4 * lane) = vp;
   }
+  group_and(true, bar_id);  // q' and the patched rows visible to the group
 
   // ---- S = q' K^T over this warp's 32 slots (4 n-tiles of 8 slots).
   const int grp = lane >> 2, tig = lane & 3;
@@ -178,20 +183,20 @@ __global__ void __launch_bounds__(kThreads)
   float acc[4][4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-  const uint32_t kbase = smem_u32(sm.k[0]);
+  const uint32_t kbase = smem_u32(st.k[0]);
 #pragma unroll
   for (int kp2 = 0; kp2 < 4; ++kp2) {  // pairs of 16-dim k-steps
     uint32_t qa0[2], qa2[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int kk = 2 * kp2 + e;
-      qa0[e] = row_ok ? sm.qa[grp][8 * kk + tig] : 0u;
-      qa2[e] = row_ok ? sm.qa[grp][8 * kk + 4 + tig] : 0u;
+      qa0[e] = row_ok ? gp.qa[grp][8 * kk + tig] : 0u;
+      qa2[e] = row_ok ? gp.qa[grp][8 * kk + 4 + tig] : 0u;
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t b[4];
-      const int slot = 32 * warp + 8 * j + (lane & 7);
+      const int slot = 32 * lw + 8 * j + (lane & 7);
       ldsm_x4(kbase + ring_off(slot, 4 * kp2 + (lane >> 3)), b);
       mma_16816(acc[j], qa0[0], 0u, qa2[0], 0u, b[0], b[1]);
       mma_16816(acc[j], qa0[1], 0u, qa2[1], 0u, b[2], b[3]);
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int j = 0; j < 4; ++j) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int s = 32 * warp + 8 * j + 2 * tig + e;
+      const int s = 32 * lw + 8 * j + 2 * tig + e;
       const bool valid = p - ((p - s) & (kWindow - 1)) >= 0;
       acc[j][e] = valid ? acc[j][e] * a.scale_log2 : -INFINITY;
       m = fmaxf(m, acc[j][e]);
@@ -225,59 +230,44 @@ __global__ void __launch_bounds__(kThreads)
   l += __shfl_xor_sync(0xffffffffu, l, 2);
   if (!row_ok) pa[0] = pa[1] = pa[2] = pa[3] = 0u;
 
-  mbar_wait(&sm.vfull, 0, &sm.abort, a.err, kSiteVFull);
-  __syncthreads();
-  if (sm.abort) {
-    if (tid == 0) mbar_wait_drain(&sm.vfull, 0);
-    return;
-  }
-  if (warp == owner) {
-    *reinterpret_cast<uint2*>(&sm.v[0][0] + patch_off) = vp;
-    *reinterpret_cast<uint2*>(a.v_cache + ring_row + 4 * lane) = vp;
-    __syncwarp();
-  }
-
   // ---- partial O = P V over this warp's slots: 16 n-tiles of 8 dims, two
   // 16-slot k-steps each.
   float oacc[16][4];
-  const uint32_t vbase = smem_u32(sm.v[0]);
+  const uint32_t vbase = smem_u32(st.v[0]);
 #pragma unroll
   for (int nd = 0; nd < 16; ++nd) {
     oacc[nd][0] = oacc[nd][1] = oacc[nd][2] = oacc[nd][3] = 0.0f;
     uint32_t b[4];
-    const int slot = 32 * warp + lane;  // matrix lane/8 = slots 8(lane/8) .. +7
+    const int slot = 32 * lw + lane;  // matrix lane/8 = slots 8(lane/8) .. +7
     ldsm_x4_trans(vbase + ring_off(slot, nd), b);
     mma_16816(oacc[nd], pa[0], 0u, pa[1], 0u, b[0], b[1]);
     mma_16816(oacc[nd], pa[2], 0u, pa[3], 0u, b[2], b[3]);
   }
 
-  __syncthreads();  // every warp is done with the K ring: reuse it for partials
-  float* part = reinterpret_cast<float*>(sm.k[0]);  // [4][G][kOStride]
+  group_and(true, bar_id);  // every warp is done with the K ring: reuse it
+  float* part = reinterpret_cast<float*>(st.k[0]);  // [4][kDecMaxGroup][kOStride]
   if (row_ok) {
-    float* dst = part + (warp * kDecMaxGroup + grp) * kOStride + 2 * tig;
+    float* dst = part + (lw * kDecMaxGroup + grp) * kOStride + 2 * tig;
 #pragma unroll
     for (int nd = 0; nd < 16; ++nd)
       *reinterpret_cast<float2*>(dst + 8 * nd) = make_float2(oacc[nd][0], oacc[nd][1]);
     if (tig == 0) {
-      sm.mw[warp][grp] = m;
-      sm.lw[warp][grp] = l;
+      gp.mw[lw][grp] = m;
+      gp.lw[lw][grp] = l;
     }
   }
-  __syncthreads();
+  group_and(true, bar_id);
 
   // ---- combine: o = (sum_w O_w 2^(m_w - m)) / (sum_w l_w 2^(m_w - m)) * sigmoid(g)
-#pragma unroll
-  for (int i = 0; i < kDecMaxGroup / 4; ++i) {
-    const int h = warp + 4 * i;
-    if (h >= a.G) break;
+  for (int h = lw; h < a.G; h += 4) {
     float mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, sm.mw[w][h]);
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, gp.mw[w][h]);
     float f[4], lsum = 0.0f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      f[w] = sm.mw[w][h] == -INFINITY ? 0.0f : ex2_approx(sm.mw[w][h] - mx);
-      lsum += f[w] * sm.lw[w][h];
+      f[w] = gp.mw[w][h] == -INFINITY ? 0.0f : ex2_approx(gp.mw[w][h] - mx);
+      lsum += f[w] * gp.lw[w][h];
     }
     float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -290,7 +280,8 @@ __global__ void __launch_bounds__(kThreads)
       y[3] += f[w] * v4.w;
     }
     const float inv_l = 1.0f / lsum;
-    const float gx[4] = {bf16_lo(gv[i].x), bf16_hi(gv[i].x), bf16_lo(gv[i].y), bf16_hi(gv[i].y)};
+    float gx[4];
+    load4(st.g[h] + 4 * lane, gx);
     float ov[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) ov[e] = y[e] * inv_l / (1.0f + __expf(-gx[e]));
@@ -300,24 +291,121 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+__global__ void __launch_bounds__(kThreads, 1)
+    swa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const DecArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long units = static_cast<long long>(a.N) * a.Hkv;
+  const long long u0 = units * blockIdx.x / gridDim.x;
+  const int n_units = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x - u0);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 2);  // the copies' expect_tx arrive + the position
+      mbar_init(&sm.empty[s], 1);
+    }
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort = &sm.abort;
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // the set-up above overlapped its tail; every read and write of global
+  // memory below waits for it to complete.  The next launch may start its own
+  // set-up as soon as SMs free up.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      const uint32_t row_bytes = kHeadDim * 2;
+      const uint32_t bytes = 4 * kHalfBytes + 2 * a.G * row_bytes + 2 * row_bytes;
+      int issued[kStages] = {0};
+      bool ok = true;
+      for (int i = 0; i < n_units; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages &&
+            !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1, abort, a.err, kSiteEmpty)) {
+          ok = false;
+          break;
+        }
+        const long long u = u0 + i;
+        const int n = static_cast<int>(u / a.Hkv), kvh = static_cast<int>(u - u / a.Hkv * a.Hkv);
+        Stage& st = sm.st[s];
+        mbar_arrive_expect_tx(&sm.full[s], bytes);
+        tma_load_4d(st.k[0], &tm_k, &sm.full[s], 0, 0, kvh, n);
+        tma_load_4d(st.k[1], &tm_k, &sm.full[s], 64, 0, kvh, n);
+        tma_load_4d(st.v[0], &tm_v, &sm.full[s], 0, 0, kvh, n);
+        tma_load_4d(st.v[1], &tm_v, &sm.full[s], 64, 0, kvh, n);
+        const long long qrow = (static_cast<long long>(n) * a.Hq + kvh * a.G) * kHeadDim;
+        const long long kvrow = (static_cast<long long>(n) * a.Hkv + kvh) * kHeadDim;
+        bulk_load(st.q, a.q + qrow, a.G * row_bytes, &sm.full[s]);
+        bulk_load(st.g, a.g + qrow, a.G * row_bytes, &sm.full[s]);
+        bulk_load(st.kn, a.k_new + kvrow, row_bytes, &sm.full[s]);
+        bulk_load(st.vn, a.v_new + kvrow, row_bytes, &sm.full[s]);
+        st.pos = a.pos[n];  // read while the copies fly
+        mbar_arrive(&sm.full[s]);  // releases the position written above
+        ++issued[s];
+      }
+      if (!ok) {
+        // Every copy issued lands before the CTA releases its shared memory.
+        for (int s = 0; s < kStages; ++s)
+          if (issued[s] > 0) mbar_wait_drain(&sm.full[s], (issued[s] - 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------- consumer group
+    const int gi = (warp - 1) >> 2, lw = (warp - 1) & 3;
+    for (int i = gi; i < n_units; i += kGroups) {
+      const int s = i % kStages;
+      const bool got = mbar_wait(&sm.full[s], (i / kStages) & 1, abort, a.err, kSiteFull);
+      if (!group_and(got, 1 + gi)) break;  // the same decision on the whole group
+      const long long u = u0 + i;
+      const int n = static_cast<int>(u / a.Hkv), kvh = static_cast<int>(u - u / a.Hkv * a.Hkv);
+      process_unit(sm.st[s], sm.grp[gi], a, n, kvh, gi, lw, lane);
+      group_and(true, 1 + gi);  // the group is done with the stage
+      if (lw == 0 && lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+  }
+  __syncthreads();
+}
+
 }  // namespace dec
 
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a,
                   cudaStream_t stream) {
+  DeviceInfo di;
+  int rc = current_device_info(&di);
+  if (rc != SWA_OK) return rc;
   const size_t smem = sizeof(dec::Smem) + 1024;
   static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  if (configured_device != di.device) {
     cudaError_t e = cudaFuncSetAttribute(dec::swa_decode_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return map_cuda_error(e);
-    configured_device = dev;
+    configured_device = di.device;
   }
-  const long long grid = static_cast<long long>(a.N) * a.Hkv;
-  dec::swa_decode_kernel<<<static_cast<unsigned>(grid), dec::kThreads, smem, stream>>>(tk, tv, a);
-  return map_cuda_error(cudaGetLastError());
+  const long long units = static_cast<long long>(a.N) * a.Hkv;
+  const long long grid = units < di.num_sms ? units : di.num_sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(dec::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddepcontrol
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return map_cuda_error(cudaLaunchKernelEx(&cfg, dec::swa_decode_kernel, tk, tv, a));
 }
 
 }  // namespace swa
