@@ -41,7 +41,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum Site {
   kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
   kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
-  kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged
+  kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged,
+  kSiteMmaDone
 };
 
 // ---------------------------------------------------------------- helpers
@@ -190,41 +191,65 @@ __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane
   return make_float2(v[0], v[1]);
 }
 
-// Gradient of one row through RoPE and RMSNorm.  dz: the gradient w.r.t. the
-// rotated, normalised row, read from TMEM columns [col, col+128) of this
-// thread's lane; x: the raw row (bf16 pairs); returns dx (bf16 pairs) and adds
-// dy (*) xhat into dw (shared, summed over the warp first).
+// Half `half` of a raw bf16 row (32 words), or zeros for a row past the end.
+__device__ __forceinline__ void load_half(const uint16_t* xrow, int half, uint32_t (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 u = xrow ? __ldg(reinterpret_cast<const uint4*>(xrow) + 8 * half + i)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    x[4 * i] = u.x;
+    x[4 * i + 1] = u.y;
+    x[4 * i + 2] = u.z;
+    x[4 * i + 3] = u.w;
+  }
+}
+
+// dy for dims [64 half, 64 half + 64): the gradient w.r.t. the rotated,
+// normalised row (TMEM columns from t_lane_col), rotated back by RoPE^-1.
 template <int kPairs>
-__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint32_t (&x)[64],
+__device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half, const float2 (*hi)[8],
+                                             const RotTables& t, int row, float (&y)[64]) {
+  uint32_t r[32];
+  tmem_ld32(t_lane_col + half * 64, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+  tmem_ld32(t_lane_col + half * 64 + 32, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
+  if (half == 0) {
+#pragma unroll
+    for (int p = 0; p < kPairs; ++p) {
+      const float2 c = rot_at(hi, t, p, row);
+      const float a = y[p], b = y[p + kPairs];
+      y[p] = a * c.x + b * c.y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
+      y[p + kPairs] = b * c.x - a * c.y;
+    }
+  }
+}
+
+// Gradient of one row through RoPE and RMSNorm.  dz: the gradient w.r.t. the
+// rotated, normalised row, in TMEM columns [t_lane_col, +128) of this thread's
+// lane; xrow: the raw row in global memory (nullptr: a row past the end).
+// Writes dx to `out` (unless nullptr) and adds dy (*) xhat into dw (shared,
+// summed over the warp first).  Works half a row at a time.
+template <int kPairs>
+__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16_t* xrow,
                                                float rinv, const float* w, const float2 (*hi)[8],
                                                const RotTables& t, int row, int lane, float* dw,
-                                               uint32_t (&dx)[64]) {
-  // Pass 1: dy (RoPE^-1 of dz), then dot = mean(xhat (*) w (*) dy) and dw.
+                                               uint16_t* out) {
+  // Pass 1: dot = mean(xhat (*) w (*) dy) and dw.
   float dot = 0.f;
-#pragma unroll
+#pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
-    uint32_t r[32];
-    tmem_ld32(t_lane_col + half * 64, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-    tmem_ld32(t_lane_col + half * 64 + 32, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
-    if (half == 0) {
-#pragma unroll
-      for (int p = 0; p < kPairs; ++p) {
-        const float2 c = rot_at(hi, t, p, row);
-        const float a = y[p], b = y[p + kPairs];
-        y[p] = a * c.x + b * c.y;            // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
-        y[p + kPairs] = b * c.x - a * c.y;
-      }
-    }
+    uint32_t x[32];
+    load_half(xrow, half, x);
+    load_dy_half<kPairs>(t_lane_col, half, hi, t, row, y);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = bf2(x[half * 32 + i]);
+      const float2 xh = bf2(x[i]);
       const int d = half * 64 + 2 * i;
       dot += y[2 * i] * w[d] * xh.x + y[2 * i + 1] * w[d + 1] * xh.y;
       y[2 * i] *= xh.x * rinv;  // dw contribution dy * xhat
@@ -236,53 +261,31 @@ __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint32
   }
   dot *= rinv * (1.0f / kHeadDim);  // x = raw, so xhat = x * rinv
   // Pass 2: dx = rinv (w dy - xhat dot).
-#pragma unroll
+#pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
-    uint32_t r[32];
-    tmem_ld32(t_lane_col + half * 64, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-    tmem_ld32(t_lane_col + half * 64 + 32, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
-    if (half == 0) {
-#pragma unroll
-      for (int p = 0; p < kPairs; ++p) {
-        const float2 c = rot_at(hi, t, p, row);
-        const float a = y[p], b = y[p + kPairs];
-        y[p] = a * c.x + b * c.y;
-        y[p + kPairs] = b * c.x - a * c.y;
-      }
-    }
+    uint32_t x[32];
+    load_half(xrow, half, x);
+    load_dy_half<kPairs>(t_lane_col, half, hi, t, row, y);
+    uint32_t o[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = bf2(x[half * 32 + i]);
+      const float2 xh = bf2(x[i]);
       const int d = half * 64 + 2 * i;
       const float g0 = rinv * (y[2 * i] * w[d] - xh.x * rinv * dot);
       const float g1 = rinv * (y[2 * i + 1] * w[d + 1] - xh.y * rinv * dot);
-      dx[half * 32 + i] = pack_bf16x2(g0, g1);
+      o[i] = pack_bf16x2(g0, g1);
+    }
+    if (out) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<uint4*>(out)[8 * half + i] =
+            make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
     }
   }
 }
 
 // One 256-byte row per thread, in 16-byte pieces (rows are 16-byte aligned).
-__device__ __forceinline__ void load_row(const uint16_t* p, uint32_t (&x)[64]) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + i);
-    x[4 * i] = u.x;
-    x[4 * i + 1] = u.y;
-    x[4 * i + 2] = u.z;
-    x[4 * i + 3] = u.w;
-  }
-}
-__device__ __forceinline__ void zero_row(uint32_t (&x)[64]) {
-#pragma unroll
-  for (int i = 0; i < 64; ++i) x[i] = 0u;
-}
 __device__ __forceinline__ void store_row(uint16_t* p, const uint32_t (&x)[64]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i)
@@ -345,13 +348,16 @@ __device__ __forceinline__ void fill_rot_hi(float2 (*hi)[8], int j, const BwdArg
 struct alignas(1024) SmemQ {
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
-  uint8_t q[kTileBytes];   // Q' of the current head, then dS of one key tile
-  uint8_t da[kTileBytes];  // dA of the current head (MMA operand)
+  // Head n works in slot n & 1: Q', then dA, then dS of each key tile, each
+  // written once the MMA reading its predecessor is done; the other slot
+  // receives Q of head n+1 meanwhile.
+  uint8_t slot[2][kTileBytes];
   RotTables rot;
   float2 rot_hi[2][kMaxPairs][8];  // per K slot
   float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
   uint64_t kfull[2], kready[2], kempty[2], vfull[2], vready[2], vempty[2];
-  uint64_t qfull, qempty, qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
+  uint64_t qfull[2], qempty[2];
+  uint64_t qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
   uint64_t tables, drain;
   uint32_t tmem_base;
   int abort;
@@ -384,8 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.vready[i], 128);
       mbar_init(&sm.vempty[i], 1);
     }
-    mbar_init(&sm.qfull, 1);
-    mbar_init(&sm.qempty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.qempty[i], 1);
+    }
     mbar_init(&sm.qready, 128);
     mbar_init(&sm.sfull, 1);
     mbar_init(&sm.pfull, 128);
@@ -465,12 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
       ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
       for (int h = 0; h < a.G && ok; ++h, ++nq) {
-        if (nq > 0 && !wait0(&sm.qempty, (nq - 1) & 1, kSiteQEmpty)) { ok = false; break; }
+        const int b = nq & 1;
+        if (nq >= 2 && !wait0(&sm.qempty[b], ((nq >> 1) - 1) & 1, kSiteQEmpty)) { ok = false; break; }
         if (lane == 0) {
           const int hq = c.kvh * a.G + h;
-          mbar_arrive_expect_tx(&sm.qfull, kTileBytes);
-          tma_load_4d(sm.q, &tm_q, &sm.qfull, 0, hq, c.t * kTile, c.b);
-          tma_load_4d(sm.q + kHalfBytes, &tm_q, &sm.qfull, 64, hq, c.t * kTile, c.b);
+          mbar_arrive_expect_tx(&sm.qfull[b], kTileBytes);
+          tma_load_4d(sm.slot[b], &tm_q, &sm.qfull[b], 0, hq, c.t * kTile, c.b);
+          tma_load_4d(sm.slot[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, c.t * kTile, c.b);
         }
       }
     }
@@ -479,7 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((kused >> s) & 1u) mbar_wait_drain(&sm.kfull[s], ((kpar >> s) & 1u) ^ 1u);
         if ((vused >> s) & 1u) mbar_wait_drain(&sm.vfull[s], ((vpar >> s) & 1u) ^ 1u);
       }
-      if (nq > 0) mbar_wait_drain(&sm.qfull, (nq - 1) & 1);
+      for (int b = 0; b < 2; ++b) {
+        const int cnt = (nq - b + 1) / 2;  // loads issued into slot b
+        if (cnt > 0) mbar_wait_drain(&sm.qfull[b], (cnt - 1) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -513,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + blk * 128, desc_kmajor(sm.q, kk), desc_kmajor(sm.k[blk ? sc : sp], kk),
-                   kIdescKK16, kk > 0);
+            mma_ss(tmem + blk * 128, desc_kmajor(sm.slot[n & 1], kk),
+                   desc_kmajor(sm.k[blk ? sc : sp], kk), kIdescKK16, kk > 0);
         mma_commit(&sm.sfull);
         if (h == 0) {
           if (c.t > 0 && c.u == 0) {
@@ -544,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 256 + blk * 128, desc_kmajor(sm.da, kk),
+            mma_ss(tmem + 256 + blk * 128, desc_kmajor(sm.slot[n & 1], kk),
                    desc_kmajor(sm.v[blk ? sc : sp], kk), kIdescKK16, kk > 0);
         mma_commit(&sm.dpfull);
         // dQ = sum over key tiles of dS K' into columns 128..255
@@ -556,15 +568,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              mma_ss(tmem + 128, desc_kmajor(sm.q, kk), desc_mn(sm.k[blk ? sc : sp], kk),
-                     kIdescKM16, acc);
+              mma_ss(tmem + 128, desc_kmajor(sm.slot[n & 1], kk),
+                     desc_mn(sm.k[blk ? sc : sp], kk), kIdescKM16, acc);
               acc = 1;
             }
             mma_commit(blk == 0 ? &sm.dq0 : &sm.dqfull);
           }
           if (!ok) break;
         }
-        mma_commit(&sm.qempty);
+        mma_commit(&sm.qempty[n & 1]);
         if (h == a.G - 1) {
           if (hp) {
             mma_commit(&sm.kempty[sp]);
@@ -634,8 +646,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       // ---- Q'
-      if (!(ok = warp_wait(&sm.qfull, ph, abort, a.err, kSiteQFull))) break;
-      const float rinv_q = norm_rope_row<kPairs>(sm.q, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
+      uint8_t* slot = sm.slot[n & 1];
+      if (!(ok = warp_wait(&sm.qfull[n & 1], (n >> 1) & 1, abort, a.err, kSiteQFull))) break;
+      const float rinv_q = norm_rope_row<kPairs>(slot, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready);
       const float lse2 = valid_row ? a.lse[lrow] * kLog2e : 0.f;
@@ -682,52 +695,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
       if (valid_row) a.ws_lse[lrow] = a.lse[lrow] + __logf(lsum);
 
-      // ---- A: dg, dA (smem and workspace), D
-      uint32_t gw[64], dow[64];
-      if (valid_row) {
-        load_row(a.g + tok * kHeadDim, gw);
-        load_row(a.dO + tok * kHeadDim, dow);
-      } else {
-        zero_row(gw);
-        zero_row(dow);
+      // ---- A: dg, dA (smem and workspace), D -- 32 dims at a time (a rolled
+      // loop keeps the code small), the next chunk's g and dO loads in flight
+      // while this one is computed (chunk 0's while the PV MMA runs).
+      const uint4* grow = reinterpret_cast<const uint4*>(a.g + tok * kHeadDim);
+      const uint4* dorow = reinterpret_cast<const uint4*>(a.dO + tok * kHeadDim);
+      uint4 gc[4], dc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        gc[i] = valid_row ? __ldg(grow + i) : make_uint4(0u, 0u, 0u, 0u);
+        dc[i] = valid_row ? __ldg(dorow + i) : make_uint4(0u, 0u, 0u, 0u);
       }
       if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
       tc_fence_after();
       float dsum = 0.f;
       {
-        uint32_t dgw[64], daw[64];
-#pragma unroll
+        uint4* dgrow = reinterpret_cast<uint4*>(a.dg + tok * kHeadDim);
+        uint4* darow = reinterpret_cast<uint4*>(a.ws_da + tok * kHeadDim);
+#pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
+          uint4 gn[4], dn[4];
+          const bool more = valid_row && ch + 1 < 4;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gn[i] = more ? __ldg(grow + 4 * (ch + 1) + i) : make_uint4(0u, 0u, 0u, 0u);
+            dn[i] = more ? __ldg(dorow + 4 * (ch + 1) + i) : make_uint4(0u, 0u, 0u, 0u);
+          }
           uint32_t x[32];
           tmem_ld32(t_row + 256 + ch * 32, x);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int wi = ch * 16 + e;
-            const float2 gg = bf2(gw[wi]), dd = bf2(dow[wi]);
-            const float a0 = __uint_as_float(x[2 * e]) * inv_l;
-            const float a1 = __uint_as_float(x[2 * e + 1]) * inv_l;
-            const float s0 = 1.0f / (1.0f + __expf(-gg.x)), s1 = 1.0f / (1.0f + __expf(-gg.y));
-            dgw[wi] = pack_bf16x2(dd.x * a0 * s0 * (1.0f - s0), dd.y * a1 * s1 * (1.0f - s1));
-            in_range &= fabsf(dd.x) <= kF16Max && fabsf(dd.y) <= kF16Max;
-            daw[wi] = pack_f16x2(dd.x * s0, dd.y * s1);
-            const float2 dr = f16x2(daw[wi]);  // D uses the rounded dA the MMAs see
-            dsum += dr.x * a0 + dr.y * a1;
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t gwv[4] = {gc[i].x, gc[i].y, gc[i].z, gc[i].w};
+            const uint32_t dwv[4] = {dc[i].x, dc[i].y, dc[i].z, dc[i].w};
+            uint32_t dgo[4], dao[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 gg = bf2(gwv[e]), dd = bf2(dwv[e]);
+              const float a0 = __uint_as_float(x[8 * i + 2 * e]) * inv_l;
+              const float a1 = __uint_as_float(x[8 * i + 2 * e + 1]) * inv_l;
+              const float s0 = 1.0f / (1.0f + __expf(-gg.x)), s1 = 1.0f / (1.0f + __expf(-gg.y));
+              dgo[e] = pack_bf16x2(dd.x * a0 * s0 * (1.0f - s0), dd.y * a1 * s1 * (1.0f - s1));
+              in_range &= fabsf(dd.x) <= kF16Max && fabsf(dd.y) <= kF16Max;
+              dao[e] = pack_f16x2(dd.x * s0, dd.y * s1);
+              const float2 dr = f16x2(dao[e]);  // D uses the rounded dA the MMAs see
+              dsum += dr.x * a0 + dr.y * a1;
+            }
+            const int c16 = 4 * ch + i;  // 16-byte piece of the row
+            const uint4 da16 = make_uint4(dao[0], dao[1], dao[2], dao[3]);
+            // dA into the MMA operand tile (row-major over dims, 128B swizzle)
+            *reinterpret_cast<uint4*>(slot + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) = da16;
+            if (valid_row) {
+              dgrow[c16] = make_uint4(dgo[0], dgo[1], dgo[2], dgo[3]);
+              darow[c16] = da16;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gc[i] = gn[i];
+            dc[i] = dn[i];
           }
         }
-        // dA into the MMA operand tile (row-major over dims, 128B swizzle)
-#pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16)
-          *reinterpret_cast<uint4*>(sm.da + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) =
-              make_uint4(daw[4 * c16], daw[4 * c16 + 1], daw[4 * c16 + 2], daw[4 * c16 + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.dafull);
-        if (valid_row) {
-          store_row(a.dg + tok * kHeadDim, dgw);
-          store_row(a.ws_da + tok * kHeadDim, daw);
-          a.ws_d[lrow] = dsum;
-        }
+        if (valid_row) a.ws_d[lrow] = dsum;
       }
 
       // ---- dS = scale P (dP - D) per key tile into the Q slot, then dQ
@@ -751,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float d1 = a.scale * inv_l * pp.y * (__uint_as_float(dp[2 * e + 1]) - dsum);
             ds[e] = pack_f16x2(d0, d1);
           }
-          uint8_t* half = sm.q + (pc >> 1) * kHalfBytes;
+          uint8_t* half = slot + (pc >> 1) * kHalfBytes;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             *reinterpret_cast<uint4*>(half + sw_off(row, (pc & 1) * 4 + i)) =
@@ -765,20 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       // ---- dq through RoPE^-1 and the RMSNorm Jacobian
-      uint32_t xq[64];
-      if (valid_row) {
-        load_row(a.q + tok * kHeadDim, xq);
-      } else {
-        zero_row(xq);
-      }
       if (!(ok = warp_wait(&sm.dqfull, ph, abort, a.err, kSiteDQFull))) break;
       tc_fence_after();
-      {
-        uint32_t dx[64];
-        norm_rope_grad<kPairs>(t_row + 128, xq, rinv_q, sm.wq, sm.rot_hi[sc], sm.rot, row, lane,
-                               sm.dw, dx);
-        if (valid_row) store_row(a.dq + tok * kHeadDim, dx);
-      }
+      norm_rope_grad<kPairs>(t_row + 128, valid_row ? a.q + tok * kHeadDim : nullptr, rinv_q,
+                             sm.wq, sm.rot_hi[sc], sm.rot, row, lane, sm.dw,
+                             valid_row ? a.dq + tok * kHeadDim : nullptr);
       tc_fence_before();
       mbar_arrive(&sm.tfree);
       if (++h == a.G) {
@@ -804,13 +827,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 struct alignas(1024) SmemKV {
   uint8_t k[kTileBytes];   // K'_j
   uint8_t v[kTileBytes];   // V_j
-  uint8_t q[kTileBytes];   // Q'_i of the current (query tile, head)
-  uint8_t da[kTileBytes];  // dA_i
+  uint8_t q[2][kTileBytes];   // Q'_i of (query tile, head) pair nq, in buffer nq & 1
+  uint8_t da[2][kTileBytes];  // dA_i
   RotTables rot;
   float2 rot_hi[2][2][kMaxPairs][8];  // [key tile parity][tile j, j+1]
   float lse2[2][kTile], dd[2][kTile];  // per query column, double-buffered
   float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
-  uint64_t kfull, vfull, kvempty, qfull, qempty, qready, staged, sfull, pfull, dkvfull, tfree;
+  uint64_t kfull, vfull, kvempty, qfull[2], qempty[2], qready, staged, sfull, pfull, dkvfull, tfree;
+  uint64_t mmadone;  // dV/dK of the previous pair finished (their TMEM operands are free)
   uint64_t tables, drain;
   uint32_t tmem_base;
   int abort;
@@ -839,10 +863,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.kfull, 2);
     mbar_init(&sm.vfull, 1);
     mbar_init(&sm.kvempty, 1);
-    mbar_init(&sm.qfull, 1);
-    mbar_init(&sm.qempty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.qempty[i], 1);
+    }
     mbar_init(&sm.qready, 128);
     mbar_init(&sm.staged, 128);
+    mbar_init(&sm.mmadone, 1);
     mbar_init(&sm.sfull, 1);
     mbar_init(&sm.pfull, 128);
     mbar_init(&sm.dkvfull, 1);
@@ -903,14 +930,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&sm.kfull);
       const int ni = n_iters(c);
       for (int i = 0; i < ni && ok; ++i, ++nq) {
-        if (nq > 0 && !(ok = wait0(&sm.qempty, (nq - 1) & 1, kSiteQEmpty))) break;
+        const int b = nq & 1;
+        if (nq >= 2 && !(ok = wait0(&sm.qempty[b], ((nq >> 1) - 1) & 1, kSiteQEmpty))) break;
         if (lane == 0) {
           const int qt = c.t + i / a.G, hq = c.kvh * a.G + i % a.G;
-          mbar_arrive_expect_tx(&sm.qfull, 2 * kTileBytes);
-          tma_load_4d(sm.q, &tm_q, &sm.qfull, 0, hq, qt * kTile, c.b);
-          tma_load_4d(sm.q + kHalfBytes, &tm_q, &sm.qfull, 64, hq, qt * kTile, c.b);
-          tma_load_4d(sm.da, &tm_da, &sm.qfull, 0, hq, qt * kTile, c.b);
-          tma_load_4d(sm.da + kHalfBytes, &tm_da, &sm.qfull, 64, hq, qt * kTile, c.b);
+          mbar_arrive_expect_tx(&sm.qfull[b], 2 * kTileBytes);
+          tma_load_4d(sm.q[b], &tm_q, &sm.qfull[b], 0, hq, qt * kTile, c.b);
+          tma_load_4d(sm.q[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, qt * kTile, c.b);
+          tma_load_4d(sm.da[b], &tm_da, &sm.qfull[b], 0, hq, qt * kTile, c.b);
+          tma_load_4d(sm.da[b] + kHalfBytes, &tm_da, &sm.qfull[b], 64, hq, qt * kTile, c.b);
         }
       }
     }
@@ -920,7 +948,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(&sm.kfull, (nkv - 1) & 1);
         mbar_wait_drain(&sm.vfull, (nkv - 1) & 1);
       }
-      if (nq > 0) mbar_wait_drain(&sm.qfull, (nq - 1) & 1);
+      for (int b = 0; b < 2; ++b) {
+        const int cnt = (nq - b + 1) / 2;  // loads issued into buffer b
+        if (cnt > 0) mbar_wait_drain(&sm.qfull[b], (cnt - 1) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -937,6 +968,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ni = n_iters(c);
         for (int i = 0; i < ni && ok; ++i, ++nq) {
           if (!W(&sm.qready, nq & 1, kSiteQReady)) break;
+          // S^T of this pair overwrites the columns dV of the previous pair
+          // reads as its A operand: start it only once that MMA is done.
+          if (nq > 0 && !W(&sm.mmadone, (nq - 1) & 1, kSiteMmaDone)) break;
           if (i == 0) {
             if (!W(&sm.vfull, it & 1, kSiteVFull)) break;
             if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
@@ -945,22 +979,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S^T = K' Q'^T (columns 256..383), dP^T = V dA^T (384..511)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 256, desc_kmajor(sm.k, kk), desc_kmajor(sm.q, kk), kIdescKK16, kk > 0);
+            mma_ss(tmem + 256, desc_kmajor(sm.k, kk), desc_kmajor(sm.q[nq & 1], kk), kIdescKK16,
+                   kk > 0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 384, desc_kmajor(sm.v, kk), desc_kmajor(sm.da, kk), kIdescKK16, kk > 0);
+            mma_ss(tmem + 384, desc_kmajor(sm.v, kk), desc_kmajor(sm.da[nq & 1], kk), kIdescKK16,
+                   kk > 0);
           mma_commit(&sm.sfull);
           if (!W(&sm.pfull, nq & 1, kSitePFull)) break;
           tc_fence_after();
           // dV += P^T dA (0..127), dK += dS^T Q' (128..255)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem, tmem + 256 + kk * 8, desc_mn(sm.da, kk), kIdescKM16, (i > 0 || kk > 0));
+            mma_ts(tmem, tmem + 256 + kk * 8, desc_mn(sm.da[nq & 1], kk), kIdescKM16,
+                   (i > 0 || kk > 0));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 128, tmem + 384 + kk * 8, desc_mn(sm.q, kk), kIdescKM16,
+            mma_ts(tmem + 128, tmem + 384 + kk * 8, desc_mn(sm.q[nq & 1], kk), kIdescKM16,
                    (i > 0 || kk > 0));
-          mma_commit(&sm.qempty);
+          mma_commit(&sm.qempty[nq & 1]);
+          mma_commit(&sm.mmadone);
         }
         if (!ok) break;
         mma_commit(&sm.dkvfull);
@@ -1003,8 +1041,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hq = c.kvh * a.G + i % a.G;
         const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // this thread's query row
         // ---- Q'_i, and lse / D of its rows for the column-wise softmax
-        if (!(ok = warp_wait(&sm.qfull, nq & 1, abort, a.err, kSiteQFull))) break;
-        norm_rope_row<kPairs>(sm.q, row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
+        if (!(ok = warp_wait(&sm.qfull[nq & 1], (nq >> 1) & 1, abort, a.err, kSiteQFull))) break;
+        norm_rope_row<kPairs>(sm.q[nq & 1], row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
         const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + qpos;
         sm.lse2[nq & 1][row] = qpos < a.T ? a.ws_lse[lrow] * kLog2e : 0.f;
         sm.dd[nq & 1][row] = qpos < a.T ? a.ws_d[lrow] : 0.f;
@@ -1057,20 +1095,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j
       const long long krow = (static_cast<long long>(c.b) * a.T + kpos) * a.Hkv + c.kvh;
-      uint32_t xk[64];
-      if (kpos < a.T) {
-        load_row(a.k + krow * kHeadDim, xk);
-      } else {
-        zero_row(xk);
-      }
       if (!(ok = warp_wait(&sm.dkvfull, it & 1, abort, a.err, kSiteDKVFull))) break;
       tc_fence_after();
-      {
-        uint32_t dx[64];
-        norm_rope_grad<kPairs>(t_row + 128, xk, rinv_k, sm.wk, sm.rot_hi[it & 1][0], sm.rot, row,
-                               lane, sm.dw, dx);
-        if (kpos < a.T) store_row(a.dk + krow * kHeadDim, dx);
-      }
+      norm_rope_grad<kPairs>(t_row + 128, kpos < a.T ? a.k + krow * kHeadDim : nullptr, rinv_k,
+                             sm.wk, sm.rot_hi[it & 1][0], sm.rot, row, lane, sm.dw,
+                             kpos < a.T ? a.dk + krow * kHeadDim : nullptr);
       {
         uint32_t dv[64];
 #pragma unroll
