@@ -459,16 +459,35 @@ def decode_bench(swa, args, world, device, stream, peaks):
 
 
 def run_profile(args, device):
-    """Warmup + steps launches of swa_fwd on the layer-shape workload, nothing
-    else, so that a profiler sees a short, predictable launch list."""
+    """Warmup + steps calls of one entry point, nothing else, so that a
+    profiler sees a short, predictable launch list: `fwd` on the layer-shape
+    workload, `decode` on one layer of the decode workload, `bwd` (with the
+    forward that produces its lse) on the training shape."""
     import hybrid_sliding_window_gated_b200 as swa
-    cfg = workloads.LAYER
-    fns, _ = fwd_workload(swa, cfg, device)
+    which = args.profile
+    if which == "fwd":
+        cfg = workloads.LAYER
+        fns, _ = fwd_workload(swa, cfg, device)
+    elif which == "decode":
+        cfg = workloads.DECODE
+        x = workloads.decode_layer_inputs(cfg, 0, device=device)
+        o = torch.empty_like(x["q"])
+        fns = [lambda: swa.decode_step(x["pos"], x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"],
+                                       x["k_cache"], x["v_cache"], rot_dim=cfg.R,
+                                       rope_base=cfg.base, eps=cfg.eps, out=o)]
+    else:
+        cfg = workloads.TRAIN
+        d = workloads.prefill_inputs(cfg, device=device, with_grad_out=True)
+        o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], rope_base=cfg.base,
+                         want_lse=True)
+        fns = [lambda: swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"],
+                               rope_base=cfg.base)]
     for i in range(args.warmup + args.steps):
         fns[i % len(fns)]()
     torch.cuda.synchronize()
     code, site = swa.get_last_device_error()
-    return {"profile": cfg.name, "launches": args.warmup + args.steps, "device_error": code}
+    return {"profile": cfg.name, "entry": which, "launches": args.warmup + args.steps,
+            "device_error": code}
 
 
 def run_reference(args, rank, world):
@@ -514,8 +533,8 @@ def main():
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true",
-                    help="only warmup + steps launches of the headline kernel (for ncu)")
+    ap.add_argument("--profile", choices=["fwd", "decode", "bwd"], default=None,
+                    help="only warmup + steps calls of one entry point (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -536,7 +555,7 @@ def main():
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
                                              device_id=device)
-    if args.profile:
+    if args.profile is not None:
         line = run_profile(args, device)
     else:
         line = run_swa(args, rank, world, device)
