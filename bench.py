@@ -180,6 +180,23 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- timing
 
+def max_over_ranks(ms, world):
+    """The slowest rank's device time: every rank takes part (same collective
+    in every rank's sequence); the tensor lives where the backend wants it."""
+    if world <= 1:
+        return ms
+    on_gpu = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, world, steps, ms):
+    """Whole-job units per second: every rank processed `units_per_rank` per
+    step (weak scaling), timed by the slowest rank."""
+    return units_per_rank * world * steps / (ms / 1e3)
+
+
 def timed_loop(step_fns, steps, warmup, stream, world, sampler=None, per_launch=None):
     """Run warmup steps, then time `steps` steps between barriers on `stream`.
 
@@ -211,11 +228,7 @@ def timed_loop(step_fns, steps, warmup, stream, world, sampler=None, per_launch=
         ev1.record(stream)
     torch.cuda.synchronize()
     t1 = time.perf_counter()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
     per = None
     if launch_evs:
         per = sum(a.elapsed_time(b) for a, b in launch_evs) / len(launch_evs)
@@ -314,8 +327,7 @@ def run_swa(args, rank, world, device):
     clocks = sampler.summary(t0, t1)
 
     tokens_per_rank = cfg.B * cfg.T
-    total_tokens = tokens_per_rank * world * args.steps
-    value = total_tokens / (ms / 1e3)
+    value = aggregate_throughput(tokens_per_rank, world, args.steps, ms)
     bytes_launch = FWD_BYTES_PER_TOKEN(cfg) * tokens_per_rank
     achieved = bytes_launch / (per_launch_ms / 1e3) / 1e9
     traffic = committed_traffic("swa_fwd_kernel_layer_shape.txt", ["fwd.cu", "ptx.cuh", "swa_internal.h"])
