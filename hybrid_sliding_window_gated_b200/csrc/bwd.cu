@@ -28,6 +28,7 @@
 #include <cuda_fp16.h>
 
 #include "bwd_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace swa {
@@ -376,11 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
   int n_tiles = u1 - u0;
 
-  if (tid < kHeadDim) {
-    sm.wq[tid] = a.wq[tid];
-    sm.wk[tid] = a.wk[tid];
-    sm.dw[tid] = 0.f;
-  }
+  if (tid < kHeadDim) sm.dw[tid] = 0.f;
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.kfull[i], 2);
@@ -412,6 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
+  }
+  // A programmatic dependent of the previous kernel on the stream: every
+  // global access below (the weights included) waits for it to complete.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid < kHeadDim) {
+    sm.wq[tid] = a.wq[tid];
+    sm.wk[tid] = a.wk[tid];
   }
   tc_fence_before();
   __syncthreads();
@@ -854,11 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
   int n_tiles = u1 - u0;
 
-  if (tid < kHeadDim) {
-    sm.wq[tid] = a.wq[tid];
-    sm.wk[tid] = a.wk[tid];
-    sm.dw[tid] = 0.f;
-  }
+  if (tid < kHeadDim) sm.dw[tid] = 0.f;
   if (tid == 0) {
     mbar_init(&sm.kfull, 2);
     mbar_init(&sm.vfull, 1);
@@ -882,6 +883,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
+  }
+  // A programmatic dependent of the previous kernel on the stream: every
+  // global access below (the weights included) waits for it to complete.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid < kHeadDim) {
+    sm.wq[tid] = a.wq[tid];
+    sm.wk[tid] = a.wk[tid];
   }
   tc_fence_before();
   __syncthreads();
@@ -1147,12 +1156,11 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
-  swa_bwd_q_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem_q, stream>>>(tq, tk, tv, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return map_cuda_error(e);
-  swa_bwd_kv_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem_kv, stream>>>(tq, tk, tv,
-                                                                                     tda, a);
-  return map_cuda_error(cudaGetLastError());
+  int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreads,
+                            smem_q, stream, tq, tk, tv, a);
+  if (rc != SWA_OK) return rc;
+  return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem_kv,
+                          stream, tq, tk, tv, tda, a);
 }
 
 }  // namespace bwd

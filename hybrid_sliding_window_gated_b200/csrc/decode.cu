@@ -22,6 +22,7 @@
 // row, in shared memory and in the ring, with k' (rounded to bf16) and v_new
 // before reading it.
 #include "decode_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 #include "warp_mma.cuh"
 
@@ -395,17 +396,8 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a
   }
   const long long units = static_cast<long long>(a.N) * a.Hkv;
   const long long grid = units < di.num_sms ? units : di.num_sms;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(dec::kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddepcontrol
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return map_cuda_error(cudaLaunchKernelEx(&cfg, dec::swa_decode_kernel, tk, tv, a));
+  return launch_dependent(dec::swa_decode_kernel, static_cast<unsigned>(grid), dec::kThreads, smem,
+                          stream, tk, tv, a);
 }
 
 }  // namespace swa

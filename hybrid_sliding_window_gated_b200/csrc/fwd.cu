@@ -62,6 +62,7 @@
 // product of a per-tile table rot((128 j + 16 a) w), a in 0..7, computed by the
 // producer's lanes for each K tile (fp64 range reduction, then sincosf), and a
 // per-CTA table rot(b w), b in 0..15.
+#include "launch.cuh"
 #include "ptx.cuh"
 #include "swa_internal.h"
 
@@ -319,12 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = u1 - u0;
   const int n_heads = n_tiles * a.G;
 
-  if (tid < kHeadDim) {
-    const float wq = a.wq[tid], wk = a.wk[tid];
-    sm.wq[tid] = wq;
-    sm.wk[tid] = wk;
-    sm.wkq[tid] = wk * wq;
-  }
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.kfull[i], 2);  // the copy's expect_tx arrive + the rotation table
@@ -357,6 +352,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
+  }
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: the set-up above overlapped its tail; every global read or write
+  // below (the weights included) waits for it to complete.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid < kHeadDim) {
+    const float wq = a.wq[tid], wk = a.wk[tid];
+    sm.wq[tid] = wq;
+    sm.wk[tid] = wk;
+    sm.wkq[tid] = wk * wq;
   }
   tc_fence_before();
   __syncthreads();
@@ -785,9 +791,8 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
-  swa_fwd_kernel<kPairs><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, tg,
-                                                                                 to, a);
-  return map_cuda_error(cudaGetLastError());
+  return launch_dependent(swa_fwd_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem,
+                          stream, tq, tk, tv, tg, to, a);
 }
 
 }  // namespace fwd
