@@ -114,12 +114,12 @@ def bwd_workspace_size(B, T, Hq, Hkv, *, head_dim=128, window=128, rot_dim=42):
 
 
 def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
-        scale=0.0, workspace=None, grads=None, stream=None):
+        scale=0.0, workspace=None, grads=None, flags=0, stream=None):
     """Gradients (dq, dk, dv, dg, dwq, dwk) of sum(o * dO) for the forward above."""
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
-                    rope_base=rope_base, eps=eps, scale=scale)
+                    rope_base=rope_base, eps=eps, scale=scale, flags=flags)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g),
                  torch.zeros(D, dtype=torch.float32, device=q.device),
@@ -155,14 +155,14 @@ def bwd_noalloc(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_bas
 
 
 def decode_step(pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, *, rot_dim=42, rope_base=1e7,
-                eps=1e-6, scale=0.0, out=None, stream=None):
+                eps=1e-6, scale=0.0, out=None, flags=0, stream=None):
     """One decode step; updates the [N,Hkv,128,128] rings in place, returns o [N,Hq,128]."""
     N, Hq, D = q.shape
     Hkv, W = k_cache.shape[1], k_cache.shape[2]
     if out is None:
         out = torch.empty_like(q)
     p = make_params(N, 1, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
-                    eps=eps, scale=scale)
+                    eps=eps, scale=scale, flags=flags)
     rc = lib().swa_decode_step(ctypes.byref(p), _ptr(pos), _ptr(q), _ptr(k_new), _ptr(v_new),
                                _ptr(g), _ptr(wq), _ptr(wk), _ptr(k_cache), _ptr(v_cache), _ptr(out),
                                _stream(stream))

@@ -245,6 +245,7 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
   a.total_tiles = static_cast<long long>(a.tiles_per_chain) * p->B * p->Hkv;
   a.scale = score_scale(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.flags = p->flags;
   a.eps = p->eps;
   a.q = q;
   a.k = k;
@@ -320,6 +321,7 @@ int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t*
   a.Hkv = p->Hkv;
   a.G = p->Hq / p->Hkv;
   a.half_rot = p->rot_dim / 2;
+  a.flags = p->flags;
   a.scale_log2 = score_scale(p) * 1.4426950408889634f;
   a.eps = p->eps;
   a.pos = pos;

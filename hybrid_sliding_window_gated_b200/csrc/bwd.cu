@@ -43,7 +43,7 @@ enum Site {
   kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
   kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
   kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged,
-  kSiteMmaDone
+  kSiteMmaDone, kSiteForced
 };
 
 // ---------------------------------------------------------------- helpers
@@ -359,7 +359,7 @@ struct alignas(1024) SmemQ {
   uint64_t kfull[2], kready[2], kempty[2], vfull[2], vready[2], vempty[2];
   uint64_t qfull[2], qempty[2];
   uint64_t qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
-  uint64_t tables, drain;
+  uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
   uint32_t tmem_base;
   int abort;
 };
@@ -403,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.tfree, 128);
     mbar_init(&sm.tables, 128);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.never, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -511,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
         return ok;
       };
+      if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
       for (int n = 0; n < n_heads && ok; ++n) {
         const uint32_t ph = n & 1;
         const bool hp = c.t > 0;
@@ -840,7 +842,7 @@ struct alignas(1024) SmemKV {
   float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
   uint64_t kfull, vfull, kvempty, qfull[2], qempty[2], qready, staged, sfull, pfull, dkvfull, tfree;
   uint64_t mmadone;  // dV/dK of the previous pair finished (their TMEM operands are free)
-  uint64_t tables, drain;
+  uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
   uint32_t tmem_base;
   int abort;
 };
@@ -877,6 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.tfree, 128);
     mbar_init(&sm.tables, 128);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.never, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -972,6 +975,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
         return ok;
       };
+      if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
       Cursor c = cursor_at(a, u0);
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
         const int ni = n_iters(c);

@@ -11,6 +11,7 @@ struct BwdArgs {
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   float eps;
+  int flags;  // SWA_FLAG_* debug bits (0 in normal use)
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* g;

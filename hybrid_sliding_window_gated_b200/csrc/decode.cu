@@ -56,6 +56,7 @@ struct alignas(1024) Smem {
   Stage st[kStages];
   Group grp[kGroups];
   uint64_t full[kStages], empty[kStages];
+  uint64_t never;  // completed by nothing: SWA_FLAG_FORCE_TIMEOUT waits on it
   int abort;
 };
 // The partial outputs [4 warps][G heads][kOStride] reuse a stage's K ring once
@@ -63,7 +64,7 @@ struct alignas(1024) Smem {
 static_assert(4 * kDecMaxGroup * kOStride * 4 <= 2 * kHalfBytes, "partial O does not fit");
 static_assert(sizeof(Smem) + 1024 <= 232448, "decode shared memory");
 
-enum Site { kSiteFull = 0x40, kSiteEmpty, kSiteGroup };
+enum Site { kSiteFull = 0x40, kSiteEmpty, kSiteGroup, kSiteForced };
 
 // Byte offset of 16-byte chunk c (0..15) of slot row s in a [half][slot][64]
 // 128B-swizzled ring tile.
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.full[s], 2);  // the copies' expect_tx arrive + the position
       mbar_init(&sm.empty[s], 1);
     }
+    mbar_init(&sm.never, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -364,7 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------- consumer group
     const int gi = (warp - 1) >> 2, lw = (warp - 1) & 3;
-    for (int i = gi; i < n_units; i += kGroups) {
+    bool live = true;
+    if (a.flags & SWA_FLAG_FORCE_TIMEOUT)  // a wait that runs out, for the tests
+      live = group_and(mbar_wait(&sm.never, 0, abort, a.err, kSiteForced), 1 + gi);
+    for (int i = gi; live && i < n_units; i += kGroups) {
       const int s = i % kStages;
       const bool got = mbar_wait(&sm.full[s], (i / kStages) & 1, abort, a.err, kSiteFull);
       if (!group_and(got, 1 + gi)) break;  // the same decision on the whole group

@@ -9,6 +9,7 @@ constexpr int kDecMaxGroup = 8;  // query heads per KV head the decode kernel ta
 struct DecArgs {
   int N, Hq, Hkv, G;
   int half_rot;      // rot_dim / 2 rotated pairs
+  int flags;         // SWA_FLAG_* debug bits (0 in normal use)
   float scale_log2;  // softmax scale * log2(e)
   float eps;
   const int64_t* pos;

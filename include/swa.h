@@ -69,8 +69,9 @@ enum {
 };
 
 /* Debug bits for swa_params_t.flags (0 in normal use).  FORCE_TIMEOUT makes
- * the kernel wait on a barrier that nothing completes, so tests can check
- * that the bounded wait ends the kernel and reports SWA_ERR_DEVICE_TIMEOUT. */
+ * the kernels of swa_fwd, swa_bwd and swa_decode_step wait on a barrier that
+ * nothing completes, so tests can check that the bounded wait ends the kernel
+ * (its copies drained, TMEM freed) and reports SWA_ERR_DEVICE_TIMEOUT. */
 enum { SWA_FLAG_FORCE_TIMEOUT = 1 };
 
 typedef struct swa_params {

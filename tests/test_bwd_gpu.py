@@ -112,3 +112,16 @@ def test_weights_beyond_fp16_operands_are_reported():
     assert swa.get_last_device_error()[0] == swa.ERR_INVALID_ARG
     # the context still computes correct gradients afterwards
     check_bwd(workloads.TINY)
+
+
+def test_forced_timeout_is_reported_and_context_survives():
+    cfg, d = _small_inputs()
+    o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], want_lse=True)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"],
+            flags=swa.FLAG_FORCE_TIMEOUT)
+    code, site = swa.get_last_device_error()
+    assert code == swa.ERR_DEVICE_TIMEOUT and site >= 0x100
+    assert swa.get_last_device_error()[0] == swa.OK
+    check_bwd(workloads.TINY)

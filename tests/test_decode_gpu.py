@@ -126,3 +126,20 @@ def test_saturated_gate_gives_zero():
     o = swa.decode_step(inp["pos"], inp["q"], inp["k"], inp["v"], inp["g"], inp["wq"], inp["wk"],
                         inp["k_cache"], inp["v_cache"], rope_base=cfg.base)
     assert torch.count_nonzero(o).item() == 0
+
+
+def test_forced_timeout_is_reported_and_context_survives():
+    """A wait that nothing completes ends by its time limit; the kernel drains
+    its copies, reports the site, and the next call computes correctly."""
+    cfg = workloads.Decode("decode test", N=5, layers=1, Hq=8, Hkv=2, base=1e4, seed=14)
+    inp = workloads.decode_layer_inputs(cfg, layer=0)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    assert swa.get_last_device_error()[0] == swa.OK
+    kc, vc = d["k_cache"].clone(), d["v_cache"].clone()
+    swa.decode_step(d["pos"], d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], kc, vc,
+                    rope_base=cfg.base, flags=swa.FLAG_FORCE_TIMEOUT)
+    code, site = swa.get_last_device_error()
+    assert code == swa.ERR_DEVICE_TIMEOUT and site >= 0x100
+    assert swa.get_last_device_error()[0] == swa.OK
+    o, kc2, vc2, o_ref, kc_ref, vc_ref = run_both(inp, 42, cfg.base)
+    assert_parity(to_f64(o), o_ref, "decode o after a forced timeout")

@@ -125,3 +125,8 @@ def test_forced_timeout_is_reported_and_context_survives():
     assert code == swa.ERR_DEVICE_TIMEOUT and site >= 0x100
     assert swa.get_last_device_error()[0] == swa.OK  # cleared
     check_full(cfg)  # the context is still usable and results are right
+
+
+def test_training_shape_forward_full():
+    """The 1 x 16384 training shape, every output element against the oracle."""
+    check_full(workloads.TRAIN)
