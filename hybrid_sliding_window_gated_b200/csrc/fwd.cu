@@ -29,13 +29,15 @@
 //               One thread per row throughout, so 1/rms(q) and 1/l stay in
 //               registers.
 //
-// Q slot reuse.  Region r owns Q slot r.  Once QK^T(n) has read Q(n), the slot
-// receives the gate tile g(n) by TMA (it lands while the softmax runs); the
-// epilogue overwrites it in place with o(n), which leaves by TMA store; then
-// Q(n+2) is loaded into the slot.  All bulk global traffic (q, k, v, g in; o
-// out) thus moves by TMA: the load/store unit touches only shared memory,
-// since a row-per-thread pattern on global memory touches 32 cache lines per
-// warp instruction.
+// Q slots.  Head n uses slot n % 3 of three.  The producer loads Q(n) there
+// once the o store of head n-3 has read the slot; once QK^T(n) has read Q(n),
+// the slot receives the gate tile g(n) by TMA (it lands while the softmax
+// runs); the epilogue overwrites it in place with o(n), which leaves by TMA
+// store, and the slot goes back to the producer.  With two heads in flight the
+// third slot holds the next Q, so a region never waits for its Q load.  All
+// bulk global traffic (q, k, v, g in; o out) moves by TMA: the load/store
+// unit touches only shared memory, since a row-per-thread pattern on global
+// memory touches 32 cache lines per warp instruction.
 //
 // TMEM (512 columns) holds two regions of 256 columns.  For a head in region
 // r: S = Q [K_{t-1} K_t]^T fills all 256 columns (fp32); the softmax writes P
@@ -84,28 +86,27 @@ constexpr int kTileBytes = 2 * kHalfBytes;  // a full 128 x 128 bf16 tile
 struct alignas(1024) Smem {
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
-  uint8_t q[2][kTileBytes];
-  float2 rot_lo[kMaxPairs][16];        // rot(b * w_p), b = 0..15
-  float2 rot_hi[2][kMaxPairs][8];      // rot((128 j + 16 a) * w_p) per K slot
+  uint8_t q[3][kTileBytes];  // head n uses slot n % 3: Q(n), then g(n), then o(n)
+  float2 rot_tile[2][kMaxPairs];  // rot(128 j * w_p) of the K tile in each slot
   float wq[kHeadDim];
   float wk[kHeadDim];
-  float wkq[kHeadDim];    // wk * wq, for the K dims that RoPE leaves alone
   uint64_t kfull[2], kready[2], kempty[2];
   uint64_t vfull[2], vempty[2];
-  uint64_t qfull[2], qready[2];
+  uint64_t qfull[3], qready[2];
   uint64_t sfull[2], pfull[2], ofull[2], tfree[2];
-  uint64_t gfull[2], ostore[2];  // gate tile landed / o written, per region
-  uint64_t tables, drain, never;
+  uint64_t gfull[3], ostore[2];  // gate tile landed (per slot) / o written (per region)
+  uint64_t slotfree[3];          // the o store has read the slot: it may take the next Q
+  uint64_t drain, never;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory over the 227 KiB per-CTA limit");
+static_assert(sizeof(Smem) <= 232448, "shared memory over the 227 KiB per-CTA limit");
 
 // Wait-site ids reported through the device error word.
 enum Site {
   kSiteKEmpty = 1, kSiteVEmpty, kSiteOStore, kSiteKFull, kSiteQFull, kSiteKReady,
   kSiteQReady, kSiteTFree, kSiteVFull, kSitePFull, kSiteSFull, kSiteOFull, kSiteForced,
-  kSiteTables, kSiteGFull
+  kSiteGFull, kSiteSlotFree, kSiteAlign
 };
 
 // Position inside a CTA's contiguous run of tiles, advanced without division.
@@ -172,10 +173,11 @@ __device__ __forceinline__ float2 cmul(float2 x, float2 y) {
   return make_float2(x.x * y.x - x.y * y.y, x.x * y.y + x.y * y.x);
 }
 
-// Rotation (cos, sin) of position 128 j + row for pair p, from the tables.
-__device__ __forceinline__ float2 rot_at(const Smem& sm, int kslot, int p, int row) {
-  return cmul(sm.rot_hi[kslot][p][row >> 4], sm.rot_lo[p][row & 15]);
-}
+// Number of rotation factors a thread keeps (at least one, so the array exists).
+template <int kPairs>
+struct RowRot {
+  float2 r[kPairs > 0 ? kPairs : 1];  // rot(row * w_p): fixed per thread
+};
 
 // Sum of squares of a 128-element bf16 row held in two swizzled halves.
 __device__ __forceinline__ float row_sumsq(const uint8_t* h0, const uint8_t* h1, int row) {
@@ -198,10 +200,11 @@ __device__ __forceinline__ float row_sumsq(const uint8_t* h0, const uint8_t* h1,
 
 // Rotate the first 2*kPairs dims of a row in place: y = R(x * scale * wr),
 // rotate-half pairs (p, p + kPairs).  Dims of the rotated chunks beyond
-// 2*kPairs are multiplied by scale * wo, or left as they are (kKeepOthers).
+// 2*kPairs are multiplied by scale * wo * wo2, or left as they are (kKeepOthers).
 template <int kPairs, bool kKeepOthers>
 __device__ __forceinline__ void rope_chunks(uint8_t* h0, int row, float scale, const float* wr,
-                                            const float* wo, const Smem& sm, int kslot) {
+                                            const float* wo, const float* wo2, const float2* rtile,
+                                            const RowRot<kPairs>& rr) {
   constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
   float x[kRopeChunks * 8];
 #pragma unroll
@@ -216,10 +219,10 @@ __device__ __forceinline__ void rope_chunks(uint8_t* h0, int row, float scale, c
   }
 #pragma unroll
   for (int d = 2 * kPairs; d < kRopeChunks * 8; ++d)
-    if (!kKeepOthers) x[d] = x[d] * scale * wo[d];
+    if (!kKeepOthers) x[d] = x[d] * scale * wo[d] * wo2[d];
 #pragma unroll
   for (int p = 0; p < kPairs; ++p) {
-    const float2 t = rot_at(sm, kslot, p, row);
+    const float2 t = cmul(rtile[p], rr.r[p]);  // rot((128 j + row) w_p)
     const float u = x[p] * scale * wr[p];
     const float v = x[p + kPairs] * scale * wr[p + kPairs];
     x[p] = u * t.x - v * t.y;            // x_p cos - x_{p+P} sin
@@ -230,17 +233,21 @@ __device__ __forceinline__ void rope_chunks(uint8_t* h0, int row, float scale, c
     *reinterpret_cast<uint4*>(h0 + sw_off(row, c)) = pack8(x + 8 * c);
 }
 
-// Scale dims [8*c0, 128) of a row in place by scale * w[d] (f32x2 math).
+// Scale dims [8*c0, 128) of a row in place by scale * w[d] * w2[d] (f32x2 math).
 __device__ __forceinline__ void scale_chunks(uint8_t* h0, uint8_t* h1, int row, int c0,
-                                             float scale, const float* w) {
+                                             float scale, const float* w, const float* w2) {
   const float2 sc = make_float2(scale, scale);
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     if (c < c0) continue;
     uint8_t* p = (c < 8 ? h0 : h1) + sw_off(row, c & 7);
     const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const float4 wa = *reinterpret_cast<const float4*>(w + 8 * c);
-    const float4 wb = *reinterpret_cast<const float4*>(w + 8 * c + 4);
+    const float4 wa1 = *reinterpret_cast<const float4*>(w + 8 * c);
+    const float4 wb1 = *reinterpret_cast<const float4*>(w + 8 * c + 4);
+    const float4 wa2 = *reinterpret_cast<const float4*>(w2 + 8 * c);
+    const float4 wb2 = *reinterpret_cast<const float4*>(w2 + 8 * c + 4);
+    const float4 wa = make_float4(wa1.x * wa2.x, wa1.y * wa2.y, wa1.z * wa2.z, wa1.w * wa2.w);
+    const float4 wb = make_float4(wb1.x * wb2.x, wb1.y * wb2.y, wb1.z * wb2.z, wb1.w * wb2.w);
     const float2 y0 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.x), make_float2(wa.x, wa.y)), sc);
     const float2 y1 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.y), make_float2(wa.z, wa.w)), sc);
     const float2 y2 = __fmul2_rn(__fmul2_rn(bf16x2_to_f2(u.z), make_float2(wb.x, wb.y)), sc);
@@ -258,24 +265,25 @@ __device__ __forceinline__ void scale_chunks(uint8_t* h0, uint8_t* h1, int row, 
 // elsewhere].
 template <int kPairs>
 __device__ __forceinline__ void transform_k_row(uint8_t* tile, int row, const Smem& sm, int kslot,
-                                                float eps) {
+                                                const RowRot<kPairs>& rr, float eps) {
   uint8_t* h0 = tile;
   uint8_t* h1 = tile + kHalfBytes;
   const float rinv = rsqrtf(row_sumsq(h0, h1, row) * (1.0f / kHeadDim) + eps);
   constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
   if constexpr (kRopeChunks > 0)
-    rope_chunks<kPairs, false>(h0, row, rinv, sm.wk, sm.wkq, sm, kslot);
-  scale_chunks(h0, h1, row, kRopeChunks, rinv, sm.wkq);
+    rope_chunks<kPairs, false>(h0, row, rinv, sm.wk, sm.wk, sm.wq, sm.rot_tile[kslot], rr);
+  scale_chunks(h0, h1, row, kRopeChunks, rinv, sm.wk, sm.wq);
 }
 
 // Q row: q'' = [RoPE(q * wq) on the rotated dims; q unchanged elsewhere].
 // Returns 1/rms(q), which the softmax applies to the scores.
 template <int kPairs>
 __device__ __forceinline__ float transform_q_row(uint8_t* tile, int row, const Smem& sm,
-                                                 int kslot, float eps) {
+                                                 int kslot, const RowRot<kPairs>& rr, float eps) {
   const float rinv = rsqrtf(row_sumsq(tile, tile + kHalfBytes, row) * (1.0f / kHeadDim) + eps);
   constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
-  if constexpr (kRopeChunks > 0) rope_chunks<kPairs, true>(tile, row, 1.0f, sm.wq, sm.wq, sm, kslot);
+  if constexpr (kRopeChunks > 0)
+    rope_chunks<kPairs, true>(tile, row, 1.0f, sm.wq, sm.wq, sm.wq, sm.rot_tile[kslot], rr);
   return rinv;
 }
 
@@ -308,12 +316,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                    const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                      ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];  // 128B-swizzled tiles need 1 KiB
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (smem_u32(smem_raw) & 1023u) {  // the layout above assumes the alignment; never copy into it otherwise
+    if (tid == 0) atomicCAS(a.err, 0, kDevErrTimeoutBase + kSiteAlign);
+    return;
+  }
 
   const int u0 = static_cast<int>(a.total_tiles * blockIdx.x / gridDim.x);
   const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
@@ -327,16 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kempty[i], 1);
       mbar_init(&sm.vfull[i], 1);
       mbar_init(&sm.vempty[i], 1);
-      mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qready[i], 128);
       mbar_init(&sm.sfull[i], 1);
       mbar_init(&sm.pfull[i], 128);
       mbar_init(&sm.ofull[i], 1);
       mbar_init(&sm.tfree[i], 128);
-      mbar_init(&sm.gfull[i], 1);
       mbar_init(&sm.ostore[i], 128);
     }
-    mbar_init(&sm.tables, 128);
+    for (int i = 0; i < 3; ++i) {  // per Q slot
+      mbar_init(&sm.qfull[i], 1);
+      mbar_init(&sm.gfull[i], 1);
+      mbar_init(&sm.slotfree[i], 1);
+    }
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.never, 1);
     sm.abort = 0;
@@ -362,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float wq = a.wq[tid], wk = a.wk[tid];
     sm.wq[tid] = wq;
     sm.wk[tid] = wk;
-    sm.wkq[tid] = wk * wq;
   }
   tc_fence_before();
   __syncthreads();
@@ -396,12 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(dst + kHalfBytes, map, full, 64, c.kvh, j * kTile, c.b);
         }
         if (is_k) {
-          // rot((128 j + 16 a) w_p) for this tile, then the second arrive on kfull.
-          for (int e = lane; e < kPairs * 8; e += 32) {
-            const int p = e >> 3, ai = e & 7;
+          // rot(128 j w_p) for this tile, then the second arrive on kfull.
+          if (lane < kPairs) {
             float cv, sv;
-            rope_cos_sin(static_cast<double>(j) * kTile + 16.0 * ai, a.inv_freq[p], &cv, &sv);
-            sm.rot_hi[s][p][ai] = make_float2(cv, sv);
+            rope_cos_sin(static_cast<double>(j) * kTile, a.inv_freq[lane], &cv, &sv);
+            sm.rot_tile[s][lane] = make_float2(cv, sv);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(full);
@@ -409,17 +420,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         ring.advance(s);
         return true;
       };
+      // Q(n) goes into slot n % 3 as soon as the o store of head n-3 has read
+      // it, so each region finds its next Q already loaded.
+      int nq = 0;  // Q loads issued
       Cursor c = cursor_at(a, u0);
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
         if (need_prev(c))  // first tile of a run: key tile t-1 as well
           ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
         ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
+        for (int h = 0; h < a.G && ok; ++h) {
+          const int qs = nq % 3;
+          if (nq >= 3 && !wait0(&sm.slotfree[qs], ((nq / 3) - 1) & 1, kSiteSlotFree)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            const int hq = c.kvh * a.G + h;
+            mbar_arrive_expect_tx(&sm.qfull[qs], kTileBytes);
+            tma_load_4d(sm.q[qs], &tm_q, &sm.qfull[qs], 0, hq, c.t * kTile, c.b);
+            tma_load_4d(sm.q[qs] + kHalfBytes, &tm_q, &sm.qfull[qs], 64, hq, c.t * kTile, c.b);
+            tma_prefetch_4d(&tm_g, 0, hq, c.t * kTile, c.b);  // warm L2 for the gate tile
+            tma_prefetch_4d(&tm_g, 64, hq, c.t * kTile, c.b);
+          }
+          ++nq;
+        }
       }
       if (!ok && lane == 0) {
         // Drain the loads this warp issued before the CTA releases its memory.
         for (int s = 0; s < 2; ++s) {
           if (kr.was_used(s)) mbar_wait_drain(&sm.kfull[s], kr.parity(s) ^ 1u);
           if (vr.was_used(s)) mbar_wait_drain(&sm.vfull[s], vr.parity(s) ^ 1u);
+        }
+        for (int s = 0; s < 3; ++s) {
+          const int cntq = (nq - s + 2) / 3;  // Q loads into slot s
+          if (cntq > 0) mbar_wait_drain(&sm.qfull[s], static_cast<uint32_t>(cntq - 1) & 1);
         }
       }
     } else if (warp == 1 && lane == 0) {
@@ -451,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint8_t* kt = sm.k[blk == 0 ? sp : sc];
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(s_base + blk * 128, desc_kmajor(sm.q[r], kk), desc_kmajor(kt, kk), kIdescQK,
+              mma_ss(s_base + blk * 128, desc_kmajor(sm.q[m % 3], kk), desc_kmajor(kt, kk), kIdescQK,
                      kk > 0);
           }
           mma_commit(&sm.sfull[r]);
@@ -509,15 +543,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq4 = warp & 3;  // TMEM lane quarter
     const int row = wq4 * 32 + lane;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16) + r * 256;
-    // rot(b w_p), b = 0..15, filled once by warpgroup 0.
-    if (r == 0) {
-      for (int e = row; e < kPairs * 16; e += 128) {
-        const int p = e >> 4, bi = e & 15;
-        float cv, sv;
-        rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
-        sm.rot_lo[p][bi] = make_float2(cv, sv);
-      }
-      mbar_arrive(&sm.tables);
+    // rot(row w_p): this thread's row never changes, so its factor of every
+    // rotation stays in registers; the tile factor rot(128 j w_p) comes with
+    // each K tile.
+    RowRot<kPairs> rr;
+#pragma unroll
+    for (int p = 0; p < kPairs; ++p) {
+      float cv, sv;
+      rope_cos_sin(static_cast<double>(row), a.inv_freq[p], &cv, &sv);
+      rr.r[p] = make_float2(cv, sv);
     }
     const float sl2 = a.scale_log2;
     float wmq = 0.f, wmk = 0.f;
@@ -528,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Score bound in log2 units, with a 1/64 margin for the bf16 rounding of q', k'.
     const float bound = sl2 * kHeadDim * wmq * wmk * (1.0f + 1.0f / 64.0f);
     const bool exact = !(2.0f * bound <= 120.0f);
-    bool ok = mbar_wait(&sm.tables, 0, abort, a.err, kSiteTables);
+    bool ok = true;
 
     // K loads are accounted in order by both warpgroups (the same sequence the
     // producer issues); the warpgroup that owns the first head of a tile
@@ -542,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = j & 1;
           if (transform_last && acct == upto) {
             if (!mbar_wait(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
-            transform_k_row<kPairs>(sm.k[s], row, sm, s, a.eps);
+            transform_k_row<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
             fence_proxy_async_smem();
             mbar_arrive(&sm.kready[s]);
           } else if (acct == upto && j == kc.t) {
@@ -559,25 +593,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
-    // Row 0 of the warpgroup issues the warpgroup's own copies: Q(n) and g(n)
-    // into Q slot r, o(n) out of it.
+    // Row 0 of the warpgroup issues its copies through head n's slot n % 3:
+    // g(n) in, o(n) out, then releases the slot to the producer.
     const bool elected = row == 0;
-    int q_issued = 0, g_issued = 0;  // copies issued by this thread, for the drain
-    auto issue_q = [&](const Cursor& cn) {
-      const int hq = cn.kvh * a.G + cn.h;
-      mbar_arrive_expect_tx(&sm.qfull[r], kTileBytes);
-      tma_load_4d(sm.q[r], &tm_q, &sm.qfull[r], 0, hq, cn.t * kTile, cn.b);
-      tma_load_4d(sm.q[r] + kHalfBytes, &tm_q, &sm.qfull[r], 64, hq, cn.t * kTile, cn.b);
-      tma_prefetch_4d(&tm_g, 0, hq, cn.t * kTile, cn.b);  // warm L2 for the gate tile
-      tma_prefetch_4d(&tm_g, 64, hq, cn.t * kTile, cn.b);
-      ++q_issued;
-    };
+    // Gate copies this thread issued into each slot, and the barrier phase of
+    // the last one (slots are shared by both regions), for the drain.
+    int g_issued[3] = {0, 0, 0};
+    uint32_t last_g_phase[3] = {0u, 0u, 0u};
 
     Cursor c = cursor_at(a, u0);
     if (r == 1) next_head(c, a);
-    if (elected && r < n_heads) issue_q(c);
     for (int n = r; n < n_heads && ok; n += 2) {
       const uint32_t cnt = static_cast<uint32_t>(n >> 1);
+      const int qs = n % 3;                                   // this head's slot
+      const uint32_t qph = static_cast<uint32_t>(n / 3) & 1;  // its use of that slot
       const int hq = c.kvh * a.G + c.h;
       const long long pos = static_cast<long long>(c.t) * kTile + row;
 
@@ -585,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // then Q(n).  rot_hi of slot t&1 stays valid until K_{t+2} is loaded,
       // after every QK^T of tile t+1.
       if (!account(c.u, c.h == 0)) { ok = false; break; }
-      if (!mbar_wait(&sm.qfull[r], cnt & 1, abort, a.err, kSiteQFull)) { ok = false; break; }
-      const float rinv = transform_q_row<kPairs>(sm.q[r], row, sm, c.t & 1, a.eps);
+      if (!mbar_wait(&sm.qfull[qs], qph, abort, a.err, kSiteQFull)) { ok = false; break; }
+      const float rinv = transform_q_row<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready[r]);
 
@@ -594,10 +623,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&sm.sfull[r], cnt & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
       if (elected) {  // QK^T(n) has read Q(n): the slot takes the gate tile now
-        mbar_arrive_expect_tx(&sm.gfull[r], kTileBytes);
-        tma_load_4d(sm.q[r], &tm_g, &sm.gfull[r], 0, hq, c.t * kTile, c.b);
-        tma_load_4d(sm.q[r] + kHalfBytes, &tm_g, &sm.gfull[r], 64, hq, c.t * kTile, c.b);
-        ++g_issued;
+        mbar_arrive_expect_tx(&sm.gfull[qs], kTileBytes);
+        tma_load_4d(sm.q[qs], &tm_g, &sm.gfull[qs], 0, hq, c.t * kTile, c.b);
+        tma_load_4d(sm.q[qs] + kHalfBytes, &tm_g, &sm.gfull[qs], 64, hq, c.t * kTile, c.b);
+        ++g_issued[qs];
+        last_g_phase[qs] = qph;
       }
       // The MMA saw unnormalised q rows; 1/rms(q) enters with the softmax scale.
       const float rs = sl2 * rinv;
@@ -698,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue E(n): o = A/l * sigmoid(g) = (A * l^-1/2) * (1 + tanh(g/2)),
       // written over g(n) in Q slot r, 32 columns per step.
       if (!mbar_wait(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
-      if (!mbar_wait(&sm.gfull[r], cnt & 1, abort, a.err, kSiteGFull)) { ok = false; break; }
+      if (!mbar_wait(&sm.gfull[qs], qph, abort, a.err, kSiteGFull)) { ok = false; break; }
       tc_fence_after();
       const float2 hl2 = make_float2(0.5f / l, 0.5f / l);
       {
@@ -713,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&sm.tfree[r]);  // region r may take the next QK^T now
           }
-          uint8_t* half = sm.q[r] + (ch >> 1) * kHalfBytes;
+          uint8_t* half = sm.q[qs] + (ch >> 1) * kHalfBytes;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {  // four 16-byte pieces of this chunk
             uint4* gp = reinterpret_cast<uint4*>(half + sw_off(row, (ch & 1) * 4 + i));
@@ -741,22 +771,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       next_head(cn, a);
       next_head(cn, a);
       if (elected) {
-        // o(n) out of the slot (rows past T are clipped by the copy), then
-        // Q(n+2) in once the store has read it.
+        // o(n) out of the slot (rows past T are clipped by the copy); once the
+        // store has read it the slot goes back to the producer.
         if (!mbar_wait(&sm.ostore[r], cnt & 1, abort, a.err, kSiteOStore)) { ok = false; break; }
-        tma_store_4d(&tm_o, sm.q[r], 0, hq, c.t * kTile, c.b);
-        tma_store_4d(&tm_o, sm.q[r] + kHalfBytes, 64, hq, c.t * kTile, c.b);
+        tma_store_4d(&tm_o, sm.q[qs], 0, hq, c.t * kTile, c.b);
+        tma_store_4d(&tm_o, sm.q[qs] + kHalfBytes, 64, hq, c.t * kTile, c.b);
         bulk_commit();
         bulk_wait_read<0>();
-        if (n + 2 < n_heads) issue_q(cn);
+        mbar_arrive(&sm.slotfree[qs]);
       }
       c = cn;
     }
     if (elected) {
       if (!ok) {
         // Drain this thread's loads before the CTA releases its memory.
-        if (q_issued > 0) mbar_wait_drain(&sm.qfull[r], static_cast<uint32_t>(q_issued - 1) & 1);
-        if (g_issued > 0) mbar_wait_drain(&sm.gfull[r], static_cast<uint32_t>(g_issued - 1) & 1);
+        for (int s2 = 0; s2 < 3; ++s2)
+          if (g_issued[s2] > 0) mbar_wait_drain(&sm.gfull[s2], last_g_phase[s2]);
       }
       bulk_wait_all();  // every store complete before the CTA exits
     }
@@ -774,7 +804,7 @@ template <int kPairs>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
                 cudaStream_t stream) {
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = sizeof(Smem);
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
