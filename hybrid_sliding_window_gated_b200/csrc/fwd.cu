@@ -183,7 +183,7 @@ struct RowRot {
 __device__ __forceinline__ float row_sumsq(const uint8_t* h0, const uint8_t* h1, int row) {
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                    make_float2(0.f, 0.f)};  // independent chains for ILP
-#pragma unroll
+#pragma unroll 2
   for (int c = 0; c < 8; ++c) {
     const uint4 x = *reinterpret_cast<const uint4*>(h0 + sw_off(row, c));
     const uint4 y = *reinterpret_cast<const uint4*>(h1 + sw_off(row, c));
@@ -237,9 +237,8 @@ __device__ __forceinline__ void rope_chunks(uint8_t* h0, int row, float scale, c
 __device__ __forceinline__ void scale_chunks(uint8_t* h0, uint8_t* h1, int row, int c0,
                                              float scale, const float* w, const float* w2) {
   const float2 sc = make_float2(scale, scale);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    if (c < c0) continue;
+#pragma unroll 1
+  for (int c = c0; c < 16; ++c) {
     uint8_t* p = (c < 8 ? h0 : h1) + sw_off(row, c & 7);
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     const float4 wa1 = *reinterpret_cast<const float4*>(w + 8 * c);
@@ -390,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
         bool w = true;
-        if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+        if (lane == 0) w = mbar_wait_inl(bar, par, abort, a.err, site);
         return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
       };
       auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {
@@ -460,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------------------------------------------------------- MMA issuer
       Ring kr, vr;  // readiness of K (after the transform) and V slots
       bool ok = true;
-      if (a.flags & SWA_FLAG_FORCE_TIMEOUT) ok = mbar_wait(&sm.never, 0, abort, a.err, kSiteForced);
+      if (a.flags & SWA_FLAG_FORCE_TIMEOUT) ok = mbar_wait_inl(&sm.never, 0, abort, a.err, kSiteForced);
       Cursor cq = cursor_at(a, u0), cp = cq;
       for (int n = 0; n < n_heads && ok; n += 2) {
         // QK^T for heads n and n+1, then PV for both (regions n&1 alternate).
@@ -470,14 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sp = (cq.t + 1) & 1, sc = cq.t & 1;
           if (cq.h == 0) {
             if (need_prev(cq)) {
-              if (!mbar_wait(&sm.kready[sp], kr.parity(sp), abort, a.err, kSiteKReady)) { ok = false; break; }
+              if (!mbar_wait_inl(&sm.kready[sp], kr.parity(sp), abort, a.err, kSiteKReady)) { ok = false; break; }
               kr.advance(sp);
             }
-            if (!mbar_wait(&sm.kready[sc], kr.parity(sc), abort, a.err, kSiteKReady)) { ok = false; break; }
+            if (!mbar_wait_inl(&sm.kready[sc], kr.parity(sc), abort, a.err, kSiteKReady)) { ok = false; break; }
             kr.advance(sc);
           }
-          if (!mbar_wait(&sm.qready[r], cnt & 1, abort, a.err, kSiteQReady)) { ok = false; break; }
-          if (cnt > 0 && !mbar_wait(&sm.tfree[r], (cnt - 1) & 1, abort, a.err, kSiteTFree)) { ok = false; break; }
+          if (!mbar_wait_inl(&sm.qready[r], cnt & 1, abort, a.err, kSiteQReady)) { ok = false; break; }
+          if (cnt > 0 && !mbar_wait_inl(&sm.tfree[r], (cnt - 1) & 1, abort, a.err, kSiteTFree)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s_base = tmem + r * 256;
           const bool hp = has_prev(cq);
@@ -500,13 +499,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sp = (cp.t + 1) & 1, sc = cp.t & 1;
           if (cp.h == 0) {
             if (need_prev(cp)) {
-              if (!mbar_wait(&sm.vfull[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
+              if (!mbar_wait_inl(&sm.vfull[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
               vr.advance(sp);
             }
-            if (!mbar_wait(&sm.vfull[sc], vr.parity(sc), abort, a.err, kSiteVFull)) { ok = false; break; }
+            if (!mbar_wait_inl(&sm.vfull[sc], vr.parity(sc), abort, a.err, kSiteVFull)) { ok = false; break; }
             vr.advance(sc);
           }
-          if (!mbar_wait(&sm.pfull[r], cnt & 1, abort, a.err, kSitePFull)) { ok = false; break; }
+          if (!mbar_wait_inl(&sm.pfull[r], cnt & 1, abort, a.err, kSitePFull)) { ok = false; break; }
           tc_fence_after();
           const uint32_t p_base = tmem + r * 256;
           const bool hp = has_prev(cp);
@@ -575,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = need_prev(kc) ? kc.t - 1 : kc.t; j <= kc.t; ++j) {
           const int s = j & 1;
           if (transform_last && acct == upto) {
-            if (!mbar_wait(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
+            if (!mbar_wait_inl(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
             transform_k_row<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
             fence_proxy_async_smem();
             mbar_arrive(&sm.kready[s]);
@@ -584,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // producer publishes with kfull.  The slot cannot be refilled
             // before every QK^T of tile t+1, which waits for this warpgroup,
             // so the phase seen here is the current one.
-            if (!mbar_wait(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
+            if (!mbar_wait_inl(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
           }
           kr.advance(s);
         }
@@ -614,13 +613,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // then Q(n).  rot_hi of slot t&1 stays valid until K_{t+2} is loaded,
       // after every QK^T of tile t+1.
       if (!account(c.u, c.h == 0)) { ok = false; break; }
-      if (!mbar_wait(&sm.qfull[qs], qph, abort, a.err, kSiteQFull)) { ok = false; break; }
+      if (!mbar_wait_inl(&sm.qfull[qs], qph, abort, a.err, kSiteQFull)) { ok = false; break; }
       const float rinv = transform_q_row<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready[r]);
 
       // ---- softmax S(n)
-      if (!mbar_wait(&sm.sfull[r], cnt & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
+      if (!mbar_wait_inl(&sm.sfull[r], cnt & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
       if (elected) {  // QK^T(n) has read Q(n): the slot takes the gate tile now
         mbar_arrive_expect_tx(&sm.gfull[qs], kTileBytes);
@@ -637,7 +636,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Row maximum over the band: key tile t-1 gives columns c > row, key
         // tile t columns c <= row; pieces entirely outside the band are skipped.
         float m = -INFINITY;
+#pragma unroll 1
         for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+#pragma unroll 1
           for (int pc = 0; pc < 4; ++pc) {
             const bool none = blk == 0 ? (pc < wq4) : (pc > wq4);
             if (none) continue;
@@ -664,47 +665,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 l2 = make_float2(0.f, 0.f);
       const float2 rs2 = make_float2(rs, rs), nms2 = make_float2(-ms, -ms);
       {
-        uint32_t v[2][32];
-        tmem_ld32(t_row + (na > 0 ? wq4 * 32 : 128), v[0]);
+        // Chunk i of the band: 32 columns of S in, 16 columns of packed P out.
+        // Loops stay rolled (two chunk bodies per variant): the region code
+        // is refetched by every head, so its size decides instruction-cache
+        // hits.
+        auto chunk_col = [&](int i) { return i < na ? wq4 * 32 + i * 32 : 128 + (i - na) * 32; };
+        auto chunk = [&](const uint32_t(&x)[32], int i) {
+          const int blk = i < na ? 0 : 1;
+          const int pc = blk == 0 ? wq4 + i : i - na;
+          uint32_t pk[16];
+          if (pc != wq4) {
 #pragma unroll
-        for (int i = 0; i < 5; ++i) {
-          if (i < nch) {
-            const int blk = i < na ? 0 : 1;
-            const int pc = blk == 0 ? wq4 + i : i - na;
-            tmem_wait_ld();
-            if (i + 1 < nch) {  // next chunk's load overlaps this one's math
-              const int blk1 = i + 1 < na ? 0 : 1;
-              const int pc1 = blk1 == 0 ? wq4 + i + 1 : i + 1 - na;
-              tmem_ld32(t_row + blk1 * 128 + pc1 * 32, v[(i + 1) & 1]);
+            for (int e = 0; e < 16; ++e) {
+              const float2 z = __ffma2_rn(
+                  make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
+              const float2 p = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+              l2 = __fadd2_rn(l2, p);
+              pk[e] = pack_bf16x2(p.x, p.y);
             }
-            const uint32_t(&x)[32] = v[i & 1];
-            uint32_t pk[16];
-            if (pc != wq4) {
+          } else {  // the diagonal chunk: mask per column
+            const int c0 = pc * 32;
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float2 z = __ffma2_rn(
-                    make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
-                const float2 p = make_float2(ex2_approx(z.x), ex2_approx(z.y));
-                l2 = __fadd2_rn(l2, p);
-                pk[e] = pack_bf16x2(p.x, p.y);
-              }
-            } else {  // the diagonal chunk: mask per column
-              const int c0 = pc * 32;
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int cc = c0 + 2 * e;
-                const bool in0 = blk == 0 ? (cc > row) : (cc <= row);
-                const bool in1 = blk == 0 ? (cc + 1 > row) : (cc + 1 <= row);
-                const float2 z = __ffma2_rn(
-                    make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
-                const float2 p =
-                    make_float2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
-                l2 = __fadd2_rn(l2, p);
-                pk[e] = pack_bf16x2(p.x, p.y);
-              }
+            for (int e = 0; e < 16; ++e) {
+              const int cc = c0 + 2 * e;
+              const bool in0 = blk == 0 ? (cc > row) : (cc <= row);
+              const bool in1 = blk == 0 ? (cc + 1 > row) : (cc + 1 <= row);
+              const float2 z = __ffma2_rn(
+                  make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), rs2, nms2);
+              const float2 p =
+                  make_float2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
+              l2 = __fadd2_rn(l2, p);
+              pk[e] = pack_bf16x2(p.x, p.y);
             }
-            tmem_st16(t_row + blk * 64 + pc * 16, pk);
           }
+          tmem_st16(t_row + blk * 64 + pc * 16, pk);
+        };
+        // One register buffer: while a warp waits for its chunk, the SM runs
+        // the other warps; the smaller loop keeps the region code in cache.
+#pragma unroll 1
+        for (int i = 0; i < nch; ++i) {
+          uint32_t va[32];
+          tmem_ld32(t_row + chunk_col(i), va);
+          tmem_wait_ld();
+          chunk(va, i);
         }
       }
       {
@@ -727,22 +730,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- epilogue E(n): o = A/l * sigmoid(g) = (A * l^-1/2) * (1 + tanh(g/2)),
       // written over g(n) in Q slot r, 32 columns per step.
-      if (!mbar_wait(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
-      if (!mbar_wait(&sm.gfull[qs], qph, abort, a.err, kSiteGFull)) { ok = false; break; }
+      if (!mbar_wait_inl(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
+      if (!mbar_wait_inl(&sm.gfull[qs], qph, abort, a.err, kSiteGFull)) { ok = false; break; }
       tc_fence_after();
       const float2 hl2 = make_float2(0.5f / l, 0.5f / l);
       {
-        uint32_t ov[2][32];
-        tmem_ld32(t_row + 128, ov[0]);
-#pragma unroll
-        for (int ch = 0; ch < kHeadDim / 32; ++ch) {
-          tmem_wait_ld();
-          if (ch + 1 < kHeadDim / 32) {
-            tmem_ld32(t_row + 128 + (ch + 1) * 32, ov[(ch + 1) & 1]);
-          } else {
-            tc_fence_before();
-            mbar_arrive(&sm.tfree[r]);  // region r may take the next QK^T now
-          }
+        // Chunk ch: 32 columns of O, written over the same columns of g.
+        auto gate = [&](const uint32_t(&ov)[32], int ch) {
           uint8_t* half = sm.q[qs] + (ch >> 1) * kHalfBytes;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {  // four 16-byte pieces of this chunk
@@ -754,14 +748,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 4; ++e) {
               const float2 t =
                   tanh2_f16(__fmul2_rn(bf16x2_to_f2(gw[e]), make_float2(0.5f, 0.5f)));
-              const float2 acc = __fmul2_rn(make_float2(__uint_as_float(ov[ch & 1][8 * i + 2 * e]),
-                                                        __uint_as_float(ov[ch & 1][8 * i + 2 * e + 1])),
+              const float2 acc = __fmul2_rn(make_float2(__uint_as_float(ov[8 * i + 2 * e]),
+                                                        __uint_as_float(ov[8 * i + 2 * e + 1])),
                                             hl2);
               const float2 o2 = __ffma2_rn(acc, t, acc);
               ow[e] = pack_bf16x2(o2.x, o2.y);
             }
             *gp = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
+        };
+#pragma unroll 1
+        for (int ch = 0; ch < kHeadDim / 32; ++ch) {
+          uint32_t oa[32];
+          tmem_ld32(t_row + 128 + ch * 32, oa);
+          tmem_wait_ld();
+          if (ch + 1 == kHeadDim / 32) {
+            tc_fence_before();
+            mbar_arrive(&sm.tfree[r]);  // region r may take the next QK^T now
+          }
+          gate(oa, ch);
         }
       }
       fence_proxy_async_smem();
@@ -773,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elected) {
         // o(n) out of the slot (rows past T are clipped by the copy); once the
         // store has read it the slot goes back to the producer.
-        if (!mbar_wait(&sm.ostore[r], cnt & 1, abort, a.err, kSiteOStore)) { ok = false; break; }
+        if (!mbar_wait_inl(&sm.ostore[r], cnt & 1, abort, a.err, kSiteOStore)) { ok = false; break; }
         tma_store_4d(&tm_o, sm.q[qs], 0, hq, c.t * kTile, c.b);
         tma_store_4d(&tm_o, sm.q[qs] + kHalfBytes, 64, hq, c.t * kTile, c.b);
         bulk_commit();

@@ -68,8 +68,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // kWaitLimitNs (or at once if another role already raised `abort`), records
 // kDevErrTimeoutBase + site in the sticky device error word `err` (first error
 // wins) and raises `abort`.
+// The waiting loop lives out of line: every role has many wait sites, and
+// only the first try_wait of each is on the fast path.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                   int* err, int site) {
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(err, 0, kDevErrTimeoutBase + site);
+      *abort = 1;
+      return false;
+    }
+  }
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, err, site);
+}
+// The same wait with the loop inlined, for kernels whose warpgroups change
+// their register budgets (setmaxnreg), where ptxas cannot place calls.
+__device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              int* err, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
@@ -354,17 +378,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Rotation angle p * inv_freq reduced to [-pi, pi] in fp64 (positions reach
-// 2.6e5 radians, far beyond what an fp32 product and reduction keep), then
-// evaluated with the fp32 sincosf.
+// Rotation angle p * inv_freq, as a multiple of pi reduced to [-1, 1] in fp64
+// (positions reach 2.6e5 radians, far beyond what an fp32 product and
+// reduction keep), then evaluated with the fp32 sincospif, which needs no
+// large-argument path.
 __device__ __forceinline__ void rope_cos_sin(double pos, double inv_freq, float* c, float* s) {
-  const double kTwoPi = 6.283185307179586;
-  const double kInvTwoPi = 0.15915494309189535;
-  double a = pos * inv_freq;
-  double k = rint(a * kInvTwoPi);
-  double r = fma(-k, kTwoPi, a);
-  r = fma(-k, 2.4492935982947064e-16, r);  // low part of 2*pi
-  sincosf(static_cast<float>(r), s, c);
+  const double x = pos * (inv_freq * 0.3183098861837907);  // angle / pi
+  const double r = x - 2.0 * rint(0.5 * x);
+  sincospif(static_cast<float>(r), s, c);
 }
 
 }  // namespace swa
