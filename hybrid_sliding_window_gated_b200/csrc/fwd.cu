@@ -17,9 +17,11 @@
 // group and by two query tiles.
 //
 // Roles (384 threads, three warpgroups; registers rebalanced with setmaxnreg):
-//   warp 0      K/V producer (lane 0 issues TMA; all lanes compute each K
-//               tile's rotation table)
+//   warp 0      K and Q producer (lane 0 issues TMA; all lanes compute each
+//               K tile's rotation table)
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one lane)
+//   warp 3      V producer (one lane), so a V tile that waits for its slot
+//               holds up no K or Q load
 //   warps 4-7   region 0 (even head slots), warps 8-11 region 1 (odd).  For
 //               each of its heads a region warpgroup normalises and rotates
 //               the Q rows (and the K rows of a tile whose first head it owns)
@@ -60,10 +62,16 @@
 // constant, so the result equals the max-subtracted form.  Weights outside
 // that range fall back to an exact two-pass (row max first) softmax.
 //
-// Rotation angles.  Position p = 128 j + 16 a + b: the rotation by p w is the
-// product of a per-tile table rot((128 j + 16 a) w), a in 0..7, computed by the
-// producer's lanes for each K tile (fp64 range reduction, then sincosf), and a
-// per-CTA table rot(b w), b in 0..15.
+// Rotation angles.  Position p = 128 j + i: the rotation by p w is the
+// product of a per-tile table rot(128 j w), computed by the producer's lanes
+// for each K tile (fp64 reduction of the angle as a multiple of pi, then
+// sincospif), and rot(i w) for the thread's own row i, which each region
+// thread keeps in registers.
+//
+// Code size.  The region loop runs once per head on every SM, so its
+// instructions are refetched all the time; when they miss the instruction
+// cache, every SM fetches from L2 while L2 is busiest.  The chunk loops of the
+// softmax and the epilogue therefore stay rolled, with one register buffer.
 #include "launch.cuh"
 #include "ptx.cuh"
 #include "swa_internal.h"
@@ -384,39 +392,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     regs_dec<kRegsControl>();
     if (warp == 0) {
-      // ---------------------------------------------------------- producer
-      Ring kr, vr;
+      // -------------------------------------------------- K and Q producer
+      Ring kr;
       bool ok = true;
       auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
         bool w = true;
         if (lane == 0) w = mbar_wait_inl(bar, par, abort, a.err, site);
         return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
       };
-      auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {
+      auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {  // K tiles only
+        (void)is_k;
         const int s = j & 1;
-        Ring& ring = is_k ? kr : vr;
-        uint64_t* full = is_k ? &sm.kfull[s] : &sm.vfull[s];
-        uint64_t* empty = is_k ? &sm.kempty[s] : &sm.vempty[s];
-        if (ring.was_used(s) && !wait0(empty, ring.parity(s) ^ 1u, is_k ? kSiteKEmpty : kSiteVEmpty))
-          return false;
+        if (kr.was_used(s) && !wait0(&sm.kempty[s], kr.parity(s) ^ 1u, kSiteKEmpty)) return false;
         if (lane == 0) {
-          uint8_t* dst = is_k ? sm.k[s] : sm.v[s];
-          const CUtensorMap* map = is_k ? &tm_k : &tm_v;
-          mbar_arrive_expect_tx(full, kTileBytes);
-          tma_load_4d(dst, map, full, 0, c.kvh, j * kTile, c.b);
-          tma_load_4d(dst + kHalfBytes, map, full, 64, c.kvh, j * kTile, c.b);
+          mbar_arrive_expect_tx(&sm.kfull[s], kTileBytes);
+          tma_load_4d(sm.k[s], &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
+          tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 64, c.kvh, j * kTile, c.b);
         }
-        if (is_k) {
-          // rot(128 j w_p) for this tile, then the second arrive on kfull.
-          if (lane < kPairs) {
-            float cv, sv;
-            rope_cos_sin(static_cast<double>(j) * kTile, a.inv_freq[lane], &cv, &sv);
-            sm.rot_tile[s][lane] = make_float2(cv, sv);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(full);
+        // rot(128 j w_p) for this tile, then the second arrive on kfull.
+        if (lane < kPairs) {
+          float cv, sv;
+          rope_cos_sin(static_cast<double>(j) * kTile, a.inv_freq[lane], &cv, &sv);
+          sm.rot_tile[s][lane] = make_float2(cv, sv);
         }
-        ring.advance(s);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.kfull[s]);
+        kr.advance(s);
         return true;
       };
       // Q(n) goes into slot n % 3 as soon as the o store of head n-3 has read
@@ -424,9 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nq = 0;  // Q loads issued
       Cursor c = cursor_at(a, u0);
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
-        if (need_prev(c))  // first tile of a run: key tile t-1 as well
-          ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
-        ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
+        if (need_prev(c)) ok = load_kv(true, c.t - 1, c);  // first tile of a run: key tile t-1 too
+        ok = ok && load_kv(true, c.t, c);
         for (int h = 0; h < a.G && ok; ++h) {
           const int qs = nq % 3;
           if (nq >= 3 && !wait0(&sm.slotfree[qs], ((nq / 3) - 1) & 1, kSiteSlotFree)) {
@@ -446,14 +446,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok && lane == 0) {
         // Drain the loads this warp issued before the CTA releases its memory.
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 2; ++s)
           if (kr.was_used(s)) mbar_wait_drain(&sm.kfull[s], kr.parity(s) ^ 1u);
-          if (vr.was_used(s)) mbar_wait_drain(&sm.vfull[s], vr.parity(s) ^ 1u);
-        }
         for (int s = 0; s < 3; ++s) {
           const int cntq = (nq - s + 2) / 3;  // Q loads into slot s
           if (cntq > 0) mbar_wait_drain(&sm.qfull[s], static_cast<uint32_t>(cntq - 1) & 1);
         }
+      }
+    } else if (warp == 3 && lane == 0) {
+      // -------------------------------------------------------- V producer
+      // Its own thread: a V tile waits for the last PV of the tile before,
+      // and no K or Q load should queue behind that.
+      Ring vr;
+      bool ok = true;
+      Cursor c = cursor_at(a, u0);
+      for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+        for (int j = need_prev(c) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+          const int s = j & 1;
+          if (vr.was_used(s) &&
+              !(ok = mbar_wait_inl(&sm.vempty[s], vr.parity(s) ^ 1u, abort, a.err, kSiteVEmpty)))
+            break;
+          mbar_arrive_expect_tx(&sm.vfull[s], kTileBytes);
+          tma_load_4d(sm.v[s], &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
+          tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 64, c.kvh, j * kTile, c.b);
+          vr.advance(s);
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < 2; ++s)
+          if (vr.was_used(s)) mbar_wait_drain(&sm.vfull[s], vr.parity(s) ^ 1u);
       }
     } else if (warp == 1 && lane == 0) {
       // -------------------------------------------------------- MMA issuer
@@ -617,6 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float rinv = transform_q_row<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready[r]);
+
 
       // ---- softmax S(n)
       if (!mbar_wait_inl(&sm.sfull[r], cnt & 1, abort, a.err, kSiteSFull)) { ok = false; break; }
