@@ -741,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 gg = bf2(gwv[e]), dd = bf2(dwv[e]);
               const float a0 = __uint_as_float(x[8 * i + 2 * e]) * inv_l;
               const float a1 = __uint_as_float(x[8 * i + 2 * e + 1]) * inv_l;
-              const float s0 = 1.0f / (1.0f + __expf(-gg.x)), s1 = 1.0f / (1.0f + __expf(-gg.y));
+              const float s0 = sigmoid_fast(gg.x), s1 = sigmoid_fast(gg.y);  // one MUFU op each
               dgo[e] = pack_bf16x2(dd.x * a0 * s0 * (1.0f - s0), dd.y * a1 * s1 * (1.0f - s1));
               in_range &= fabsf(dd.x) <= kF16Max && fabsf(dd.y) <= kF16Max;
               dao[e] = pack_f16x2(dd.x * s0, dd.y * s1);
