@@ -658,41 +658,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float rinv_q = norm_rope_row<kPairs>(slot, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready);
-      const float lse2 = valid_row ? a.lse[lrow] * kLog2e : 0.f;
-      float lsum = 0.f;
+      // Rows past T take lse = +inf: their P is exactly 0 with no mask.
+      const float lse2 = valid_row ? a.lse[lrow] * kLog2e : INFINITY;
+      float2 lsum2 = make_float2(0.f, 0.f);
 
       // ---- P = exp(s - lse) on the band, packed over columns 0..127
       if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
       tc_fence_after();
-      for (int blk = 0; blk < 2; ++blk) {
-        for (int pc = 0; pc < 4; ++pc) {
-          // key tile t-1 keeps columns > row, key tile t columns <= row
-          // Warp-uniform (tcgen05.ld is warp-collective); row validity is in the mask.
-          const bool any = blk == 0 ? (hp && pc >= wq4) : (pc <= wq4);
-          uint32_t pk[16];
-          if (any) {
-            uint32_t x[32];
-            tmem_ld32(t_row + blk * 128 + pc * 32, x);
-            tmem_wait_ld();
+      {
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {
+#pragma unroll 1
+          for (int pc = 0; pc < 4; ++pc) {
+            // key tile t-1 keeps columns > row, key tile t columns <= row; only
+            // chunk pc == wq4 straddles the band edge.  Warp-uniform
+            // (tcgen05.ld is warp-collective).
+            const bool any = blk == 0 ? (hp && pc >= wq4) : (pc <= wq4);
+            uint32_t pk[16];
+            if (any) {
+              uint32_t x[32];
+              tmem_ld32(t_row + blk * 128 + pc * 32, x);
+              tmem_wait_ld();
+              if (pc != wq4) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c0 = pc * 32 + 2 * e;
-              const bool in0 = valid_row && (blk == 0 ? c0 > row : c0 <= row);
-              const bool in1 = valid_row && (blk == 0 ? c0 + 1 > row : c0 + 1 <= row);
-              const float p0 = in0 ? ex2_approx(__uint_as_float(x[2 * e]) * a.scale_log2 - lse2) : 0.f;
-              const float p1 =
-                  in1 ? ex2_approx(__uint_as_float(x[2 * e + 1]) * a.scale_log2 - lse2) : 0.f;
-              pk[e] = pack_f16x2(p0, p1);
-              const float2 pr = f16x2(pk[e]);  // the values the MMAs see
-              lsum += pr.x + pr.y;
+                for (int e = 0; e < 16; ++e) {
+                  const float2 z = __ffma2_rn(
+                      make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
+                  pk[e] = pack_f16x2(ex2_approx(z.x), ex2_approx(z.y));
+                  lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));  // the values the MMAs see
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const int c0 = pc * 32 + 2 * e;
+                  const bool in0 = blk == 0 ? c0 > row : c0 <= row;
+                  const bool in1 = blk == 0 ? c0 + 1 > row : c0 + 1 <= row;
+                  const float2 z = __ffma2_rn(
+                      make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
+                  pk[e] = pack_f16x2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
+                  lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));
+                }
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = 0u;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            tmem_st16(t_row + blk * 64 + pc * 16, pk);
           }
-          tmem_st16(t_row + blk * 64 + pc * 16, pk);
         }
       }
+      const float lsum = lsum2.x + lsum2.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.pfull);
@@ -715,7 +731,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
       tc_fence_after();
-      float dsum = 0.f;
+      float2 dsum2 = make_float2(0.f, 0.f);
+      const float2 il2 = make_float2(inv_l, inv_l);
+      float dmax = 0.f;  // largest |dO| of the row: fp16 staging range
       {
         uint4* dgrow = reinterpret_cast<uint4*>(a.dg + tok * kHeadDim);
         uint4* darow = reinterpret_cast<uint4*>(a.ws_da + tok * kHeadDim);
@@ -739,14 +757,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 gg = bf2(gwv[e]), dd = bf2(dwv[e]);
-              const float a0 = __uint_as_float(x[8 * i + 2 * e]) * inv_l;
-              const float a1 = __uint_as_float(x[8 * i + 2 * e + 1]) * inv_l;
-              const float s0 = sigmoid_fast(gg.x), s1 = sigmoid_fast(gg.y);  // one MUFU op each
-              dgo[e] = pack_bf16x2(dd.x * a0 * s0 * (1.0f - s0), dd.y * a1 * s1 * (1.0f - s1));
-              in_range &= fabsf(dd.x) <= kF16Max && fabsf(dd.y) <= kF16Max;
-              dao[e] = pack_f16x2(dd.x * s0, dd.y * s1);
-              const float2 dr = f16x2(dao[e]);  // D uses the rounded dA the MMAs see
-              dsum += dr.x * a0 + dr.y * a1;
+              const float2 av = __fmul2_rn(
+                  make_float2(__uint_as_float(x[8 * i + 2 * e]), __uint_as_float(x[8 * i + 2 * e + 1])),
+                  il2);                                                    // A / l
+              const float2 sg = make_float2(sigmoid_fast(gg.x), sigmoid_fast(gg.y));  // one MUFU op each
+              const float2 ds = __ffma2_rn(make_float2(-sg.x, -sg.y), sg, sg);      // s (1 - s)
+              const float2 dgv = __fmul2_rn(__fmul2_rn(dd, av), ds);
+              dgo[e] = pack_bf16x2(dgv.x, dgv.y);
+              dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+              const float2 dav = __fmul2_rn(dd, sg);
+              dao[e] = pack_f16x2(dav.x, dav.y);
+              dsum2 = __ffma2_rn(f16x2(dao[e]), av, dsum2);  // D uses the rounded dA the MMAs see
             }
             const int c16 = 4 * ch + i;  // 16-byte piece of the row
             const uint4 da16 = make_uint4(dao[0], dao[1], dao[2], dao[3]);
@@ -766,8 +787,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.dafull);
-        if (valid_row) a.ws_d[lrow] = dsum;
       }
+      const float dsum = dsum2.x + dsum2.y;
+      in_range &= !(dmax > kF16Max);
+      if (valid_row) a.ws_d[lrow] = dsum;
 
       // ---- dS = scale P (dP - D) per key tile into the Q slot, then dQ
       if (!(ok = warp_wait(&sm.dpfull, ph, abort, a.err, kSiteDPFull))) break;

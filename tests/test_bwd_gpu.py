@@ -104,6 +104,18 @@ def test_values_beyond_fp16_range_are_reported():
     assert swa.get_last_device_error()[0] == swa.OK  # cleared
 
 
+def test_upstream_gradient_beyond_fp16_range_is_reported():
+    """dA = dO * sigmoid(g) is staged in fp16 too: a dO past its range is refused."""
+    cfg, d = _small_inputs()
+    o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], want_lse=True)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    d["dO"][0, 150, 2, 100] = -2.0e5
+    swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"])
+    assert swa.get_last_device_error()[0] == swa.ERR_INVALID_ARG
+    assert swa.get_last_device_error()[0] == swa.OK
+
+
 def test_weights_beyond_fp16_operands_are_reported():
     cfg, d = _small_inputs()
     o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], want_lse=True)
