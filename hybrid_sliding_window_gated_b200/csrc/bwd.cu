@@ -869,6 +869,8 @@ struct alignas(1024) SmemKV {
   uint32_t tmem_base;
   int abort;
 };
+static_assert(offsetof(SmemKV, lse2) % 16 == 0 && offsetof(SmemKV, dd) % 16 == 0,
+              "per-column lse / D are read as float4");
 static_assert(sizeof(SmemKV) + 1024 <= 232448, "pass 2 shared memory");
 
 template <int kPairs>
@@ -1091,9 +1093,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float* l2 = sm.lse2[nq & 1];
         const float* dd = sm.dd[nq & 1];
+        // Query columns past T (the last, partial tile) and key rows past T
+        // are outside; only chunk wq4 straddles the band edge.
+        const int col_end = static_cast<int>(min(static_cast<long long>(kTile),
+                                                 a.T - static_cast<long long>(c.t + dt) * kTile));
+        const float2 kval2 = kpos < a.T ? make_float2(1.f, 1.f) : make_float2(0.f, 0.f);
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+        const float2 scale2 = make_float2(a.scale, a.scale);
+#pragma unroll 1
         for (int pc = 0; pc < 4; ++pc) {
           // query tile j keeps columns >= row, tile j+1 columns < row
-          // Warp-uniform (tcgen05.ld is warp-collective); key validity is in the mask.
+          // (warp-uniform: tcgen05.ld is warp-collective).
           const bool any = dt == 0 ? (pc >= wq4) : (pc <= wq4);
           uint32_t pk[16], dk[16];
           if (any) {
@@ -1101,21 +1111,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(t_row + 256 + pc * 32, s);
             tmem_ld32(t_row + 384 + pc * 32, dp);
             tmem_wait_ld();
+            const bool edge = pc == wq4 || pc * 32 + 32 > col_end;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float pv[2], dv[2];
+            for (int e4 = 0; e4 < 8; ++e4) {  // four columns per step
+              const float4 l4 = *reinterpret_cast<const float4*>(l2 + pc * 32 + 4 * e4);
+              const float4 d4 = *reinterpret_cast<const float4*>(dd + pc * 32 + 4 * e4);
 #pragma unroll
-              for (int f = 0; f < 2; ++f) {
-                const int col = pc * 32 + 2 * e + f;
-                const long long q_abs = static_cast<long long>(c.t + dt) * kTile + col;
-                const bool in = kpos < a.T && q_abs < a.T && (dt == 0 ? col >= row : col < row);
-                const float p =
-                    in ? ex2_approx(__uint_as_float(s[2 * e + f]) * a.scale_log2 - l2[col]) : 0.f;
-                pv[f] = p;
-                dv[f] = a.scale * p * (__uint_as_float(dp[2 * e + f]) - dd[col]);
+              for (int h = 0; h < 2; ++h) {
+                const int e = 2 * e4 + h;
+                const float2 nl = h == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
+                const float2 dv2 = h == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
+                const float2 z = __ffma2_rn(
+                    make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sc2, nl);
+                float2 p = __fmul2_rn(make_float2(ex2_approx(z.x), ex2_approx(z.y)), kval2);
+                if (edge) {
+                  const int col = pc * 32 + 2 * e;
+                  const bool in0 = col < col_end && (dt == 0 ? col >= row : col < row);
+                  const bool in1 = col + 1 < col_end && (dt == 0 ? col + 1 >= row : col + 1 < row);
+                  p = make_float2(in0 ? p.x : 0.f, in1 ? p.y : 0.f);
+                }
+                const float2 dsv = __fmul2_rn(
+                    __fmul2_rn(scale2, p),
+                    __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                               make_float2(-dv2.x, -dv2.y)));
+                pk[e] = pack_f16x2(p.x, p.y);
+                dk[e] = pack_f16x2(dsv.x, dsv.y);
               }
-              pk[e] = pack_f16x2(pv[0], pv[1]);
-              dk[e] = pack_f16x2(dv[0], dv[1]);
             }
           } else {
 #pragma unroll
