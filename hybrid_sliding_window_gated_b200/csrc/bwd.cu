@@ -206,26 +206,27 @@ __device__ __forceinline__ void load_half(const uint16_t* xrow, int half, uint32
 }
 
 // dy for dims [64 half, 64 half + 64): the gradient w.r.t. the rotated,
-// normalised row (TMEM columns from t_lane_col), rotated back by RoPE^-1.
+// normalised row (TMEM columns from t_lane_col), rotated back by RoPE^-1 with
+// this row's rotation factors `rc`.
 template <int kPairs>
-__device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half, const float2 (*hi)[8],
-                                             const RotTables& t, int row, float (&y)[64]) {
-  uint32_t r[32];
+__device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half,
+                                             const float2 (&rc)[kPairs > 0 ? kPairs : 1],
+                                             float (&y)[64]) {
+  uint32_t r[32], r2[32];
   tmem_ld32(t_lane_col + half * 64, r);
+  tmem_ld32(t_lane_col + half * 64 + 32, r2);
   tmem_wait_ld();
 #pragma unroll
-  for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-  tmem_ld32(t_lane_col + half * 64 + 32, r);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) y[32 + i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 32; ++i) {
+    y[i] = __uint_as_float(r[i]);
+    y[32 + i] = __uint_as_float(r2[i]);
+  }
   if (half == 0) {
 #pragma unroll
     for (int p = 0; p < kPairs; ++p) {
-      const float2 c = rot_at(hi, t, p, row);
       const float a = y[p], b = y[p + kPairs];
-      y[p] = a * c.x + b * c.y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
-      y[p + kPairs] = b * c.x - a * c.y;
+      y[p] = a * rc[p].x + b * rc[p].y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
+      y[p + kPairs] = b * rc[p].x - a * rc[p].y;
     }
   }
 }
@@ -234,48 +235,57 @@ __device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half, cons
 // rotated, normalised row, in TMEM columns [t_lane_col, +128) of this thread's
 // lane; xrow: the raw row in global memory (nullptr: a row past the end).
 // Writes dx to `out` (unless nullptr) and adds dy (*) xhat into dw (shared,
-// summed over the warp first).  Works half a row at a time.
+// summed over the warp first).  Works half a row at a time; the rotation
+// factors are computed once for both passes.
 template <int kPairs>
 __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16_t* xrow,
                                                float rinv, const float* w, const float2 (*hi)[8],
                                                const RotTables& t, int row, int lane, float* dw,
                                                uint16_t* out) {
+  float2 rc[kPairs > 0 ? kPairs : 1];
+#pragma unroll
+  for (int p = 0; p < kPairs; ++p) rc[p] = rot_at(hi, t, p, row);
+  const float2 rinv2 = make_float2(rinv, rinv);
   // Pass 1: dot = mean(xhat (*) w (*) dy) and dw.
-  float dot = 0.f;
+  float2 dot2 = make_float2(0.f, 0.f);
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
     uint32_t x[32];
     load_half(xrow, half, x);
-    load_dy_half<kPairs>(t_lane_col, half, hi, t, row, y);
+    load_dy_half<kPairs>(t_lane_col, half, rc, y);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = bf2(x[i]);
+      const float2 xh = __fmul2_rn(bf2(x[i]), rinv2);  // xhat
+      const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
       const int d = half * 64 + 2 * i;
-      dot += y[2 * i] * w[d] * xh.x + y[2 * i + 1] * w[d + 1] * xh.y;
-      y[2 * i] *= xh.x * rinv;  // dw contribution dy * xhat
-      y[2 * i + 1] *= xh.y * rinv;
+      dot2 = __ffma2_rn(__fmul2_rn(yv, make_float2(w[d], w[d + 1])), xh, dot2);
+      const float2 c = __fmul2_rn(yv, xh);  // dw contribution dy * xhat
+      y[2 * i] = c.x;
+      y[2 * i + 1] = c.y;
     }
     const float2 s = warp_reduce_scatter64(y, lane);
     atomicAdd(dw + half * 64 + 2 * lane, s.x);
     atomicAdd(dw + half * 64 + 2 * lane + 1, s.y);
   }
-  dot *= rinv * (1.0f / kHeadDim);  // x = raw, so xhat = x * rinv
+  const float dot = (dot2.x + dot2.y) * (1.0f / kHeadDim);
+  const float2 ndot2 = make_float2(-dot, -dot);
   // Pass 2: dx = rinv (w dy - xhat dot).
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
     uint32_t x[32];
     load_half(xrow, half, x);
-    load_dy_half<kPairs>(t_lane_col, half, hi, t, row, y);
+    load_dy_half<kPairs>(t_lane_col, half, rc, y);
     uint32_t o[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = bf2(x[i]);
+      const float2 xh = __fmul2_rn(bf2(x[i]), rinv2);
       const int d = half * 64 + 2 * i;
-      const float g0 = rinv * (y[2 * i] * w[d] - xh.x * rinv * dot);
-      const float g1 = rinv * (y[2 * i + 1] * w[d + 1] - xh.y * rinv * dot);
-      o[i] = pack_bf16x2(g0, g1);
+      const float2 g = __fmul2_rn(
+          rinv2, __ffma2_rn(xh, ndot2,
+                            __fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(w[d], w[d + 1]))));
+      o[i] = pack_bf16x2(g.x, g.y);
     }
     if (out) {
 #pragma unroll
