@@ -60,6 +60,20 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 __device__ __forceinline__ float2 f16x2(uint32_t u) {
   return __half22float2(*reinterpret_cast<const __half2*>(&u));
 }
+// 32 bytes of one row per thread in one access (rows are 32-byte aligned):
+// a warp's row-per-thread access then touches each 32-byte sector once.
+__device__ __forceinline__ void ld32B(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st32B(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // Largest magnitude the fp16 staging of V and dA carries (the fp16 maximum).
 constexpr float kF16Max = 65504.0f;
 
@@ -731,13 +745,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- A: dg, dA (smem and workspace), D -- 32 dims at a time (a rolled
       // loop keeps the code small), the next chunk's g and dO loads in flight
       // while this one is computed (chunk 0's while the PV MMA runs).
-      const uint4* grow = reinterpret_cast<const uint4*>(a.g + tok * kHeadDim);
-      const uint4* dorow = reinterpret_cast<const uint4*>(a.dO + tok * kHeadDim);
-      uint4 gc[4], dc[4];
+      const uint8_t* grow = reinterpret_cast<const uint8_t*>(a.g + tok * kHeadDim);
+      const uint8_t* dorow = reinterpret_cast<const uint8_t*>(a.dO + tok * kHeadDim);
+      uint32_t gc[16], dc[16];  // this chunk's 32 columns of g and dO
+      {
+        uint32_t (&g0)[8] = *reinterpret_cast<uint32_t(*)[8]>(gc);
+        uint32_t (&g1)[8] = *reinterpret_cast<uint32_t(*)[8]>(gc + 8);
+        uint32_t (&d0)[8] = *reinterpret_cast<uint32_t(*)[8]>(dc);
+        uint32_t (&d1)[8] = *reinterpret_cast<uint32_t(*)[8]>(dc + 8);
+        if (valid_row) {
+          ld32B(grow, g0);
+          ld32B(grow + 32, g1);
+          ld32B(dorow, d0);
+          ld32B(dorow + 32, d1);
+        } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        gc[i] = valid_row ? __ldg(grow + i) : make_uint4(0u, 0u, 0u, 0u);
-        dc[i] = valid_row ? __ldg(dorow + i) : make_uint4(0u, 0u, 0u, 0u);
+          for (int i = 0; i < 16; ++i) gc[i] = dc[i] = 0u;
+        }
       }
       if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
       tc_fence_after();
@@ -745,51 +769,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 il2 = make_float2(inv_l, inv_l);
       float dmax = 0.f;  // largest |dO| of the row: fp16 staging range
       {
-        uint4* dgrow = reinterpret_cast<uint4*>(a.dg + tok * kHeadDim);
-        uint4* darow = reinterpret_cast<uint4*>(a.ws_da + tok * kHeadDim);
+        uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim);
+        uint8_t* darow = reinterpret_cast<uint8_t*>(a.ws_da + tok * kHeadDim);
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
-          uint4 gn[4], dn[4];
+          uint32_t gn[16], dn[16];
           const bool more = valid_row && ch + 1 < 4;
+          if (more) {
+            ld32B(grow + 64 * (ch + 1), *reinterpret_cast<uint32_t(*)[8]>(gn));
+            ld32B(grow + 64 * (ch + 1) + 32, *reinterpret_cast<uint32_t(*)[8]>(gn + 8));
+            ld32B(dorow + 64 * (ch + 1), *reinterpret_cast<uint32_t(*)[8]>(dn));
+            ld32B(dorow + 64 * (ch + 1) + 32, *reinterpret_cast<uint32_t(*)[8]>(dn + 8));
+          } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            gn[i] = more ? __ldg(grow + 4 * (ch + 1) + i) : make_uint4(0u, 0u, 0u, 0u);
-            dn[i] = more ? __ldg(dorow + 4 * (ch + 1) + i) : make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < 16; ++i) gn[i] = dn[i] = 0u;
           }
           uint32_t x[32];
           tmem_ld32(t_row + 256 + ch * 32, x);
           tmem_wait_ld();
+          uint32_t dgo[16], dao[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t gwv[4] = {gc[i].x, gc[i].y, gc[i].z, gc[i].w};
-            const uint32_t dwv[4] = {dc[i].x, dc[i].y, dc[i].z, dc[i].w};
-            uint32_t dgo[4], dao[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 gg = bf2(gwv[e]), dd = bf2(dwv[e]);
-              const float2 av = __fmul2_rn(
-                  make_float2(__uint_as_float(x[8 * i + 2 * e]), __uint_as_float(x[8 * i + 2 * e + 1])),
-                  il2);                                                    // A / l
-              const float2 sg = make_float2(sigmoid_fast(gg.x), sigmoid_fast(gg.y));  // one MUFU op each
-              const float2 ds = __ffma2_rn(make_float2(-sg.x, -sg.y), sg, sg);      // s (1 - s)
-              const float2 dgv = __fmul2_rn(__fmul2_rn(dd, av), ds);
-              dgo[e] = pack_bf16x2(dgv.x, dgv.y);
-              dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
-              const float2 dav = __fmul2_rn(dd, sg);
-              dao[e] = pack_f16x2(dav.x, dav.y);
-              dsum2 = __ffma2_rn(f16x2(dao[e]), av, dsum2);  // D uses the rounded dA the MMAs see
-            }
-            const int c16 = 4 * ch + i;  // 16-byte piece of the row
-            const uint4 da16 = make_uint4(dao[0], dao[1], dao[2], dao[3]);
-            // dA into the MMA operand tile (row-major over dims, 128B swizzle)
-            *reinterpret_cast<uint4*>(slot + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) = da16;
-            if (valid_row) {
-              dgrow[c16] = make_uint4(dgo[0], dgo[1], dgo[2], dgo[3]);
-              darow[c16] = da16;
-            }
+          for (int e = 0; e < 16; ++e) {
+            const float2 gg = bf2(gc[e]), dd = bf2(dc[e]);
+            const float2 av = __fmul2_rn(
+                make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), il2);  // A / l
+            const float2 sg = make_float2(sigmoid_fast(gg.x), sigmoid_fast(gg.y));  // one MUFU op each
+            const float2 ds = __ffma2_rn(make_float2(-sg.x, -sg.y), sg, sg);      // s (1 - s)
+            const float2 dgv = __fmul2_rn(__fmul2_rn(dd, av), ds);
+            dgo[e] = pack_bf16x2(dgv.x, dgv.y);
+            dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+            const float2 dav = __fmul2_rn(dd, sg);
+            dao[e] = pack_f16x2(dav.x, dav.y);
+            dsum2 = __ffma2_rn(f16x2(dao[e]), av, dsum2);  // D uses the rounded dA the MMAs see
           }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
+            // dA into the MMA operand tile (row-major over dims, 128B swizzle)
+            const int c16 = 4 * ch + i;  // 16-byte piece of the row
+            *reinterpret_cast<uint4*>(slot + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) =
+                make_uint4(dao[4 * i], dao[4 * i + 1], dao[4 * i + 2], dao[4 * i + 3]);
+          }
+          if (valid_row) {
+            st32B(dgrow + 64 * ch, *reinterpret_cast<const uint32_t(*)[8]>(dgo));
+            st32B(dgrow + 64 * ch + 32, *reinterpret_cast<const uint32_t(*)[8]>(dgo + 8));
+            st32B(darow + 64 * ch, *reinterpret_cast<const uint32_t(*)[8]>(dao));
+            st32B(darow + 64 * ch + 32, *reinterpret_cast<const uint32_t(*)[8]>(dao + 8));
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
             gc[i] = gn[i];
             dc[i] = dn[i];
           }

@@ -104,7 +104,10 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
  * (bf16) and ADDS the weight gradients into dwq, dwk [D] (fp32; the caller
  * zeroes them).  `workspace` is caller-owned device scratch of at least
  * swa_bwd_workspace_size(p) bytes, 256-byte aligned; its contents on entry
- * do not matter.  The chain rule covers the gate, the softmax, RoPE and the
+ * do not matter.  g, dO and dg must be 32-byte aligned (their rows move in
+ * 32-byte accesses); the other tensors 16-byte, as everywhere else; a
+ * misaligned pointer returns SWA_ERR_INVALID_ARG before any launch.  The
+ * chain rule covers the gate, the softmax, RoPE and the
  * RMSNorm (the weights included).  The contractions run on fp16 operands
  * (three more mantissa bits than bf16), so |v| and |dO| must stay within the
  * fp16 range (65504) and |wq|, |wk| <= 4096; values beyond are reported by

@@ -116,5 +116,9 @@ def test_bwd_host_checks(L):
     assert L.swa_bwd(ctypes.byref(p), *args, need - 1, None) == swa.ERR_INVALID_ARG
     args[14] = ctypes.c_void_p((1 << 20) + 16)  # workspace must be 256-byte aligned
     assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
+    for i in (3, 7, 11):  # g, dO, dg move in 32-byte accesses: 16-byte alignment is not enough
+        args = [good] * 15
+        args[i] = ctypes.c_void_p((1 << 20) + 16)
+        assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
     nul = ctypes.c_void_p(0)
     assert L.swa_bwd(ctypes.byref(_params(T=0)), *([nul] * 15), 0, nul) == swa.OK
