@@ -226,9 +226,10 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
   if (!q || !k || !v || !g || !wq || !wk || !lse || !dO || !dq || !dk || !dv || !dg || !dwq ||
       !dwk || !workspace)
     return SWA_ERR_INVALID_ARG;
-  // g, dO and dg rows move in 32-byte accesses, one row per thread.
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(g) || !aligned16(wq) ||
-      !aligned16(wk) || !aligned32(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+  // Rows of q, k, g, dO and of the gradients move in 32-byte accesses, one
+  // row per thread.
+  if (!aligned32(q) || !aligned32(k) || !aligned16(v) || !aligned32(g) || !aligned16(wq) ||
+      !aligned16(wk) || !aligned32(dO) || !aligned32(dq) || !aligned32(dk) || !aligned32(dv) ||
       !aligned32(dg) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
       (reinterpret_cast<uintptr_t>(dwq) & 3u) || (reinterpret_cast<uintptr_t>(dwk) & 3u) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))

@@ -208,14 +208,14 @@ __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane
 
 // Half `half` of a raw bf16 row (32 words), or zeros for a row past the end.
 __device__ __forceinline__ void load_half(const uint16_t* xrow, int half, uint32_t (&x)[32]) {
+  if (xrow) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 u = xrow ? __ldg(reinterpret_cast<const uint4*>(xrow) + 8 * half + i)
-                         : make_uint4(0u, 0u, 0u, 0u);
-    x[4 * i] = u.x;
-    x[4 * i + 1] = u.y;
-    x[4 * i + 2] = u.z;
-    x[4 * i + 3] = u.w;
+    for (int i = 0; i < 4; ++i)
+      ld32B(reinterpret_cast<const uint8_t*>(xrow) + 128 * half + 32 * i,
+            *reinterpret_cast<uint32_t(*)[8]>(x + 8 * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = 0u;
   }
 }
 
@@ -303,9 +303,9 @@ __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16
     }
     if (out) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        reinterpret_cast<uint4*>(out)[8 * half + i] =
-            make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      for (int i = 0; i < 4; ++i)
+        st32B(reinterpret_cast<uint8_t*>(out) + 128 * half + 32 * i,
+              *reinterpret_cast<const uint32_t(*)[8]>(o + 8 * i));
     }
   }
 }
@@ -313,8 +313,8 @@ __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16
 // One 256-byte row per thread, in 16-byte pieces (rows are 16-byte aligned).
 __device__ __forceinline__ void store_row(uint16_t* p, const uint32_t (&x)[64]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
-    reinterpret_cast<uint4*>(p)[i] = make_uint4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+  for (int i = 0; i < 8; ++i)
+    st32B(reinterpret_cast<uint8_t*>(p) + 32 * i, *reinterpret_cast<const uint32_t(*)[8]>(x + 8 * i));
 }
 
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {

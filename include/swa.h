@@ -104,8 +104,8 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
  * (bf16) and ADDS the weight gradients into dwq, dwk [D] (fp32; the caller
  * zeroes them).  `workspace` is caller-owned device scratch of at least
  * swa_bwd_workspace_size(p) bytes, 256-byte aligned; its contents on entry
- * do not matter.  g, dO and dg must be 32-byte aligned (their rows move in
- * 32-byte accesses); the other tensors 16-byte, as everywhere else; a
+ * do not matter.  q, k, g, dO, dq, dk, dv and dg must be 32-byte aligned
+ * (their rows move in 32-byte accesses); v 16-byte, as everywhere else; a
  * misaligned pointer returns SWA_ERR_INVALID_ARG before any launch.  The
  * chain rule covers the gate, the softmax, RoPE and the
  * RMSNorm (the weights included).  The contractions run on fp16 operands

@@ -116,7 +116,7 @@ def test_bwd_host_checks(L):
     assert L.swa_bwd(ctypes.byref(p), *args, need - 1, None) == swa.ERR_INVALID_ARG
     args[14] = ctypes.c_void_p((1 << 20) + 16)  # workspace must be 256-byte aligned
     assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
-    for i in (3, 7, 11):  # g, dO, dg move in 32-byte accesses: 16-byte alignment is not enough
+    for i in (0, 1, 3, 7, 8, 9, 10, 11):  # rows in 32-byte accesses: 16-byte alignment is not enough
         args = [good] * 15
         args[i] = ctypes.c_void_p((1 << 20) + 16)
         assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
