@@ -206,16 +206,15 @@ __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane
   return make_float2(v[0], v[1]);
 }
 
-// Half `half` of a raw bf16 row (32 words), or zeros for a row past the end.
-__device__ __forceinline__ void load_half(const uint16_t* xrow, int half, uint32_t (&x)[32]) {
+// A raw bf16 row (64 words), or zeros for a row past the end.
+__device__ __forceinline__ void load_row(const uint16_t* xrow, uint32_t (&x)[64]) {
   if (xrow) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      ld32B(reinterpret_cast<const uint8_t*>(xrow) + 128 * half + 32 * i,
-            *reinterpret_cast<uint32_t(*)[8]>(x + 8 * i));
+    for (int i = 0; i < 8; ++i)
+      ld32B(reinterpret_cast<const uint8_t*>(xrow) + 32 * i, *reinterpret_cast<uint32_t(*)[8]>(x + 8 * i));
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0u;
+    for (int i = 0; i < 64; ++i) x[i] = 0u;
   }
 }
 
@@ -247,12 +246,12 @@ __device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half,
 
 // Gradient of one row through RoPE and RMSNorm.  dz: the gradient w.r.t. the
 // rotated, normalised row, in TMEM columns [t_lane_col, +128) of this thread's
-// lane; xrow: the raw row in global memory (nullptr: a row past the end).
+// lane; x: the raw row (load_row, issued early to hide its latency).
 // Writes dx to `out` (unless nullptr) and adds dy (*) xhat into dw (shared,
 // summed over the warp first).  Works half a row at a time; the rotation
 // factors are computed once for both passes.
 template <int kPairs>
-__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16_t* xrow,
+__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint32_t (&xr)[64],
                                                float rinv, const float* w, const float2 (*hi)[8],
                                                const RotTables& t, int row, int lane, float* dw,
                                                uint16_t* out) {
@@ -265,12 +264,10 @@ __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
-    uint32_t x[32];
-    load_half(xrow, half, x);
     load_dy_half<kPairs>(t_lane_col, half, rc, y);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = __fmul2_rn(bf2(x[i]), rinv2);  // xhat
+      const float2 xh = __fmul2_rn(bf2(half ? xr[32 + i] : xr[i]), rinv2);  // xhat
       const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
       const int d = half * 64 + 2 * i;
       dot2 = __ffma2_rn(__fmul2_rn(yv, make_float2(w[d], w[d + 1])), xh, dot2);
@@ -288,13 +285,11 @@ __device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint16
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float y[64];
-    uint32_t x[32];
-    load_half(xrow, half, x);
     load_dy_half<kPairs>(t_lane_col, half, rc, y);
     uint32_t o[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float2 xh = __fmul2_rn(bf2(x[i]), rinv2);
+      const float2 xh = __fmul2_rn(bf2(half ? xr[32 + i] : xr[i]), rinv2);
       const int d = half * 64 + 2 * i;
       const float2 g = __fmul2_rn(
           rinv2, __ffma2_rn(xh, ndot2,
@@ -864,9 +859,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       // ---- dq through RoPE^-1 and the RMSNorm Jacobian
+      uint32_t xq[64];  // the raw q row, loaded while dQ is computed
+      load_row(valid_row ? a.q + tok * kHeadDim : nullptr, xq);
       if (!(ok = warp_wait(&sm.dqfull, ph, abort, a.err, kSiteDQFull))) break;
       tc_fence_after();
-      norm_rope_grad<kPairs>(t_row + 128, valid_row ? a.q + tok * kHeadDim : nullptr, rinv_q,
+      norm_rope_grad<kPairs>(t_row + 128, xq, rinv_q,
                              sm.wq, sm.rot_hi[sc], sm.rot, row, lane, sm.dw,
                              valid_row ? a.dq + tok * kHeadDim : nullptr);
       tc_fence_before();
@@ -1189,9 +1186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j
       const long long krow = (static_cast<long long>(c.b) * a.T + kpos) * a.Hkv + c.kvh;
+      uint32_t xk[64];  // the raw k row, loaded while dK is computed
+      load_row(kpos < a.T ? a.k + krow * kHeadDim : nullptr, xk);
       if (!(ok = warp_wait(&sm.dkvfull, it & 1, abort, a.err, kSiteDKVFull))) break;
       tc_fence_after();
-      norm_rope_grad<kPairs>(t_row + 128, kpos < a.T ? a.k + krow * kHeadDim : nullptr, rinv_k,
+      norm_rope_grad<kPairs>(t_row + 128, xk, rinv_k,
                              sm.wk, sm.rot_hi[it & 1][0], sm.rot, row, lane, sm.dw,
                              kpos < a.T ? a.dk + krow * kHeadDim : nullptr);
       {
