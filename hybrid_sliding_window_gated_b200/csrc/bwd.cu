@@ -1112,12 +1112,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int dt = i / a.G;  // query tile j + dt
         const int hq = c.kvh * a.G + i % a.G;
         const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // this thread's query row
-        // ---- Q'_i, and lse / D of its rows for the column-wise softmax
+        // ---- Q'_i, and lse / D of its rows for the column-wise softmax (their
+        // loads go out first, so the transform hides their latency)
+        const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + qpos;
+        const float lse_i = qpos < a.T ? __ldg(a.ws_lse + lrow) : 0.f;
+        const float d_i = qpos < a.T ? __ldg(a.ws_d + lrow) : 0.f;
         if (!(ok = warp_wait(&sm.qfull[nq & 1], (nq >> 1) & 1, abort, a.err, kSiteQFull))) break;
         norm_rope_row<kPairs>(sm.q[nq & 1], row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
-        const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + qpos;
-        sm.lse2[nq & 1][row] = qpos < a.T ? a.ws_lse[lrow] * kLog2e : 0.f;
-        sm.dd[nq & 1][row] = qpos < a.T ? a.ws_d[lrow] : 0.f;
+        sm.lse2[nq & 1][row] = lse_i * kLog2e;
+        sm.dd[nq & 1][row] = d_i;
         fence_proxy_async_smem();
         mbar_arrive(&sm.qready);
         mbar_arrive(&sm.staged);  // lse2 / dd of this pair visible to the warpgroup
