@@ -395,6 +395,7 @@ def secondary(swa, args, world, device, stream, peaks):
     torch.cuda.empty_cache()
     out["train_fwd_bwd"] = train_bench(swa, args, world, device, stream, peaks)
     out["decode_step"] = decode_bench(swa, args, world, device, stream, peaks)
+    out["prefill_to_ring"] = ring_bench(swa, args, world, device, stream, peaks)
     return out
 
 
@@ -478,11 +479,42 @@ def decode_bench(swa, args, world, device, stream, peaks):
     return res
 
 
+def ring_bench(swa, args, world, device, stream, peaks):
+    """The prefill -> ring handoff for the decode batch: 256 sequences with a
+    256-token prefix, 8 KV heads; the last 128 positions' k and v are read and
+    the K and V rings written (128 B x 4 per element row: 268 MB per call over
+    two rotating input sets of 536 MB each, > L2)."""
+    N, T, Hkv, Hq, D, W = 256, 256, 8, 32, 128, 128
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    sets = []
+    for _ in range(2):
+        k = torch.randn((N, T, Hkv, D), generator=gen).to(torch.bfloat16).to(device)
+        v = torch.randn((N, T, Hkv, D), generator=gen).to(torch.bfloat16).to(device)
+        kc = torch.empty((N, Hkv, W, D), dtype=torch.bfloat16, device=device)
+        sets.append((k, v, kc, torch.empty_like(kc)))
+    wk = (1.0 + 0.1 * torch.randn(D, generator=gen)).to(device)
+
+    def mk(x):
+        return lambda: swa.prefill_to_ring(x[0], x[1], wk, x[2], x[3], Hq=Hq, rope_base=1e7)
+    steps = max(5, min(args.steps, 20))
+    ms, per, _, _ = timed_loop([mk(x) for x in sets], steps, 3, stream, world, per_launch=True)
+    b = 4 * N * Hkv * W * D * 2  # read k, v rows; write the K and V ring slots
+    res = {"workload": f"prefill -> ring handoff, {N} sequences x {T} tokens, {Hkv} kv heads",
+           "ms_per_call": round(ms / steps, 5),
+           "algorithmic_bytes_per_call": b,
+           "achieved_GBps": round(b / (per / 1e3) / 1e9, 1),
+           "frac_of_measured_hbm": round(b / (per / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del sets
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_profile(args, device):
     """Warmup + steps calls of one entry point, nothing else, so that a
     profiler sees a short, predictable launch list: `fwd` on the layer-shape
     workload, `decode` on one layer of the decode workload, `bwd` (with the
-    forward that produces its lse) on the training shape."""
+    forward that produces its lse) on the training shape, `ring` on the
+    prefill -> ring handoff of the decode batch."""
     import hybrid_sliding_window_gated_b200 as swa
     which = args.profile
     if which == "fwd":
@@ -495,6 +527,15 @@ def run_profile(args, device):
         fns = [lambda: swa.decode_step(x["pos"], x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"],
                                        x["k_cache"], x["v_cache"], rot_dim=cfg.R,
                                        rope_base=cfg.base, eps=cfg.eps, out=o)]
+    elif which == "ring":
+        cfg = workloads.custom_prefill(256, 256, 32, 8, base=1e7, seed=7)
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        k = torch.randn((256, 256, 8, 128), generator=gen).to(torch.bfloat16).to(device)
+        v = torch.randn((256, 256, 8, 128), generator=gen).to(torch.bfloat16).to(device)
+        wk = (1.0 + 0.1 * torch.randn(128, generator=gen)).to(device)
+        kc = torch.empty((256, 8, 128, 128), dtype=torch.bfloat16, device=device)
+        vc = torch.empty_like(kc)
+        fns = [lambda: swa.prefill_to_ring(k, v, wk, kc, vc, Hq=32, rope_base=1e7)]
     else:
         cfg = workloads.TRAIN
         d = workloads.prefill_inputs(cfg, device=device, with_grad_out=True)
@@ -553,7 +594,7 @@ def main():
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "decode", "bwd"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "decode", "bwd", "ring"], default=None,
                     help="only warmup + steps calls of one entry point (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -59,6 +59,8 @@ def lib():
         L.swa_bwd_workspace_size.restype = ctypes.c_size_t
         L.swa_decode_step.argtypes = [P] + [_vp] * 11
         L.swa_decode_step.restype = ctypes.c_int
+        L.swa_prefill_to_ring.argtypes = [P] + [_vp] * 6
+        L.swa_prefill_to_ring.restype = ctypes.c_int
         L.swa_error_string.argtypes = [ctypes.c_int]
         L.swa_error_string.restype = ctypes.c_char_p
         L.swa_get_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int)]
@@ -168,6 +170,19 @@ def decode_step(pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, *, rot_dim=42
                                _stream(stream))
     _check(rc, "swa_decode_step")
     return out
+
+
+def prefill_to_ring(k, v, wk, k_cache, v_cache, *, Hq, rot_dim=42, rope_base=1e7, eps=1e-6,
+                    stream=None):
+    """Fill the [B,Hkv,128,128] decode rings from a prefill's k, v [B,T,Hkv,128]
+    (swa_prefill_to_ring), so decode_step can continue at position T."""
+    B, T, Hkv, D = k.shape
+    W = k_cache.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
+                    eps=eps)
+    rc = lib().swa_prefill_to_ring(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(wk), _ptr(k_cache),
+                                   _ptr(v_cache), _stream(stream))
+    _check(rc, "swa_prefill_to_ring")
 
 
 def get_last_device_error(stream=None):

@@ -303,6 +303,30 @@ size_t swa_bwd_workspace_size(const swa_params_t* p) {
   return bwd_ws_da_bytes(p->B, p->T, p->Hq) + 2 * bwd_ws_d_bytes(p->B, p->T, p->Hq);
 }
 
+int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf16_t* v,
+                        const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache, void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  if (!k || !v || !wk || !k_cache || !v_cache) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(wk) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return SWA_ERR_INVALID_ARG;
+  RingArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hkv = p->Hkv;
+  a.half_rot = p->rot_dim / 2;
+  a.eps = p->eps;
+  a.k = k;
+  a.v = v;
+  a.wk = wk;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  fill_inv_freq(p, a.inv_freq);
+  return launch_prefill_ring(a, static_cast<cudaStream_t>(stream));
+}
+
 int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
                     const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
                     const float* wq, const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,

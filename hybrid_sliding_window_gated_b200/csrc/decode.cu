@@ -383,6 +383,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 }
 
+// Prefill -> ring handoff.  Slot s of ring (b, kv head h) takes the latest
+// prefill position p <= T-1 with p = s (mod W): k' = RoPE_p(RMSNorm(k_p))
+// rounded to bf16, exactly as a decode step writes its new token, and v_p as
+// it is.  Slots that no position reaches (s > T-1) keep their contents.  One
+// warp per (sequence, slot): the slot's rotation is computed once for all KV
+// heads, whose rows lie next to each other; 4 dims per lane, so each 256-byte
+// row is one coalesced access.
+__global__ void __launch_bounds__(128) swa_prefill_ring_kernel(const RingArgs a) {
+  __shared__ __align__(16) float scratch[4][kHeadDim];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;
+  const int b = static_cast<int>(gw / kWindow), s = static_cast<int>(gw % kWindow);
+  if (b >= a.B || s > a.T - 1) return;  // warp-uniform
+  const long long p = (a.T - 1) - ((a.T - 1 - s) % kWindow);
+  float cs = 1.0f, sn = 0.0f;
+  if (lane < a.half_rot) rope_cos_sin(static_cast<double>(p), a.inv_freq[lane], &cs, &sn);
+  for (int h = 0; h < a.Hkv; ++h) {
+    const long long row = ((static_cast<long long>(b) * a.T + p) * a.Hkv + h) * kHeadDim;
+    float x[4];
+    load4(a.k + row + 4 * lane, x);
+    const uint2 vv = *reinterpret_cast<const uint2*>(a.v + row + 4 * lane);
+    norm_rope_row(x, a.wk, a.eps, scratch[warp], lane, a.half_rot, cs, sn);
+    const long long ring_row = ((static_cast<long long>(b) * a.Hkv + h) * kWindow + s) * kHeadDim;
+    *reinterpret_cast<uint2*>(a.k_cache + ring_row + 4 * lane) =
+        make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+    *reinterpret_cast<uint2*>(a.v_cache + ring_row + 4 * lane) = vv;
+  }
+}
+
 }  // namespace dec
 
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a,
@@ -403,6 +434,13 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a
   const long long grid = units < di.num_sms ? units : di.num_sms;
   return launch_dependent(dec::swa_decode_kernel, static_cast<unsigned>(grid), dec::kThreads, smem,
                           stream, tk, tv, a);
+}
+
+int launch_prefill_ring(const RingArgs& a, cudaStream_t stream) {
+  const long long grid = static_cast<long long>(a.B) * (kWindow / 4);  // 4 warps per block
+  if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  return launch_dependent(dec::swa_prefill_ring_kernel, static_cast<unsigned>(grid), 128, 0, stream,
+                          a);
 }
 
 }  // namespace swa

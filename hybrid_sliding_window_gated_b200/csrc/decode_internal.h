@@ -32,4 +32,19 @@ constexpr int kDevErrBadPosition = 0x200;
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a,
                   cudaStream_t stream);
 
+// Prefill -> ring handoff (see swa_prefill_to_ring).
+struct RingArgs {
+  int B, T, Hkv;
+  int half_rot;
+  float eps;
+  const uint16_t* k;  // [B, T, Hkv, D]
+  const uint16_t* v;
+  const float* wk;
+  uint16_t* k_cache;  // [B, Hkv, W, D]
+  uint16_t* v_cache;
+  double inv_freq[kMaxPairs];
+};
+
+int launch_prefill_ring(const RingArgs& a, cudaStream_t stream);
+
 }  // namespace swa

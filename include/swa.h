@@ -155,6 +155,22 @@ int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t*
                     const float* wq, const float* wk, swa_bf16_t* k_cache,
                     swa_bf16_t* v_cache, swa_bf16_t* o, void* stream);
 
+/*
+ * Prefill -> ring handoff: after a prefill of p->T tokens, fill the decode
+ * rings so that swa_decode_step can continue at position T.  k, v:
+ * [B,T,Hkv,D] bf16 (the prefill's raw k and v); wk [D] fp32.  k_cache,
+ * v_cache: [B,Hkv,W,D] bf16 rings, updated in place: slot s receives the
+ * latest position p <= T-1 with p = s (mod W) -- k' = RoPE(RMSNorm(k_p)),
+ * rounded to bf16 exactly as swa_decode_step writes its new token, and v_p
+ * (bit-exact copy).  Slots that no position reaches (s > T-1, when T < W)
+ * keep their contents, which the decode ignores.  Pointers 16-byte aligned;
+ * returns SWA_ERR_INVALID_ARG / UNSUPPORTED like swa_fwd.  No counterpart in
+ * the pages beyond the serving view (the window layers' KV cache holds the
+ * last W tokens: jaehun.me review, "Why the KV Cache Shrinks by 6.4x").
+ */
+int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf16_t* v,
+                        const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache, void* stream);
+
 /* Static description of an error code. */
 const char* swa_error_string(int code);
 

@@ -205,6 +205,31 @@ def decode(pos, q, k_new, v_new, g, wq, wk, k_cache_bits, v_cache_bits, *, R, ba
     return o, kc, vc
 
 
+def prefill_to_ring(k, v, wk, k_cache_bits, v_cache_bits, *, R, base, eps):
+    """Decode rings after a prefill of T tokens.
+
+    Slot s of ring (b, h) holds the key and value of the latest position
+    p <= T-1 with p = s (mod W), the slot a decode step of that position
+    writes (jaehun.me review, "Why the KV Cache Shrinks by 6.4x": the window
+    layers keep only their last W tokens): k' = RoPE_p(RMSNorm(k_p, wk))
+    rounded to bf16, and v_p unchanged.  Slots no position reaches keep their
+    bits.  k, v: [B, T, Hkv, D] (fp64 values of bf16 inputs); caches
+    [B, Hkv, W, D] as uint16 bf16 bits (copied, not modified).
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    kc = np.array(k_cache_bits, dtype=np.uint16, copy=True, order="C")
+    vc = np.array(v_cache_bits, dtype=np.uint16, copy=True, order="C")
+    B, T = k.shape[0], k.shape[1]
+    W = kc.shape[2]
+    for p in range(max(0, T - W), T):  # the last W positions, each to its own slot
+        s = p % W
+        kp = norm_rope(k[:, p], wk, np.full(B, float(p)), R, base, eps)  # [B, Hkv, D]
+        kc[:, :, s, :] = bf16_round_array(kp)
+        vc[:, :, s, :] = bf16_round_array(v[:, p])
+    return kc, vc
+
+
 def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, bytes_per_elt: int) -> int:
     """KV-cache bytes per token for ``layers`` layers that keep every token."""
     return int(lib().oracle_kv_bytes_per_token(layers, kv_heads, head_dim, bytes_per_elt))

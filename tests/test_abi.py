@@ -122,3 +122,17 @@ def test_bwd_host_checks(L):
         assert L.swa_bwd(ctypes.byref(p), *args, need, None) == swa.ERR_INVALID_ARG
     nul = ctypes.c_void_p(0)
     assert L.swa_bwd(ctypes.byref(_params(T=0)), *([nul] * 15), 0, nul) == swa.OK
+
+
+def test_prefill_to_ring_host_checks(L):
+    nul = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(1 << 20)
+    p = _params(B=2, T=300, Hq=8, Hkv=2)
+    assert L.swa_prefill_to_ring(ctypes.byref(p), *([nul] * 5), nul) == swa.ERR_INVALID_ARG
+    assert L.swa_prefill_to_ring(ctypes.byref(_params(B=0)), *([nul] * 5), nul) == swa.OK
+    assert L.swa_prefill_to_ring(ctypes.byref(_params(T=0)), *([nul] * 5), nul) == swa.OK
+    assert L.swa_prefill_to_ring(ctypes.byref(_params(window=64)), *([good] * 5), nul) == \
+        swa.ERR_UNSUPPORTED
+    args = [good] * 5
+    args[3] = ctypes.c_void_p((1 << 20) + 8)  # rings must be 16-byte aligned
+    assert L.swa_prefill_to_ring(ctypes.byref(p), *args, nul) == swa.ERR_INVALID_ARG

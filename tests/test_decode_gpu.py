@@ -143,3 +143,57 @@ def test_forced_timeout_is_reported_and_context_survives():
     assert swa.get_last_device_error()[0] == swa.OK
     o, kc2, vc2, o_ref, kc_ref, vc_ref = run_both(inp, 42, cfg.base)
     assert_parity(to_f64(o), o_ref, "decode o after a forced timeout")
+
+
+@pytest.mark.parametrize("T", [1, 77, 128, 300])
+def test_prefill_to_ring_matches_oracle(T):
+    """swa_prefill_to_ring: V slots bit-exact, K slots within one bf16 step of
+    the oracle's k', slots no position reaches untouched."""
+    cfg = workloads.custom_prefill(2, T, 8, 2, base=1e7, g_std=1.0, seed=30 + T)
+    inp = workloads.prefill_inputs(cfg)
+    gen = torch.Generator(device="cpu").manual_seed(T)
+    kc0 = (torch.randn((2, 2, 128, 128), generator=gen) * 50).to(torch.bfloat16)
+    vc0 = (torch.randn((2, 2, 128, 128), generator=gen) * 50).to(torch.bfloat16)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    kc, vc = kc0.to(DEV), vc0.to(DEV)
+    swa.prefill_to_ring(d["k"], d["v"], d["wk"], kc, vc, Hq=8, rot_dim=cfg.R, rope_base=cfg.base,
+                        eps=cfg.eps)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    kr, vr = oracle.prefill_to_ring(f64(inp["k"]), f64(inp["v"]), f64(inp["wk"]), bits(kc0),
+                                    bits(vc0), R=cfg.R, base=cfg.base, eps=cfg.eps)
+    got_k, got_v = bits(kc), bits(vc)
+    assert np.array_equal(got_v, vr)
+    reached = min(T, 128)
+    assert np.array_equal(got_k[:, :, reached:], bits(kc0)[:, :, reached:])
+    gk = oracle.bf16_bits_to_f64(got_k[:, :, :reached])
+    rk = oracle.bf16_bits_to_f64(kr[:, :, :reached])
+    assert np.all(np.abs(gk - rk) <= np.abs(rk) * 2.0 ** -7 + 1e-30)
+    assert np.mean(got_k[:, :, :reached] == kr[:, :, :reached]) > 0.95
+
+
+def test_prefill_then_decode_continues_the_sequence():
+    """Prefill T tokens (forward + ring handoff), then decode token T: the
+    decode row equals row T of the oracle's forward over T + 1 tokens."""
+    T = 200
+    cfg = workloads.custom_prefill(2, T + 1, 8, 2, base=1e7, g_std=1.0, seed=33)
+    inp = workloads.prefill_inputs(cfg)
+    o_ref, _ = oracle.fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                          f64(inp["wq"]), f64(inp["wk"]), W=cfg.W, R=cfg.R, base=cfg.base,
+                          eps=cfg.eps)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    pre = {x: d[x][:, :T].contiguous() for x in ("q", "k", "v", "g")}
+    o_pre = swa.fwd(pre["q"], pre["k"], pre["v"], pre["g"], d["wq"], d["wk"], rot_dim=cfg.R,
+                    rope_base=cfg.base, eps=cfg.eps)
+    kc = torch.zeros((2, 2, 128, 128), dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    swa.prefill_to_ring(pre["k"], pre["v"], d["wk"], kc, vc, Hq=8, rot_dim=cfg.R,
+                        rope_base=cfg.base, eps=cfg.eps)
+    pos = torch.full((2,), T, dtype=torch.int64, device=DEV)
+    o_dec = swa.decode_step(pos, d["q"][:, T].contiguous(), d["k"][:, T].contiguous(),
+                            d["v"][:, T].contiguous(), d["g"][:, T].contiguous(), d["wq"], d["wk"],
+                            kc, vc, rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    assert_parity(to_f64(o_pre), o_ref[:, :T], "prefill rows")
+    assert_parity(to_f64(o_dec), o_ref[:, T], "decode row after the ring handoff")

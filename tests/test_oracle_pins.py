@@ -326,6 +326,27 @@ def test_decode_equals_prefill_row(p):
     assert np.array_equal(kc2[0, :, s], oracle.bf16_round_array(kp[0]))
 
 
+@pytest.mark.parametrize("T", [1, 50, 128, 131, 260])
+def test_prefill_to_ring_equals_sequential_decode(T):
+    """The rings after a prefill of T tokens hold what T decode steps
+    (positions 0..T-1) leave behind, starting from the same noise; slots no
+    position reaches keep the noise."""
+    W, R, base, eps, Hq, Hkv, D, B = 128, 42, 1e7, 1e-6, 4, 2, 128, 2
+    q, k, v, g, wq, wk = rand_inputs(B, T, Hq, Hkv, D, seed=60 + T)
+    rng = np.random.default_rng(T)
+    kc0 = oracle.bf16_round_array(rng.standard_normal((B, Hkv, W, D)) * 50)
+    vc0 = oracle.bf16_round_array(rng.standard_normal((B, Hkv, W, D)) * 50)
+    kc, vc = kc0, vc0
+    for t in range(T):
+        _, kc, vc = oracle.decode(np.full(B, t), q[:, t], k[:, t], v[:, t], g[:, t], wq, wk,
+                                  kc, vc, R=R, base=base, eps=eps)
+    kr, vr = oracle.prefill_to_ring(k, v, wk, kc0, vc0, R=R, base=base, eps=eps)
+    assert np.array_equal(kr, kc) and np.array_equal(vr, vc)
+    if T < W:
+        assert np.array_equal(kr[:, :, T:], kc0[:, :, T:])
+        assert np.array_equal(vr[:, :, T:], vc0[:, :, T:])
+
+
 def test_decode_matches_dense_over_ring_contents():
     """Decode output = dense softmax over the ring's keys (positions known)."""
     W, R, base, eps, Hq, Hkv, D, N = 128, 42, 1e7, 1e-6, 8, 2, 128, 3
