@@ -34,7 +34,14 @@
 namespace swa {
 namespace bwd {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;   // key-major pass
+constexpr int kThreadsQ = 384;  // query-major pass: control + two compute warpgroups
+// Query-major pass: launch budget 384 x 168 registers, rebalanced with
+// setmaxnreg between the control warpgroup and the two compute warpgroups.
+constexpr int kRegsLaunchQ = 168;
+constexpr int kRegsControl = 56;
+constexpr int kRegsCompute = 224;
+static_assert(kRegsControl + 2 * kRegsCompute <= 3 * kRegsLaunchQ, "register split");
 constexpr int kHalfBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 (one TMA box)
 constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -43,7 +50,7 @@ enum Site {
   kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
   kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
   kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged,
-  kSiteMmaDone, kSiteForced
+  kSiteMmaDone, kSiteForced, kSiteXchg
 };
 
 // ---------------------------------------------------------------- helpers
@@ -109,7 +116,7 @@ __device__ __forceinline__ float2 cmul(float2 x, float2 y) {
 // warp-collective tcgen05 loads and stores that follow never run divergent.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err, int site) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err, site));
+  return __all_sync(0xffffffffu, mbar_wait_inl(bar, parity, abort, err, site));
 }
 
 struct RotTables {
@@ -379,13 +386,17 @@ struct alignas(1024) SmemQ {
   uint64_t qfull[2], qempty[2];
   uint64_t qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
   uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
+  // Row-sum exchanges between the two compute warpgroups (l, D, the dq dot).
+  uint64_t xlb, xdb, xtb;
+  float xl[2][kTile], xd[2][kTile], xt[2][kTile];
+  float rinvq[kTile];  // 1/rms of each Q row (cg 0 computes it; both use it)
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(SmemQ) + 1024 <= 232448, "pass 1 shared memory");
 
 template <int kPairs>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsQ, 1)
     swa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -412,15 +423,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.qready, 128);
     mbar_init(&sm.sfull, 1);
-    mbar_init(&sm.pfull, 128);
+    mbar_init(&sm.pfull, 256);
     mbar_init(&sm.afull, 1);
-    mbar_init(&sm.dafull, 128);
+    mbar_init(&sm.dafull, 256);
     mbar_init(&sm.dpfull, 1);
-    mbar_init(&sm.dsfull, 128);
+    mbar_init(&sm.dsfull, 256);
     mbar_init(&sm.dq0, 1);
     mbar_init(&sm.dqfull, 1);
-    mbar_init(&sm.tfree, 128);
-    mbar_init(&sm.tables, 128);
+    mbar_init(&sm.tfree, 256);
+    mbar_init(&sm.tables, 256);
+    mbar_init(&sm.xlb, 256);
+    mbar_init(&sm.xdb, 256);
+    mbar_init(&sm.xtb, 256);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.never, 1);
     sm.abort = 0;
@@ -457,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int n_heads = n_tiles * a.G;
 
+  if (warp < 4) regs_dec<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint32_t kpar = 0, vpar = 0, kused = 0, vused = 0;  // per-slot parity / used bits
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nq = 0;
     auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
       bool w = true;
-      if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+      if (lane == 0) w = mbar_wait_inl(bar, par, abort, a.err, site);
       return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
     };
     auto load_kv = [&](bool is_k, int j, const Cursor& c) -> bool {
@@ -528,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Cursor c = cursor_at(a, u0);
       int h = 0;
       auto W = [&](uint64_t* bar, uint32_t par, int site) {
-        if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
+        if (ok) ok = mbar_wait_inl(bar, par, abort, a.err, site);
         return ok;
       };
       if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
@@ -625,11 +640,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------------------------------------------- compute warpgroup
-    const int row = tid - 128;
+    // --------------------------------------------------- compute warpgroups
+    // Two warpgroups share every query row: thread r of each owns row r
+    // (TMEM lane r).  Warpgroup cg takes
+    //   - the K transform (cg 0) or the V conversion (cg 1) of a new key tile,
+    //     and cg 0 the Q transform;
+    //   - chunks i = cg, cg + 2, ... of P over the band;
+    //   - columns [64 cg, 64 cg + 64) of the gate/dA phase, of dS and of the
+    //     dq epilogue.
+    // Row sums (l, D and the dq Jacobian's dot) are exchanged through shared
+    // memory, each under a bounded mbarrier wait that both warpgroups arrive on.
+    regs_inc<kRegsCompute>();
+    const int cg = (warp - 4) >> 2;
+    const int row = (tid - 128) & 127;
     const int wq4 = warp & 3;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16);
-    for (int e = row; e < kPairs * 16; e += 128) {
+    for (int e = tid - 128; e < kPairs * 16; e += 256) {
       const int p = e >> 4, bi = e & 15;
       float cv, sv;
       rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
@@ -639,7 +665,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = warp_wait(&sm.tables, 0, abort, a.err, kSiteTables);
     uint32_t kpar = 0, vpar = 0;
     bool in_range = true;  // v and dO within the fp16 staging range
-    int nds = 0, ndq0 = 0;
+    int ndq0 = 0;
+    // Publish this warpgroup's partial of a row sum and add the partner's.
+    auto exchange = [&](uint64_t* bar, float (*buf)[kTile], float v, uint32_t par, int site,
+                        float& total) -> bool {
+      buf[cg][row] = v;
+      mbar_arrive(bar);
+      if (!warp_wait(bar, par, abort, a.err, site)) return false;
+      total = v + buf[cg ^ 1][row];
+      return true;
+    };
     Cursor c = cursor_at(a, u0);
     int h = 0;
     for (int n = 0; n < n_heads && ok; ++n) {
@@ -652,82 +687,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long tok = (static_cast<long long>(c.b) * a.T + pos) * a.Hq + hq;  // row of q/g/dO
       const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + pos;  // lse / D
 
-      // ---- K' of this tile's new key tiles (first head of the tile)
+      // ---- K' (cg 0) and V in fp16 (cg 1) of this tile's new key tiles
       if (h == 0) {
         for (int j = (c.t > 0 && c.u == 0) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
           const int s = j & 1;
-          ok = warp_wait(&sm.kfull[s], (kpar >> s) & 1u, abort, a.err, kSiteKFull);
-          if (!ok) break;
-          norm_rope_row<kPairs>(sm.k[s], row, sm.wk, sm.rot_hi[s], sm.rot, a.eps);
-          fence_proxy_async_smem();
-          mbar_arrive(&sm.kready[s]);
-          kpar ^= 1u << s;
-          ok = warp_wait(&sm.vfull[s], (vpar >> s) & 1u, abort, a.err, kSiteVFull);
-          if (!ok) break;
-          in_range &= row_to_f16(sm.v[s], row);
-          fence_proxy_async_smem();
-          mbar_arrive(&sm.vready[s]);
-          vpar ^= 1u << s;
+          if (cg == 0) {
+            ok = warp_wait(&sm.kfull[s], (kpar >> s) & 1u, abort, a.err, kSiteKFull);
+            if (!ok) break;
+            norm_rope_row<kPairs>(sm.k[s], row, sm.wk, sm.rot_hi[s], sm.rot, a.eps);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.kready[s]);
+            kpar ^= 1u << s;
+          } else {
+            ok = warp_wait(&sm.vfull[s], (vpar >> s) & 1u, abort, a.err, kSiteVFull);
+            if (!ok) break;
+            in_range &= row_to_f16(sm.v[s], row);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.vready[s]);
+            vpar ^= 1u << s;
+          }
         }
         if (!ok) break;
       }
-      // ---- Q'
+      // ---- Q' (cg 0)
       uint8_t* slot = sm.slot[n & 1];
-      if (!(ok = warp_wait(&sm.qfull[n & 1], (n >> 1) & 1, abort, a.err, kSiteQFull))) break;
-      const float rinv_q = norm_rope_row<kPairs>(slot, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.qready);
+      const uint8_t* grow = reinterpret_cast<const uint8_t*>(a.g + tok * kHeadDim) + 128 * cg;
+      const uint8_t* dorow = reinterpret_cast<const uint8_t*>(a.dO + tok * kHeadDim) + 128 * cg;
+      if (cg == 0) {
+        if (!(ok = warp_wait(&sm.qfull[n & 1], (n >> 1) & 1, abort, a.err, kSiteQFull))) break;
+        sm.rinvq[row] = norm_rope_row<kPairs>(slot, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.qready);
+      }
       // Rows past T take lse = +inf: their P is exactly 0 with no mask.
       const float lse2 = valid_row ? a.lse[lrow] * kLog2e : INFINITY;
-      float2 lsum2 = make_float2(0.f, 0.f);
+      // this warpgroup's 64 columns of g and dO, in flight during P
+      uint32_t gc[32], dc[32];  // this warpgroup's 64 columns of g and dO
+      if (valid_row) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ld32B(grow + 32 * i, *reinterpret_cast<uint32_t(*)[8]>(gc + 8 * i));
+          ld32B(dorow + 32 * i, *reinterpret_cast<uint32_t(*)[8]>(dc + 8 * i));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) gc[i] = dc[i] = 0u;
+      }
 
-      // ---- P = exp(s - lse) on the band, packed over columns 0..127
+      // ---- P = exp(s - lse) on the band.  The in-band 32-column chunks are
+      // key tile t-1's wq4..3 (when it exists), then key tile t's 0..wq4;
+      // this warpgroup takes every other one.  P is packed over S's first 128
+      // columns, which the other warpgroup may still be reading, so the
+      // stores wait for the exchange of the row sums.
       if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
       tc_fence_after();
-      {
-        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
-#pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {
-#pragma unroll 1
-          for (int pc = 0; pc < 4; ++pc) {
-            // key tile t-1 keeps columns > row, key tile t columns <= row; only
-            // chunk pc == wq4 straddles the band edge.  Warp-uniform
-            // (tcgen05.ld is warp-collective).
-            const bool any = blk == 0 ? (hp && pc >= wq4) : (pc <= wq4);
-            uint32_t pk[16];
-            if (any) {
-              uint32_t x[32];
-              tmem_ld32(t_row + blk * 128 + pc * 32, x);
-              tmem_wait_ld();
-              if (pc != wq4) {
+      const int na = hp ? 4 - wq4 : 0;  // chunks of key tile t-1 in the band
+      const int nch = na + wq4 + 1;
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
+      float2 lsum2 = make_float2(0.f, 0.f);
+      uint32_t pk[3][16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const float2 z = __ffma2_rn(
-                      make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
-                  pk[e] = pack_f16x2(ex2_approx(z.x), ex2_approx(z.y));
-                  lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));  // the values the MMAs see
-                }
-              } else {
+      for (int k = 0; k < 3; ++k) {
+        const int i = cg + 2 * k;
+        if (i < nch) {
+          const int blk = i < na ? 0 : 1;
+          const int pc = blk == 0 ? wq4 + i : i - na;
+          uint32_t x[32];
+          tmem_ld32(t_row + blk * 128 + pc * 32, x);
+          tmem_wait_ld();
+          if (pc != wq4) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const int c0 = pc * 32 + 2 * e;
-                  const bool in0 = blk == 0 ? c0 > row : c0 <= row;
-                  const bool in1 = blk == 0 ? c0 + 1 > row : c0 + 1 <= row;
-                  const float2 z = __ffma2_rn(
-                      make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
-                  pk[e] = pack_f16x2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
-                  lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));
-                }
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            for (int e = 0; e < 16; ++e) {
+              const float2 z = __ffma2_rn(
+                  make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
+              pk[k][e] = pack_f16x2(ex2_approx(z.x), ex2_approx(z.y));
+              lsum2 = __fadd2_rn(lsum2, f16x2(pk[k][e]));  // the values the MMAs see
             }
-            tmem_st16(t_row + blk * 64 + pc * 16, pk);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = pc * 32 + 2 * e;
+              const bool in0 = blk == 0 ? c0 > row : c0 <= row;
+              const bool in1 = blk == 0 ? c0 + 1 > row : c0 + 1 <= row;
+              const float2 z = __ffma2_rn(
+                  make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
+              pk[k][e] = pack_f16x2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
+              lsum2 = __fadd2_rn(lsum2, f16x2(pk[k][e]));
+            }
           }
         }
       }
-      const float lsum = lsum2.x + lsum2.y;
+      float lsum;
+      if (!(ok = exchange(&sm.xlb, sm.xl, lsum2.x + lsum2.y, ph, kSiteXchg, lsum))) break;
+      {
+        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int i = cg + 2 * k;
+          if (i < nch) {
+            const int blk = i < na ? 0 : 1;
+            const int pc = blk == 0 ? wq4 + i : i - na;
+            tmem_st16(t_row + blk * 64 + pc * 16, pk[k]);
+          }
+        }
+        // chunks outside the band: key tile t-1's below wq4 (or all of it
+        // when it does not exist) by cg 0, key tile t's above wq4 by cg 1
+        for (int pc = 0; pc < 4; ++pc) {
+          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + pc * 16, zero16);
+          if (cg == 1 && pc > wq4) tmem_st16(t_row + 64 + pc * 16, zero16);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.pfull);
@@ -735,57 +805,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // are renormalised to sum to exactly 1 under this pass's scores, and the
       // corrected normaliser goes to the key-major pass.
       const float inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
-      if (valid_row) a.ws_lse[lrow] = a.lse[lrow] + __logf(lsum);
+      if (cg == 0 && valid_row) a.ws_lse[lrow] = a.lse[lrow] + __logf(lsum);
 
-      // ---- A: dg, dA (smem and workspace), D -- 32 dims at a time (a rolled
-      // loop keeps the code small), the next chunk's g and dO loads in flight
-      // while this one is computed (chunk 0's while the PV MMA runs).
-      const uint8_t* grow = reinterpret_cast<const uint8_t*>(a.g + tok * kHeadDim);
-      const uint8_t* dorow = reinterpret_cast<const uint8_t*>(a.dO + tok * kHeadDim);
-      uint32_t gc[16], dc[16];  // this chunk's 32 columns of g and dO
-      {
-        uint32_t (&g0)[8] = *reinterpret_cast<uint32_t(*)[8]>(gc);
-        uint32_t (&g1)[8] = *reinterpret_cast<uint32_t(*)[8]>(gc + 8);
-        uint32_t (&d0)[8] = *reinterpret_cast<uint32_t(*)[8]>(dc);
-        uint32_t (&d1)[8] = *reinterpret_cast<uint32_t(*)[8]>(dc + 8);
-        if (valid_row) {
-          ld32B(grow, g0);
-          ld32B(grow + 32, g1);
-          ld32B(dorow, d0);
-          ld32B(dorow + 32, d1);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) gc[i] = dc[i] = 0u;
-        }
-      }
+      // ---- A: dg, dA (smem and workspace) and D over this warpgroup's 64
+      // columns (TMEM chunks 2 cg, 2 cg + 1)
       if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
       tc_fence_after();
       float2 dsum2 = make_float2(0.f, 0.f);
       const float2 il2 = make_float2(inv_l, inv_l);
       float dmax = 0.f;  // largest |dO| of the row: fp16 staging range
       {
-        uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim);
-        uint8_t* darow = reinterpret_cast<uint8_t*>(a.ws_da + tok * kHeadDim);
+        uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim) + 128 * cg;
+        uint8_t* darow = reinterpret_cast<uint8_t*>(a.ws_da + tok * kHeadDim) + 128 * cg;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t gn[16], dn[16];
-          const bool more = valid_row && ch + 1 < 4;
-          if (more) {
-            ld32B(grow + 64 * (ch + 1), *reinterpret_cast<uint32_t(*)[8]>(gn));
-            ld32B(grow + 64 * (ch + 1) + 32, *reinterpret_cast<uint32_t(*)[8]>(gn + 8));
-            ld32B(dorow + 64 * (ch + 1), *reinterpret_cast<uint32_t(*)[8]>(dn));
-            ld32B(dorow + 64 * (ch + 1) + 32, *reinterpret_cast<uint32_t(*)[8]>(dn + 8));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) gn[i] = dn[i] = 0u;
-          }
+        for (int hc = 0; hc < 2; ++hc) {
+          const int ch = 2 * cg + hc;  // 32-column chunk of the row
           uint32_t x[32];
           tmem_ld32(t_row + 256 + ch * 32, x);
           tmem_wait_ld();
           uint32_t dgo[16], dao[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float2 gg = bf2(gc[e]), dd = bf2(dc[e]);
+            const uint32_t gw = gc[e];
+            const uint32_t dw = dc[e];
+            const float2 gg = bf2(gw), dd = bf2(dw);
             const float2 av = __fmul2_rn(
                 make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), il2);  // A / l
             const float2 sg = make_float2(sigmoid_fast(gg.x), sigmoid_fast(gg.y));  // one MUFU op each
@@ -805,45 +848,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(dao[4 * i], dao[4 * i + 1], dao[4 * i + 2], dao[4 * i + 3]);
           }
           if (valid_row) {
-            st32B(dgrow + 64 * ch, *reinterpret_cast<const uint32_t(*)[8]>(dgo));
-            st32B(dgrow + 64 * ch + 32, *reinterpret_cast<const uint32_t(*)[8]>(dgo + 8));
-            st32B(darow + 64 * ch, *reinterpret_cast<const uint32_t(*)[8]>(dao));
-            st32B(darow + 64 * ch + 32, *reinterpret_cast<const uint32_t(*)[8]>(dao + 8));
+            st32B(dgrow + 64 * hc, *reinterpret_cast<const uint32_t(*)[8]>(dgo));
+            st32B(dgrow + 64 * hc + 32, *reinterpret_cast<const uint32_t(*)[8]>(dgo + 8));
+            st32B(darow + 64 * hc, *reinterpret_cast<const uint32_t(*)[8]>(dao));
+            st32B(darow + 64 * hc + 32, *reinterpret_cast<const uint32_t(*)[8]>(dao + 8));
           }
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            gc[i] = gn[i];
-            dc[i] = dn[i];
+          for (int e = 0; e < 16; ++e) {  // the second chunk's g and dO move down
+            gc[e] = gc[16 + e];
+            dc[e] = dc[16 + e];
           }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.dafull);
       }
-      const float dsum = dsum2.x + dsum2.y;
       in_range &= !(dmax > kF16Max);
-      if (valid_row) a.ws_d[lrow] = dsum;
+      float dsum;
+      if (!(ok = exchange(&sm.xdb, sm.xd, dsum2.x + dsum2.y, ph, kSiteXchg, dsum))) break;
+      if (cg == 0 && valid_row) a.ws_d[lrow] = dsum;
 
-      // ---- dS = scale P (dP - D) per key tile into the Q slot, then dQ
+      // ---- dS = scale P (dP - D) per key tile into the Q slot (this
+      // warpgroup's 64 columns), then dQ
+      uint32_t xq[32];  // this warpgroup's half of the raw q row, loaded while dS and dQ run
+      if (valid_row) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          ld32B(reinterpret_cast<const uint8_t*>(a.q + tok * kHeadDim) + 128 * cg + 32 * i,
+                *reinterpret_cast<uint32_t(*)[8]>(xq + 8 * i));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xq[i] = 0u;
+      }
       if (!(ok = warp_wait(&sm.dpfull, ph, abort, a.err, kSiteDPFull))) break;
       tc_fence_after();
+      const float2 sl2 = make_float2(a.scale * inv_l, a.scale * inv_l), nd2 = make_float2(-dsum, -dsum);
       for (int blk = hp ? 0 : 1; blk < 2 && ok; ++blk) {
         if (blk == 1 && hp) {  // the MMA has read dS of key tile t-1 from the slot
           if (!(ok = warp_wait(&sm.dq0, ndq0 & 1, abort, a.err, kSiteDQ0))) break;
           ++ndq0;
         }
-        for (int pc = 0; pc < 4; ++pc) {
-          uint32_t pk[16], dp[32];
-          tmem_ld16(t_row + blk * 64 + pc * 16, pk);
+#pragma unroll 1
+        for (int hc = 0; hc < 2; ++hc) {
+          const int pc = 2 * cg + hc;
+          uint32_t pkc[16], dp[32];
+          tmem_ld16(t_row + blk * 64 + pc * 16, pkc);
           tmem_ld32(t_row + 256 + blk * 128 + pc * 32, dp);
           tmem_wait_ld();
           uint32_t ds[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float2 pp = f16x2(pk[e]);
-            const float d0 = a.scale * inv_l * pp.x * (__uint_as_float(dp[2 * e]) - dsum);
-            const float d1 = a.scale * inv_l * pp.y * (__uint_as_float(dp[2 * e + 1]) - dsum);
-            ds[e] = pack_f16x2(d0, d1);
+            const float2 v = __fmul2_rn(
+                __fmul2_rn(f16x2(pkc[e]), sl2),
+                __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                           nd2));
+            ds[e] = pack_f16x2(v.x, v.y);
           }
           uint8_t* half = slot + (pc >> 1) * kHalfBytes;
 #pragma unroll
@@ -854,20 +913,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.dsfull);
-        ++nds;
       }
       if (!ok) break;
 
-      // ---- dq through RoPE^-1 and the RMSNorm Jacobian
-      uint32_t xq[64];  // the raw q row, loaded while dQ is computed
-      load_row(valid_row ? a.q + tok * kHeadDim : nullptr, xq);
+      // ---- dq through RoPE^-1 and the RMSNorm Jacobian, over this
+      // warpgroup's half of the row (the rotated dims are all in half 0)
       if (!(ok = warp_wait(&sm.dqfull, ph, abort, a.err, kSiteDQFull))) break;
       tc_fence_after();
-      norm_rope_grad<kPairs>(t_row + 128, xq, rinv_q,
-                             sm.wq, sm.rot_hi[sc], sm.rot, row, lane, sm.dw,
-                             valid_row ? a.dq + tok * kHeadDim : nullptr);
-      tc_fence_before();
-      mbar_arrive(&sm.tfree);
+      {
+        const float rinv = sm.rinvq[row];  // written by cg 0 before the first exchange
+        const float2 rinv2 = make_float2(rinv, rinv);
+        float y[64];
+        {
+          uint32_t r[32], r2[32];
+          tmem_ld32(t_row + 128 + cg * 64, r);
+          tmem_ld32(t_row + 128 + cg * 64 + 32, r2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            y[i] = __uint_as_float(r[i]);
+            y[32 + i] = __uint_as_float(r2[i]);
+          }
+        }
+        if (cg == 0) {  // RoPE^-1 on the rotated pairs, all in the first half
+#pragma unroll
+          for (int p = 0; p < kPairs; ++p) {
+            const float2 rcp = rot_at(sm.rot_hi[sc], sm.rot, p, row);
+            const float a0 = y[p], b0 = y[p + kPairs];
+            y[p] = a0 * rcp.x + b0 * rcp.y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
+            y[p + kPairs] = b0 * rcp.x - a0 * rcp.y;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.tfree);  // dQ has been read from TMEM
+        float2 dot2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 xh = __fmul2_rn(bf2(xq[i]), rinv2);  // xhat
+          const int d = 64 * cg + 2 * i;
+          dot2 = __ffma2_rn(__fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]),
+                                       make_float2(sm.wq[d], sm.wq[d + 1])),
+                            xh, dot2);
+        }
+        float dot;
+        if (!(ok = exchange(&sm.xtb, sm.xt, dot2.x + dot2.y, ph, kSiteXchg, dot))) break;
+        dot *= 1.0f / kHeadDim;
+        const float2 ndot2 = make_float2(-dot, -dot);
+        uint8_t* out = reinterpret_cast<uint8_t*>(a.dq + tok * kHeadDim) + 128 * cg;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {  // dx = rinv (w dy - xhat dot), 16 dims at a time
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int i = 8 * i4 + e;
+            const float2 xh = __fmul2_rn(bf2(xq[i]), rinv2);
+            const int d = 64 * cg + 2 * i;
+            const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
+            const float2 g = __fmul2_rn(
+                rinv2, __ffma2_rn(xh, ndot2, __fmul2_rn(yv, make_float2(sm.wq[d], sm.wq[d + 1]))));
+            o[e] = pack_bf16x2(g.x, g.y);
+            const float2 cv = __fmul2_rn(yv, xh);  // dw contribution dy * xhat, in place
+            y[2 * i] = cv.x;
+            y[2 * i + 1] = cv.y;
+          }
+          if (valid_row) st32B(out + 32 * i4, o);
+        }
+        const float2 sw = warp_reduce_scatter64(y, lane);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane, sw.x);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane + 1, sw.y);
+      }
       if (++h == a.G) {
         h = 0;
         next_tile(c, a);
@@ -883,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
   // per-CTA dwq into the caller's accumulator
-  if (tid >= 128 && !*abort) atomicAdd(a.dwq + (tid - 128), sm.dw[tid - 128]);
+  if (tid >= 128 && tid < 256 && !*abort) atomicAdd(a.dwq + (tid - 128), sm.dw[tid - 128]);
 }
 
 // ======================================================= pass 2: key-major
@@ -980,7 +1094,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nq = 0, nkv = 0;
     auto wait0 = [&](uint64_t* bar, uint32_t par, int site) -> bool {
       bool w = true;
-      if (lane == 0) w = mbar_wait(bar, par, abort, a.err, site);
+      if (lane == 0) w = mbar_wait_inl(bar, par, abort, a.err, site);
       return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
     };
     Cursor c = cursor_at(a, u0);
@@ -1031,7 +1145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int nq = 0;
       auto W = [&](uint64_t* bar, uint32_t par, int site) {
-        if (ok) ok = mbar_wait(bar, par, abort, a.err, site);
+        if (ok) ok = mbar_wait_inl(bar, par, abort, a.err, site);
         return ok;
       };
       if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
@@ -1232,7 +1346,13 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(swa_bwd_q_kernel<kPairs>,
+    // The query-major pass's register split (setmaxnreg) assumes the kernel
+    // was built with the full launch budget per thread; refuse otherwise.
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, swa_bwd_q_kernel<kPairs>);
+    if (e != cudaSuccess) return map_cuda_error(e);
+    if (attr.numRegs != kRegsLaunchQ) return SWA_ERR_UNSUPPORTED;
+    e = cudaFuncSetAttribute(swa_bwd_q_kernel<kPairs>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_q));
     if (e == cudaSuccess)
@@ -1243,7 +1363,7 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
-  int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreads,
+  int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreadsQ,
                             smem_q, stream, tq, tk, tv, a);
   if (rc != SWA_OK) return rc;
   return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem_kv,
