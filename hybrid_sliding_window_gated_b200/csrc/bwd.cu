@@ -22,9 +22,13 @@
 // Every dq row and every dk/dv row is complete inside one CTA: no atomics
 // except the per-CTA sums of dwq and dwk.
 //
-// Roles (256 threads): warp 0 TMA producer (its lanes also compute rotation
-// tables), warp 1 TMEM allocator and MMA issuer, warps 4-7 the compute
-// warpgroup (one thread per tile row).  Waits are bounded as in the forward.
+// Roles: warp 0 TMA producer (its lanes also compute rotation tables), warp 1
+// TMEM allocator and MMA issuer.  The key-major pass (256 threads) has one
+// compute warpgroup, warps 4-7, one thread per tile row.  The query-major pass
+// (384 threads, registers rebalanced with setmaxnreg) has two, warps 4-7 and
+// 8-11, sharing every row: each takes half of the row's columns and they
+// exchange the row sums through shared memory.  Waits are bounded as in the
+// forward (inlined: ptxas places no calls under setmaxnreg).
 #include <cuda_fp16.h>
 
 #include "bwd_internal.h"
