@@ -23,12 +23,15 @@
 // except the per-CTA sums of dwq and dwk.
 //
 // Roles: warp 0 TMA producer (its lanes also compute rotation tables), warp 1
-// TMEM allocator and MMA issuer.  The key-major pass (256 threads) has one
-// compute warpgroup, warps 4-7, one thread per tile row.  The query-major pass
-// (384 threads, registers rebalanced with setmaxnreg) has two, warps 4-7 and
-// 8-11, sharing every row: each takes half of the row's columns and they
-// exchange the row sums through shared memory.  Waits are bounded as in the
-// forward (inlined: ptxas places no calls under setmaxnreg).
+// TMEM allocator and MMA issuer; both passes run 384 threads with registers
+// rebalanced by setmaxnreg and two compute warpgroups, warps 4-7 and 8-11,
+// thread r of each on tile row r.  In the query-major pass they share every
+// row: each takes half of the row's columns and they exchange the row sums
+// through shared memory.  In the key-major pass the (query tile, head) pairs
+// alternate between them, so that one transforms the next pair's Q while the
+// other turns the current pair's S^T and dP^T into P^T and dS^T; the dk and dv
+// rows are split by halves.  Waits are bounded as in the forward (inlined:
+// ptxas places no calls under setmaxnreg).
 #include <cuda_fp16.h>
 
 #include "bwd_internal.h"
@@ -38,14 +41,13 @@
 namespace swa {
 namespace bwd {
 
-constexpr int kThreads = 256;   // key-major pass
-constexpr int kThreadsQ = 384;  // query-major pass: control + two compute warpgroups
-// Query-major pass: launch budget 384 x 168 registers, rebalanced with
-// setmaxnreg between the control warpgroup and the two compute warpgroups.
-constexpr int kRegsLaunchQ = 168;
+// Both passes: a control warpgroup and two compute warpgroups, launch budget
+// 384 x 168 registers, rebalanced with setmaxnreg between them.
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;
 constexpr int kRegsControl = 56;
 constexpr int kRegsCompute = 224;
-static_assert(kRegsControl + 2 * kRegsCompute <= 3 * kRegsLaunchQ, "register split");
+static_assert(kRegsControl + 2 * kRegsCompute <= 3 * kRegsLaunch, "register split");
 constexpr int kHalfBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 (one TMA box)
 constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -217,112 +219,6 @@ __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane
   return make_float2(v[0], v[1]);
 }
 
-// A raw bf16 row (64 words), or zeros for a row past the end.
-__device__ __forceinline__ void load_row(const uint16_t* xrow, uint32_t (&x)[64]) {
-  if (xrow) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      ld32B(reinterpret_cast<const uint8_t*>(xrow) + 32 * i, *reinterpret_cast<uint32_t(*)[8]>(x + 8 * i));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 64; ++i) x[i] = 0u;
-  }
-}
-
-// dy for dims [64 half, 64 half + 64): the gradient w.r.t. the rotated,
-// normalised row (TMEM columns from t_lane_col), rotated back by RoPE^-1 with
-// this row's rotation factors `rc`.
-template <int kPairs>
-__device__ __forceinline__ void load_dy_half(uint32_t t_lane_col, int half,
-                                             const float2 (&rc)[kPairs > 0 ? kPairs : 1],
-                                             float (&y)[64]) {
-  uint32_t r[32], r2[32];
-  tmem_ld32(t_lane_col + half * 64, r);
-  tmem_ld32(t_lane_col + half * 64 + 32, r2);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    y[i] = __uint_as_float(r[i]);
-    y[32 + i] = __uint_as_float(r2[i]);
-  }
-  if (half == 0) {
-#pragma unroll
-    for (int p = 0; p < kPairs; ++p) {
-      const float a = y[p], b = y[p + kPairs];
-      y[p] = a * rc[p].x + b * rc[p].y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
-      y[p + kPairs] = b * rc[p].x - a * rc[p].y;
-    }
-  }
-}
-
-// Gradient of one row through RoPE and RMSNorm.  dz: the gradient w.r.t. the
-// rotated, normalised row, in TMEM columns [t_lane_col, +128) of this thread's
-// lane; x: the raw row (load_row, issued early to hide its latency).
-// Writes dx to `out` (unless nullptr) and adds dy (*) xhat into dw (shared,
-// summed over the warp first).  Works half a row at a time; the rotation
-// factors are computed once for both passes.
-template <int kPairs>
-__device__ __forceinline__ void norm_rope_grad(uint32_t t_lane_col, const uint32_t (&xr)[64],
-                                               float rinv, const float* w, const float2 (*hi)[8],
-                                               const RotTables& t, int row, int lane, float* dw,
-                                               uint16_t* out) {
-  float2 rc[kPairs > 0 ? kPairs : 1];
-#pragma unroll
-  for (int p = 0; p < kPairs; ++p) rc[p] = rot_at(hi, t, p, row);
-  const float2 rinv2 = make_float2(rinv, rinv);
-  // Pass 1: dot = mean(xhat (*) w (*) dy) and dw.
-  float2 dot2 = make_float2(0.f, 0.f);
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    float y[64];
-    load_dy_half<kPairs>(t_lane_col, half, rc, y);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float2 xh = __fmul2_rn(bf2(half ? xr[32 + i] : xr[i]), rinv2);  // xhat
-      const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
-      const int d = half * 64 + 2 * i;
-      dot2 = __ffma2_rn(__fmul2_rn(yv, make_float2(w[d], w[d + 1])), xh, dot2);
-      const float2 c = __fmul2_rn(yv, xh);  // dw contribution dy * xhat
-      y[2 * i] = c.x;
-      y[2 * i + 1] = c.y;
-    }
-    const float2 s = warp_reduce_scatter64(y, lane);
-    atomicAdd(dw + half * 64 + 2 * lane, s.x);
-    atomicAdd(dw + half * 64 + 2 * lane + 1, s.y);
-  }
-  const float dot = (dot2.x + dot2.y) * (1.0f / kHeadDim);
-  const float2 ndot2 = make_float2(-dot, -dot);
-  // Pass 2: dx = rinv (w dy - xhat dot).
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    float y[64];
-    load_dy_half<kPairs>(t_lane_col, half, rc, y);
-    uint32_t o[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float2 xh = __fmul2_rn(bf2(half ? xr[32 + i] : xr[i]), rinv2);
-      const int d = half * 64 + 2 * i;
-      const float2 g = __fmul2_rn(
-          rinv2, __ffma2_rn(xh, ndot2,
-                            __fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(w[d], w[d + 1]))));
-      o[i] = pack_bf16x2(g.x, g.y);
-    }
-    if (out) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        st32B(reinterpret_cast<uint8_t*>(out) + 128 * half + 32 * i,
-              *reinterpret_cast<const uint32_t(*)[8]>(o + 8 * i));
-    }
-  }
-}
-
-// One 256-byte row per thread, in 16-byte pieces (rows are 16-byte aligned).
-__device__ __forceinline__ void store_row(uint16_t* p, const uint32_t (&x)[64]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    st32B(reinterpret_cast<uint8_t*>(p) + 32 * i, *reinterpret_cast<const uint32_t(*)[8]>(x + 8 * i));
-}
-
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
   return make_desc_sw128(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
 }
@@ -400,7 +296,7 @@ struct alignas(1024) SmemQ {
 static_assert(sizeof(SmemQ) + 1024 <= 232448, "pass 1 shared memory");
 
 template <int kPairs>
-__global__ void __launch_bounds__(kThreadsQ, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     swa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -1013,9 +909,12 @@ struct alignas(1024) SmemKV {
   uint8_t da[2][kTileBytes];  // dA_i
   RotTables rot;
   float2 rot_hi[2][2][kMaxPairs][8];  // [key tile parity][tile j, j+1]
-  float lse2[2][kTile], dd[2][kTile];  // per query column, double-buffered
+  float lse2[2][2][kTile], dd[2][2][kTile];  // per query column: [warpgroup][its pair parity]
   float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
-  uint64_t kfull, vfull, kvempty, qfull[2], qempty[2], qready, staged, sfull, pfull, dkvfull, tfree;
+  float rinvk[kTile];   // 1/rms of each K row (cg 0 computes it; both use it)
+  float xt[2][kTile];   // per-warpgroup halves of each dk row's Jacobian dot
+  uint64_t kfull, vfull, kvempty, qfull[2], qempty[2], kvready, dkvfull, tfree, xtb;
+  uint64_t qready[2], staged[2], sfull[2], pfull[2];  // per warpgroup: pair nq is warpgroup nq & 1's
   uint64_t mmadone;  // dV/dK of the previous pair finished (their TMEM operands are free)
   uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
   uint32_t tmem_base;
@@ -1047,14 +946,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
     }
-    mbar_init(&sm.qready, 128);
-    mbar_init(&sm.staged, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.qready[i], 128);
+      mbar_init(&sm.staged[i], 128);
+      mbar_init(&sm.sfull[i], 1);
+      mbar_init(&sm.pfull[i], 128);
+    }
+    mbar_init(&sm.kvready, 256);
     mbar_init(&sm.mmadone, 1);
-    mbar_init(&sm.sfull, 1);
-    mbar_init(&sm.pfull, 128);
     mbar_init(&sm.dkvfull, 1);
-    mbar_init(&sm.tfree, 128);
-    mbar_init(&sm.tables, 128);
+    mbar_init(&sm.tfree, 256);
+    mbar_init(&sm.xtb, 256);
+    mbar_init(&sm.tables, 256);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.never, 1);
     sm.abort = 0;
@@ -1092,6 +995,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (query tiles, heads) a key tile meets: tiles j and j+1 (if it exists) x G
   auto n_iters = [&](const Cursor& c) { return (c.t + 1 < a.tiles_per_chain ? 2 : 1) * a.G; };
 
+  if (warp < 4) regs_dec<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     bool ok = true;
@@ -1157,14 +1061,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
         const int ni = n_iters(c);
         for (int i = 0; i < ni && ok; ++i, ++nq) {
-          if (!W(&sm.qready, nq & 1, kSiteQReady)) break;
+          const int cg = nq & 1, ph = (nq >> 1) & 1;  // the pair's warpgroup, its phase
+          if (i == 0) {
+            if (!W(&sm.kvready, it & 1, kSiteQReady)) break;
+            if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
+          }
+          if (!W(&sm.qready[cg], ph, kSiteQReady)) break;
           // S^T of this pair overwrites the columns dV of the previous pair
           // reads as its A operand: start it only once that MMA is done.
           if (nq > 0 && !W(&sm.mmadone, (nq - 1) & 1, kSiteMmaDone)) break;
-          if (i == 0) {
-            if (!W(&sm.vfull, it & 1, kSiteVFull)) break;
-            if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
-          }
           tc_fence_after();
           // S^T = K' Q'^T (columns 256..383), dP^T = V dA^T (384..511)
 #pragma unroll
@@ -1175,8 +1080,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tmem + 384, desc_kmajor(sm.v, kk), desc_kmajor(sm.da[nq & 1], kk), kIdescKK16,
                    kk > 0);
-          mma_commit(&sm.sfull);
-          if (!W(&sm.pfull, nq & 1, kSitePFull)) break;
+          mma_commit(&sm.sfull[cg]);
+          if (!W(&sm.pfull[cg], ph, kSitePFull)) break;
           tc_fence_after();
           // dV += P^T dA (0..127), dK += dS^T Q' (128..255)
 #pragma unroll
@@ -1201,11 +1106,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------------------------------------------- compute warpgroup
-    const int row = tid - 128;
+    // --------------------------------------------------- compute warpgroups
+    // Two warpgroups, each with thread r on key row r (TMEM lane r).  Per key
+    // tile cg 0 transforms K and cg 1 converts V; the (query tile, head) pairs
+    // alternate between them (pair nq is warpgroup nq & 1's: its Q transform,
+    // lse / D staging and P^T / dS^T), so one warpgroup transforms the next
+    // pair's Q while the other works on the current pair's scores; dk and dv
+    // are split by halves of the row.
+    regs_inc<kRegsCompute>();
+    const int cg = (warp - 4) >> 2;
+    const int row = (tid - 128) & 127;
     const int wq4 = warp & 3;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq4 * 32) << 16);
-    for (int e = row; e < kPairs * 16; e += 128) {
+    for (int e = tid - 128; e < kPairs * 16; e += 256) {
       const int p = e >> 4, bi = e & 15;
       float cv, sv;
       rope_cos_sin(static_cast<double>(bi), a.inv_freq[p], &cv, &sv);
@@ -1218,36 +1131,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor c = cursor_at(a, u0);
     for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
       const long long kpos = static_cast<long long>(c.t) * kTile + row;  // this thread's key
-      // ---- K'_j
+      // ---- K'_j (cg 0) and V_j in fp16 (cg 1), published to the MMA by kvready
+      // (kfull also publishes the tile's rotation tables, which both use)
       if (!(ok = warp_wait(&sm.kfull, it & 1, abort, a.err, kSiteKFull))) break;
-      const float rinv_k =
-          norm_rope_row<kPairs>(sm.k, row, sm.wk, sm.rot_hi[it & 1][0], sm.rot, a.eps);
-      if (!(ok = warp_wait(&sm.vfull, it & 1, abort, a.err, kSiteVFull))) break;
-      in_range &= row_to_f16(sm.v, row);
-      // (published to the MMA with the first qready below)
+      if (cg == 0) {
+        sm.rinvk[row] = norm_rope_row<kPairs>(sm.k, row, sm.wk, sm.rot_hi[it & 1][0], sm.rot, a.eps);
+      } else {
+        if (!(ok = warp_wait(&sm.vfull, it & 1, abort, a.err, kSiteVFull))) break;
+        in_range &= row_to_f16(sm.v, row);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.kvready);
       const int ni = n_iters(c);
       for (int i = 0; i < ni && ok; ++i, ++nq) {
+        if ((nq & 1) != cg) continue;  // the other warpgroup's pair
+        const int ph = (nq >> 1) & 1;   // phase of this warpgroup's barriers
         const int dt = i / a.G;  // query tile j + dt
         const int hq = c.kvh * a.G + i % a.G;
-        const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // this thread's query row
+        const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // query row `row`
         // ---- Q'_i, and lse / D of its rows for the column-wise softmax (their
         // loads go out first, so the transform hides their latency)
         const long long lrow = (static_cast<long long>(c.b) * a.Hq + hq) * a.T + qpos;
         const float lse_i = qpos < a.T ? __ldg(a.ws_lse + lrow) : 0.f;
         const float d_i = qpos < a.T ? __ldg(a.ws_d + lrow) : 0.f;
-        if (!(ok = warp_wait(&sm.qfull[nq & 1], (nq >> 1) & 1, abort, a.err, kSiteQFull))) break;
-        norm_rope_row<kPairs>(sm.q[nq & 1], row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
-        sm.lse2[nq & 1][row] = lse_i * kLog2e;
-        sm.dd[nq & 1][row] = d_i;
+        if (!(ok = warp_wait(&sm.qfull[cg], ph, abort, a.err, kSiteQFull))) break;
+        norm_rope_row<kPairs>(sm.q[cg], row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
+        float* l2 = sm.lse2[cg][ph];
+        float* dd = sm.dd[cg][ph];
+        l2[row] = lse_i * kLog2e;
+        dd[row] = d_i;
         fence_proxy_async_smem();
-        mbar_arrive(&sm.qready);
-        mbar_arrive(&sm.staged);  // lse2 / dd of this pair visible to the warpgroup
-        if (!(ok = warp_wait(&sm.staged, nq & 1, abort, a.err, kSiteStaged))) break;
+        mbar_arrive(&sm.qready[cg]);
+        mbar_arrive(&sm.staged[cg]);  // lse2 / dd of this pair visible to the warpgroup
+        if (!(ok = warp_wait(&sm.staged[cg], ph, abort, a.err, kSiteStaged))) break;
         // ---- P^T and dS^T for key row `row` against the 128 query columns
-        if (!(ok = warp_wait(&sm.sfull, nq & 1, abort, a.err, kSiteSFull))) break;
+        if (!(ok = warp_wait(&sm.sfull[cg], ph, abort, a.err, kSiteSFull))) break;
         tc_fence_after();
-        const float* l2 = sm.lse2[nq & 1];
-        const float* dd = sm.dd[nq & 1];
         // Query columns past T (the last, partial tile) and key rows past T
         // are outside; only chunk wq4 straddles the band edge.
         const int col_end = static_cast<int>(min(static_cast<long long>(kTile),
@@ -1262,8 +1181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool any = dt == 0 ? (pc >= wq4) : (pc <= wq4);
           uint32_t pk[16], dk[16];
           if (any) {
-            uint32_t s[32], dp[32];
-            tmem_ld32(t_row + 256 + pc * 32, s);
+            uint32_t sv[32], dp[32];
+            tmem_ld32(t_row + 256 + pc * 32, sv);
             tmem_ld32(t_row + 384 + pc * 32, dp);
             tmem_wait_ld();
             const bool edge = pc == wq4 || pc * 32 + 32 > col_end;
@@ -1272,12 +1191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float4 l4 = *reinterpret_cast<const float4*>(l2 + pc * 32 + 4 * e4);
               const float4 d4 = *reinterpret_cast<const float4*>(dd + pc * 32 + 4 * e4);
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int e = 2 * e4 + h;
-                const float2 nl = h == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
-                const float2 dv2 = h == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int e = 2 * e4 + h2;
+                const float2 nl = h2 == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
+                const float2 dv2 = h2 == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
                 const float2 z = __ffma2_rn(
-                    make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sc2, nl);
+                    make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2, nl);
                 float2 p = __fmul2_rn(make_float2(ex2_approx(z.x), ex2_approx(z.y)), kval2);
                 if (edge) {
                   const int col = pc * 32 + 2 * e;
@@ -1297,38 +1216,110 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = dk[e] = 0u;
           }
+          // packed over S^T / dP^T columns this thread has already read
           tmem_st16(t_row + 256 + pc * 16, pk);
           tmem_st16(t_row + 384 + pc * 16, dk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.pfull);
+        mbar_arrive(&sm.pfull[cg]);
       }
       if (!ok) break;
-      // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j
+      // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j, over this
+      // warpgroup's half of the row (the rotated dims are all in half 0)
       const long long krow = (static_cast<long long>(c.b) * a.T + kpos) * a.Hkv + c.kvh;
-      uint32_t xk[64];  // the raw k row, loaded while dK is computed
-      load_row(kpos < a.T ? a.k + krow * kHeadDim : nullptr, xk);
+      uint32_t xk[32];  // this warpgroup's half of the raw k row, loaded while dK is computed
+      if (kpos < a.T) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          ld32B(reinterpret_cast<const uint8_t*>(a.k + krow * kHeadDim) + 128 * cg + 32 * i,
+                *reinterpret_cast<uint32_t(*)[8]>(xk + 8 * i));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xk[i] = 0u;
+      }
       if (!(ok = warp_wait(&sm.dkvfull, it & 1, abort, a.err, kSiteDKVFull))) break;
       tc_fence_after();
-      norm_rope_grad<kPairs>(t_row + 128, xk, rinv_k,
-                             sm.wk, sm.rot_hi[it & 1][0], sm.rot, row, lane, sm.dw,
-                             kpos < a.T ? a.dk + krow * kHeadDim : nullptr);
       {
-        uint32_t dv[64];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t x[32];
-          tmem_ld32(t_row + ch * 32, x);
+        // cg 0 published 1/rms of the K rows with kvready of this tile
+        if (cg == 1 && !(ok = warp_wait(&sm.kvready, it & 1, abort, a.err, kSiteQReady))) break;
+        const float rinv = sm.rinvk[row];
+        const float2 rinv2 = make_float2(rinv, rinv);
+        float y[64];
+        uint32_t dvw[32];
+        {
+          uint32_t r[32], r2[32];
+          tmem_ld32(t_row + 128 + cg * 64, r);
+          tmem_ld32(t_row + 128 + cg * 64 + 32, r2);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            dv[ch * 16 + e] = pack_bf16x2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
+          for (int i = 0; i < 32; ++i) {
+            y[i] = __uint_as_float(r[i]);
+            y[32 + i] = __uint_as_float(r2[i]);
+          }
+          tmem_ld32(t_row + cg * 64, r);
+          tmem_ld32(t_row + cg * 64 + 32, r2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            dvw[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+            dvw[16 + e] = pack_bf16x2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1]));
+          }
         }
-        if (kpos < a.T) store_row(a.dv + krow * kHeadDim, dv);
+        tc_fence_before();
+        mbar_arrive(&sm.tfree);  // dK and dV have been read from TMEM
+        if (kpos < a.T) {
+          uint8_t* dvrow = reinterpret_cast<uint8_t*>(a.dv + krow * kHeadDim) + 128 * cg;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st32B(dvrow + 32 * i, *reinterpret_cast<const uint32_t(*)[8]>(dvw + 8 * i));
+        }
+        if (cg == 0) {  // RoPE^-1 on the rotated pairs, all in the first half
+#pragma unroll
+          for (int p = 0; p < kPairs; ++p) {
+            const float2 rcp = rot_at(sm.rot_hi[it & 1][0], sm.rot, p, row);
+            const float a0 = y[p], b0 = y[p + kPairs];
+            y[p] = a0 * rcp.x + b0 * rcp.y;  // R^T: (a, b) -> (a cos + b sin, b cos - a sin)
+            y[p + kPairs] = b0 * rcp.x - a0 * rcp.y;
+          }
+        }
+        float2 dot2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 xh = __fmul2_rn(bf2(xk[i]), rinv2);  // xhat
+          const int d = 64 * cg + 2 * i;
+          dot2 = __ffma2_rn(__fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]),
+                                       make_float2(sm.wk[d], sm.wk[d + 1])),
+                            xh, dot2);
+        }
+        sm.xt[cg][row] = dot2.x + dot2.y;
+        mbar_arrive(&sm.xtb);
+        if (!(ok = warp_wait(&sm.xtb, it & 1, abort, a.err, kSiteXchg))) break;
+        const float dot = (dot2.x + dot2.y + sm.xt[cg ^ 1][row]) * (1.0f / kHeadDim);
+        const float2 ndot2 = make_float2(-dot, -dot);
+        uint8_t* out = reinterpret_cast<uint8_t*>(a.dk + krow * kHeadDim) + 128 * cg;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {  // dx = rinv (w dy - xhat dot), 16 dims at a time
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int i = 8 * i4 + e;
+            const float2 xh = __fmul2_rn(bf2(xk[i]), rinv2);
+            const int d = 64 * cg + 2 * i;
+            const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
+            const float2 g = __fmul2_rn(
+                rinv2, __ffma2_rn(xh, ndot2, __fmul2_rn(yv, make_float2(sm.wk[d], sm.wk[d + 1]))));
+            o[e] = pack_bf16x2(g.x, g.y);
+            const float2 cv = __fmul2_rn(yv, xh);  // dw contribution dy * xhat, in place
+            y[2 * i] = cv.x;
+            y[2 * i + 1] = cv.y;
+          }
+          if (kpos < a.T) st32B(out + 32 * i4, o);
+        }
+        const float2 sw = warp_reduce_scatter64(y, lane);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane, sw.x);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane + 1, sw.y);
       }
-      tc_fence_before();
-      mbar_arrive(&sm.tfree);
     }
     if (!in_range) atomicCAS(a.err, 0, kDevErrRange);
   }
@@ -1339,7 +1330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (tid >= 128 && !*abort) atomicAdd(a.dwk + (tid - 128), sm.dw[tid - 128]);
+  if (tid >= 128 && tid < 256 && !*abort) atomicAdd(a.dwk + (tid - 128), sm.dw[tid - 128]);
 }
 
 template <int kPairs>
@@ -1350,12 +1341,13 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    // The query-major pass's register split (setmaxnreg) assumes the kernel
-    // was built with the full launch budget per thread; refuse otherwise.
-    cudaFuncAttributes attr;
+    // The register split (setmaxnreg) assumes each kernel was built with the
+    // full launch budget per thread; refuse otherwise.
+    cudaFuncAttributes attr, attr_kv;
     cudaError_t e = cudaFuncGetAttributes(&attr, swa_bwd_q_kernel<kPairs>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&attr_kv, swa_bwd_kv_kernel<kPairs>);
     if (e != cudaSuccess) return map_cuda_error(e);
-    if (attr.numRegs != kRegsLaunchQ) return SWA_ERR_UNSUPPORTED;
+    if (attr.numRegs != kRegsLaunch || attr_kv.numRegs != kRegsLaunch) return SWA_ERR_UNSUPPORTED;
     e = cudaFuncSetAttribute(swa_bwd_q_kernel<kPairs>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_q));
@@ -1367,7 +1359,7 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
-  int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreadsQ,
+  int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreads,
                             smem_q, stream, tq, tk, tv, a);
   if (rc != SWA_OK) return rc;
   return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem_kv,
