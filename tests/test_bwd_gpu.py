@@ -57,6 +57,16 @@ def test_backward_shapes_and_ragged_tails(B, T, Hq, Hkv):
                                        backward=True))
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv", [(40, 384, 6, 2), (50, 300, 2, 2)])
+def test_backward_odd_pair_counts_inside_a_cta(B, T, Hq, Hkv):
+    """More key tiles than CTAs, with an odd group size: the last key tile of
+    each (sequence, kv head) chain meets an odd number of (query tile, head)
+    pairs, and chains meet inside one CTA's range of tiles, so the key-major
+    pass's alternation of pairs between its warpgroups changes phase there."""
+    check_bwd(workloads.custom_prefill(B, T, Hq, Hkv, base=1e4, seed=B * 1000 + T + 11,
+                                       backward=True))
+
+
 @pytest.mark.parametrize("rot_dim", [0, 32, 48])
 def test_backward_other_rot_dims(rot_dim):
     check_bwd(workloads.custom_prefill(1, 300, 4, 2, base=1e4, seed=17, R=rot_dim, backward=True))
