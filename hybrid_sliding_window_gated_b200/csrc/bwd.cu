@@ -56,7 +56,7 @@ enum Site {
   kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
   kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
   kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged,
-  kSiteMmaDone, kSiteForced, kSiteXchg
+  kSiteMmaDone, kSiteForced, kSiteXchg, kSiteKVReady
 };
 
 // ---------------------------------------------------------------- helpers
@@ -1063,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < ni && ok; ++i, ++nq) {
           const int cg = nq & 1, ph = (nq >> 1) & 1;  // the pair's warpgroup, its phase
           if (i == 0) {
-            if (!W(&sm.kvready, it & 1, kSiteQReady)) break;
+            if (!W(&sm.kvready, it & 1, kSiteKVReady)) break;
             if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
           }
           if (!W(&sm.qready[cg], ph, kSiteQReady)) break;
@@ -1242,7 +1242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       {
         // cg 0 published 1/rms of the K rows with kvready of this tile
-        if (cg == 1 && !(ok = warp_wait(&sm.kvready, it & 1, abort, a.err, kSiteQReady))) break;
+        if (cg == 1 && !(ok = warp_wait(&sm.kvready, it & 1, abort, a.err, kSiteKVReady))) break;
         const float rinv = sm.rinvk[row];
         const float2 rinv2 = make_float2(rinv, rinv);
         float y[64];
