@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(L):
     names = declared_functions()
-    assert {"swa_fwd", "swa_bwd", "swa_decode_step", "swa_bwd_workspace_size"} <= set(names)
+    assert {"swa_fwd", "swa_bwd", "swa_decode_step", "swa_bwd_workspace_size",
+            "swa_prefill_to_ring"} <= set(names)
     out = subprocess.check_output(["nm", "-D", "--defined-only", swa.LIB_PATH], text=True)
     exported = set(re.findall(r" T (swa_\w+)", out))
     missing = [n for n in names if n not in exported]
