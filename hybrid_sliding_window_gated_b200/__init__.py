@@ -6,15 +6,18 @@ the library's sm_100a kernels.  If the compiled library is missing, importing
 the binding raises, so there is no silent CPU fallback.
 
 PyTorch serves as the owner of device memory and streams: tensors are passed
-by ``data_ptr()`` and calls are enqueued on the current CUDA stream.
+by ``data_ptr()`` and calls are enqueued on the current CUDA stream.  Before a
+pointer is passed, each tensor's dtype, element count, contiguity and device
+are checked against what the call reads or writes (``TypeError`` /
+``ValueError``); the library itself checks the sizes and alignment.
 """
 import ctypes
 import os
 
 import torch
 
-__all__ = ["fwd", "bwd", "bwd_noalloc", "bwd_workspace_size", "decode_step", "get_last_device_error",
-           "SwaError", "Params", "lib", "LIB_PATH"]
+__all__ = ["fwd", "bwd", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
+           "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswa.so")
 
@@ -84,6 +87,30 @@ def _check(rc, where):
         raise SwaError(rc, where)
 
 
+def _need(where, device, **tensors):
+    """Host-side check of the tensors a call hands to the library: each entry is
+    name=(tensor, dtype, elements the call reads or writes).  A non-empty tensor
+    must be a contiguous CUDA tensor on `device` with the dtype and at least
+    that many elements; the kernels take its pointer and the sizes in the
+    parameter block, so anything else would be misread or overrun."""
+    for name, (t, dtype, n) in tensors.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{where}: {name} must be a torch.Tensor")
+        if t.dtype != dtype:
+            raise TypeError(f"{where}: {name} is {t.dtype}, expected {dtype}")
+    used = {name: (t, n) for name, (t, _, n) in tensors.items() if n > 0}
+    for name, (t, n) in used.items():
+        if t.numel() < n:
+            raise ValueError(f"{where}: {name} has {t.numel()} elements, the call needs {n}")
+    for name, (t, n) in used.items():
+        if not t.is_contiguous():
+            raise ValueError(f"{where}: {name} must be contiguous")
+    for name, (t, n) in used.items():
+        if t.device != device or not t.is_cuda:
+            raise ValueError(f"{where}: {name} is on {t.device}, expected a CUDA tensor on "
+                             f"the device of the first input")
+
+
 def make_params(B, T, Hq, Hkv, *, head_dim=128, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
                 scale=0.0, flags=0):
     return Params(B, T, Hq, Hkv, head_dim, window, rot_dim, flags, rope_base, eps, scale)
@@ -104,6 +131,11 @@ def fwd(q, k, v, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6, 
         lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
     p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
                     rope_base=rope_base, eps=eps, scale=scale, flags=flags)
+    nq, nk = B * T * Hq * D, B * T * Hkv * D
+    bf, f32 = torch.bfloat16, torch.float32
+    opt = {} if lse is None else {"lse": (lse, f32, B * Hq * T)}
+    _need("swa_fwd", q.device, q=(q, bf, nq), k=(k, bf, nk), v=(v, bf, nk), g=(g, bf, nq),
+          wq=(wq, f32, D if nq else 0), wk=(wk, f32, D if nq else 0), out=(out, bf, nq), **opt)
     rc = lib().swa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
                        _ptr(out), _ptr(lse), _stream(stream))
     _check(rc, "swa_fwd")
@@ -113,6 +145,19 @@ def fwd(q, k, v, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6, 
 def bwd_workspace_size(B, T, Hq, Hkv, *, head_dim=128, window=128, rot_dim=42):
     p = make_params(B, T, Hq, Hkv, head_dim=head_dim, window=window, rot_dim=rot_dim)
     return int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
+
+
+def _need_bwd(where, q, k, v, g, wq, wk, lse, dO, grads, **extra):
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    nq, nk = B * T * Hq * D, B * T * Hkv * D
+    nw = D if nq else 0
+    bf, f32 = torch.bfloat16, torch.float32
+    dq, dk, dv, dg, dwq, dwk = grads
+    _need(where, q.device, q=(q, bf, nq), k=(k, bf, nk), v=(v, bf, nk), g=(g, bf, nq),
+          wq=(wq, f32, nw), wk=(wk, f32, nw), lse=(lse, f32, B * Hq * T), dO=(dO, bf, nq),
+          dq=(dq, bf, nq), dk=(dk, bf, nk), dv=(dv, bf, nk), dg=(dg, bf, nq),
+          dwq=(dwq, f32, nw), dwk=(dwk, f32, nw), **extra)
 
 
 def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
@@ -130,6 +175,8 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, e
     nbytes = int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    _need_bwd("swa_bwd", q, k, v, g, wq, wk, lse, dO, grads,
+              workspace=(workspace, torch.uint8, nbytes))
     rc = lib().swa_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
                        _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq),
                        _ptr(dwk), _ptr(workspace), workspace.numel(), _stream(stream))
@@ -149,6 +196,7 @@ def bwd_noalloc(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_bas
                  torch.zeros(D, dtype=torch.float32, device=q.device),
                  torch.zeros(D, dtype=torch.float32, device=q.device))
     dq, dk, dv, dg, dwq, dwk = grads
+    _need_bwd("swa_bwd_noalloc", q, k, v, g, wq, wk, lse, dO, grads)
     rc = lib().swa_bwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
                                _ptr(wk), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(dg), _ptr(dwq), _ptr(dwk), _stream(stream))
@@ -165,6 +213,12 @@ def decode_step(pos, q, k_new, v_new, g, wq, wk, k_cache, v_cache, *, rot_dim=42
         out = torch.empty_like(q)
     p = make_params(N, 1, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
                     eps=eps, scale=scale, flags=flags)
+    nq, nk = N * Hq * D, N * Hkv * D
+    bf, f32 = torch.bfloat16, torch.float32
+    _need("swa_decode_step", q.device, pos=(pos, torch.int64, N), q=(q, bf, nq),
+          k_new=(k_new, bf, nk), v_new=(v_new, bf, nk), g=(g, bf, nq),
+          wq=(wq, f32, D if N else 0), wk=(wk, f32, D if N else 0),
+          k_cache=(k_cache, bf, nk * W), v_cache=(v_cache, bf, nk * W), out=(out, bf, nq))
     rc = lib().swa_decode_step(ctypes.byref(p), _ptr(pos), _ptr(q), _ptr(k_new), _ptr(v_new),
                                _ptr(g), _ptr(wq), _ptr(wk), _ptr(k_cache), _ptr(v_cache), _ptr(out),
                                _stream(stream))
@@ -180,6 +234,12 @@ def prefill_to_ring(k, v, wk, k_cache, v_cache, *, Hq, rot_dim=42, rope_base=1e7
     W = k_cache.shape[2]
     p = make_params(B, T, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
                     eps=eps)
+    nk = B * T * Hkv * D if T else 0
+    nr = B * Hkv * W * D if T else 0
+    bf = torch.bfloat16
+    _need("swa_prefill_to_ring", k.device, k=(k, bf, nk), v=(v, bf, nk),
+          wk=(wk, torch.float32, D if nk else 0), k_cache=(k_cache, bf, nr),
+          v_cache=(v_cache, bf, nr))
     rc = lib().swa_prefill_to_ring(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(wk), _ptr(k_cache),
                                    _ptr(v_cache), _stream(stream))
     _check(rc, "swa_prefill_to_ring")

@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import hybrid_sliding_window_gated_b200 as swa
 from hybrid_sliding_window_gated_b200 import build as swa_build
@@ -137,3 +138,72 @@ def test_prefill_to_ring_host_checks(L):
     args = [good] * 5
     args[3] = ctypes.c_void_p((1 << 20) + 8)  # rings must be 16-byte aligned
     assert L.swa_prefill_to_ring(ctypes.byref(p), *args, nul) == swa.ERR_INVALID_ARG
+
+
+# ------------------------------------------- the Python binding's own checks
+
+def _prefill_cpu(B=1, T=64, Hq=4, Hkv=1):
+    bf = torch.bfloat16
+    return dict(q=torch.zeros(B, T, Hq, 128, dtype=bf), k=torch.zeros(B, T, Hkv, 128, dtype=bf),
+                v=torch.zeros(B, T, Hkv, 128, dtype=bf), g=torch.zeros(B, T, Hq, 128, dtype=bf),
+                wq=torch.ones(128), wk=torch.ones(128))
+
+
+def test_binding_rejects_tensors_the_kernels_would_misread():
+    """Checked on the host before the library is called: dtype, element count,
+    contiguity, then a CUDA device (the CPU tensors here fail that last one)."""
+    d = _prefill_cpu()
+    with pytest.raises(ValueError, match="CUDA"):
+        swa.fwd(**d)
+    with pytest.raises(TypeError, match="q is torch.float32"):
+        swa.fwd(**dict(d, q=d["q"].float()))
+    with pytest.raises(ValueError, match="k has 4096 elements"):
+        swa.fwd(**dict(d, k=d["k"][:, :32].contiguous()))
+    with pytest.raises(ValueError, match="contiguous"):
+        swa.fwd(**dict(d, g=d["g"].transpose(1, 2).contiguous().transpose(1, 2)))
+    with pytest.raises(ValueError, match="lse"):
+        swa.fwd(**d, lse=torch.empty(1, 4, 63))
+    lse = torch.zeros(1, 4, 64)
+    with pytest.raises(TypeError, match="dO is torch.float32"):
+        swa.bwd(*d.values(), lse, torch.zeros(1, 64, 4, 128))
+    with pytest.raises(TypeError, match="workspace"):
+        swa.bwd(*d.values(), lse, d["q"].clone(), workspace=torch.empty(10, dtype=torch.int32),
+                grads=(d["q"].clone(), d["k"].clone(), d["v"].clone(), d["g"].clone(),
+                       torch.zeros(128), torch.zeros(128)))
+
+
+def test_binding_checks_decode_and_ring_tensors():
+    bf = torch.bfloat16
+    N, Hq, Hkv = 3, 8, 2
+    x = dict(pos=torch.zeros(N, dtype=torch.int64), q=torch.zeros(N, Hq, 128, dtype=bf),
+             k_new=torch.zeros(N, Hkv, 128, dtype=bf), v_new=torch.zeros(N, Hkv, 128, dtype=bf),
+             g=torch.zeros(N, Hq, 128, dtype=bf), wq=torch.ones(128), wk=torch.ones(128),
+             k_cache=torch.zeros(N, Hkv, 128, 128, dtype=bf),
+             v_cache=torch.zeros(N, Hkv, 128, 128, dtype=bf))
+    with pytest.raises(TypeError, match="pos is torch.int32"):
+        swa.decode_step(**dict(x, pos=x["pos"].int()))
+    with pytest.raises(ValueError, match="v_cache has"):
+        swa.decode_step(**dict(x, v_cache=x["v_cache"][:2].contiguous()))
+    with pytest.raises(ValueError, match="CUDA"):
+        swa.decode_step(**x)
+    d = _prefill_cpu(B=N, T=200, Hq=Hq, Hkv=Hkv)
+    with pytest.raises(ValueError, match="k_cache has"):
+        swa.prefill_to_ring(d["k"], d["v"], d["wk"], x["k_cache"][:, :1].contiguous(),
+                            x["v_cache"], Hq=Hq)
+    with pytest.raises(TypeError, match="wk is torch.bfloat16"):
+        swa.prefill_to_ring(d["k"], d["v"], d["wk"].bfloat16(), x["k_cache"], x["v_cache"], Hq=Hq)
+
+
+def test_binding_passes_empty_problems_through():
+    """Empty problems skip the tensor checks and reach the library, which
+    returns without touching a pointer."""
+    bf = torch.bfloat16
+    e = dict(q=torch.zeros(1, 0, 4, 128, dtype=bf), k=torch.zeros(1, 0, 1, 128, dtype=bf),
+             v=torch.zeros(1, 0, 1, 128, dtype=bf), g=torch.zeros(1, 0, 4, 128, dtype=bf),
+             wq=torch.ones(128), wk=torch.ones(128))
+    swa.build.build()
+    assert swa.fwd(**e, stream=_NullStream()).shape == (1, 0, 4, 128)
+
+
+class _NullStream:
+    cuda_stream = 0

@@ -37,7 +37,8 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_take_the_max_and_only_rank0_reports():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    # spawn, not fork: this process may already run threads (OpenMP, torch)
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
