@@ -87,3 +87,27 @@ def test_committed_traffic_is_dropped_when_the_kernel_changes(tmp_path, monkeypa
     assert bench.committed_traffic("k.txt", ["k.cu"]) is None
     assert bench.committed_traffic("missing.txt", ["k.cu"]) is None
     assert os.path.exists(tmp_path / "profiles" / "k.txt")
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` runs the oracle on the host cores (no GPU)
+    and prints one JSON line with the same metric and workload as the GPU
+    arm, plus its cpu_baseline and e2e blocks."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                          "--warmup", "3"], cwd=root, env=env, capture_output=True, text=True,
+                         timeout=600, check=True).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 1 and rec["steps"] == 1
+    assert rec["metric"] == "gated-SWA forward tokens/s (layer-shape prefill)"
+    assert rec["unit"] == "tokens/s" and rec["higher_is_better"] is True
+    assert rec["config"]["workload"] == workloads.LAYER.name
+    assert rec["value"] > 0 and rec["cpu_baseline"]["value"] == rec["value"]
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
+    assert rec["e2e"] == {"value": rec["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
