@@ -120,6 +120,9 @@ int check_params(const swa_params_t* p, bool decode) {
     return SWA_ERR_UNSUPPORTED;
   if (p->B > (1ll << 30) || (!decode && p->T > (1ll << 30)) || p->Hq > 4096)
     return SWA_ERR_UNSUPPORTED;
+  // B x T tokens at most 2^40, so that every element count and byte offset
+  // below (B T Hq 128 x 2 bytes < 2^60) and every tile count fits in int64.
+  if (!decode && p->B * p->T > (1ll << 40)) return SWA_ERR_UNSUPPORTED;
   return SWA_OK;
 }
 

@@ -38,7 +38,9 @@
  *     attributes).
  *   - The tensor-core path needs head_dim == 128, window == 128, Hq a
  *     multiple of Hkv and rot_dim even in {0, 32, 42, 48}.  Other shapes return
- *     SWA_ERR_UNSUPPORTED; nothing silently falls back to a slow path.
+ *     SWA_ERR_UNSUPPORTED; nothing silently falls back to a slow path.  Size
+ *     limits (also SWA_ERR_UNSUPPORTED beyond them): B and T at most 2^30 each,
+ *     B x T at most 2^40 tokens, Hq at most 4096.
  *   - Errors: SWA_OK on success; SWA_ERR_INVALID_ARG (null or misaligned
  *     pointer, negative size, Hq % Hkv != 0, ...); SWA_ERR_UNSUPPORTED;
  *     SWA_ERR_CUDA (a CUDA runtime call failed, e.g. the launch); the kernels

@@ -60,6 +60,7 @@ def _params(**kw):
     (dict(head_dim=64), swa.ERR_UNSUPPORTED),         # tensor-core path is built for 128
     (dict(window=64), swa.ERR_UNSUPPORTED),
     (dict(rot_dim=40), swa.ERR_UNSUPPORTED),
+    (dict(B=1 << 20, T=1 << 21), swa.ERR_UNSUPPORTED),  # 2^41 tokens: size products overflow
 ])
 def test_bad_shapes_rejected_before_any_launch(L, kw, code):
     p = _params(**kw)
