@@ -137,3 +137,11 @@ def test_a_short_rank_makes_every_rank_raise():
         out = mgr.dict()
         mp.spawn(_short_rank_main, args=(2, _free_port(), out), nprocs=2, join=True)
         assert dict(out) == {0: "raised", 1: "raised"}
+
+
+def test_the_product_path_calls_the_kernel_wrappers():
+    import hybrid_sliding_window_gated_b200 as swa
+    from hybrid_sliding_window_gated_b200 import seqpar
+    assert seqpar._local_fwd is swa.fwd and seqpar._local_bwd is swa.bwd
+    src = open(seqpar.__file__).read()
+    assert "oracle" not in src
