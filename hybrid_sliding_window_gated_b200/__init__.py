@@ -16,7 +16,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "bwd", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
+__all__ = ["fwd", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswa.so")
@@ -56,6 +56,9 @@ def lib():
         L.swa_fwd.restype = ctypes.c_int
         L.swa_bwd.argtypes = [P] + [_vp] * 15 + [ctypes.c_size_t, _vp]
         L.swa_bwd.restype = ctypes.c_int
+        L.swa_bwd_edges.argtypes = [P] + [_vp] * 14 + [ctypes.c_int64, _vp, ctypes.c_int64, _vp,
+                                                       _vp, ctypes.c_size_t, _vp]
+        L.swa_bwd_edges.restype = ctypes.c_int
         L.swa_bwd_noalloc.argtypes = [P] + [_vp] * 15
         L.swa_bwd_noalloc.restype = ctypes.c_int
         L.swa_bwd_workspace_size.argtypes = [P]
@@ -182,6 +185,40 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4, e
                        _ptr(dwk), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "swa_bwd")
     return grads
+
+
+def bwd_edges(q, k, v, g, wq, wk, lse, dO, n_lo, n_hi, *, window=128, rot_dim=42,
+              rope_base=1e4, eps=1e-6, scale=0.0, workspace=None, grads=None, stream=None):
+    """:func:`bwd`, plus fp32 copies of dk and dv for the first ``n_lo`` and the
+    last ``n_hi`` tokens of every sequence (swa_bwd_edges).  Returns
+    ``(grads, dkv_lo, dkv_hi)`` with dkv_* of shape [B, n, Hkv, 2, 128]
+    (dk, dv) or None when n is 0."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g),
+                 torch.zeros(D, dtype=torch.float32, device=q.device),
+                 torch.zeros(D, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dg, dwq, dwk = grads
+    nbytes = int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    lo = torch.empty((B, n_lo, Hkv, 2, D), dtype=torch.float32, device=q.device) if n_lo else None
+    hi = torch.empty((B, n_hi, Hkv, 2, D), dtype=torch.float32, device=q.device) if n_hi else None
+    extra = {"workspace": (workspace, torch.uint8, nbytes)}
+    if lo is not None:
+        extra["dkv_lo"] = (lo, torch.float32, lo.numel())
+    if hi is not None:
+        extra["dkv_hi"] = (hi, torch.float32, hi.numel())
+    _need_bwd("swa_bwd_edges", q, k, v, g, wq, wk, lse, dO, grads, **extra)
+    rc = lib().swa_bwd_edges(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
+                             _ptr(wk), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                             _ptr(dwq), _ptr(dwk), n_lo, _ptr(lo), n_hi, _ptr(hi),
+                             _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "swa_bwd_edges")
+    return grads, lo, hi
 
 
 def bwd_noalloc(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4,

@@ -219,12 +219,24 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
 
 extern "C" {
 
-int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
-            const swa_bf16_t* g, const float* wq, const float* wk, const float* lse,
-            const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk, swa_bf16_t* dv, swa_bf16_t* dg,
-            float* dwq, float* dwk, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace swa {
+
+// swa_bwd and swa_bwd_edges: the edge rows' fp32 copies are optional
+// (n_lo = n_hi = 0 and null buffers for swa_bwd).
+static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                    const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                    const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                    swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, int64_t n_lo,
+                    float* edge_lo, int64_t n_hi, float* edge_hi, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   int rc = check_params(p, false);
   if (rc != SWA_OK) return rc;
+  if (n_lo < 0 || n_hi < 0 || n_lo > p->T || n_hi > p->T || (n_lo > 0 && edge_lo == nullptr) ||
+      (n_hi > 0 && edge_hi == nullptr) || (reinterpret_cast<uintptr_t>(edge_lo) & 7u) ||
+      (reinterpret_cast<uintptr_t>(edge_hi) & 7u))
+    return SWA_ERR_INVALID_ARG;
   if (p->B == 0 || p->T == 0) return SWA_OK;
   if (!q || !k || !v || !g || !wq || !wk || !lse || !dO || !dq || !dk || !dv || !dg || !dwq ||
       !dwk || !workspace)
@@ -239,7 +251,8 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
     return SWA_ERR_INVALID_ARG;
   const size_t da_bytes = bwd_ws_da_bytes(p->B, p->T, p->Hq);
   const size_t d_bytes = bwd_ws_d_bytes(p->B, p->T, p->Hq);
-  if (workspace_bytes < da_bytes + 2 * d_bytes) return SWA_ERR_INVALID_ARG;
+  const size_t ee_bytes = bwd_ws_ee_bytes(p->B, p->T, p->Hq);
+  if (workspace_bytes < bwd_ws_total_bytes(p->B, p->T, p->Hq, p->Hkv)) return SWA_ERR_INVALID_ARG;
 
   BwdArgs a{};
   a.B = static_cast<int>(p->B);
@@ -268,7 +281,14 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
   a.dwk = dwk;
   a.ws_da = static_cast<uint16_t*>(workspace);
   a.ws_d = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + da_bytes);
-  a.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + da_bytes + d_bytes);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.ws_lse = reinterpret_cast<float*>(ws + da_bytes + d_bytes);
+  a.ws_ee = reinterpret_cast<int*>(ws + da_bytes + 2 * d_bytes);
+  a.ws_ek = reinterpret_cast<int*>(ws + da_bytes + 2 * d_bytes + ee_bytes);
+  a.n_lo = static_cast<int>(n_lo);
+  a.n_hi = static_cast<int>(n_hi);
+  a.edge_lo = n_lo > 0 ? edge_lo : nullptr;
+  a.edge_hi = n_hi > 0 ? edge_hi : nullptr;
   rc = device_error_word(&a.err);
   if (rc != SWA_OK) return rc;
   fill_inv_freq(p, a.inv_freq);
@@ -285,6 +305,28 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
   return launch_bwd(p, tq, tk, tv, tda, a, static_cast<cudaStream_t>(stream));
 }
 
+}  // namespace swa
+
+extern "C" {
+
+int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
+            const swa_bf16_t* g, const float* wq, const float* wk, const float* lse,
+            const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk, swa_bf16_t* dv, swa_bf16_t* dg,
+            float* dwq, float* dwk, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, 0, nullptr, 0, nullptr,
+                  workspace, workspace_bytes, stream);
+}
+
+int swa_bwd_edges(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                  const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                  const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                  swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, int64_t n_lo,
+                  float* dkv_lo, int64_t n_hi, float* dkv_hi, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, n_lo, dkv_lo, n_hi,
+                  dkv_hi, workspace, workspace_bytes, stream);
+}
+
 int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
                     const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
                     const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
@@ -292,8 +334,7 @@ int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
   int rc = check_params(p, false);
   if (rc != SWA_OK) return rc;
   if (p->B == 0 || p->T == 0) return SWA_OK;
-  const size_t need =
-      bwd_ws_da_bytes(p->B, p->T, p->Hq) + 2 * bwd_ws_d_bytes(p->B, p->T, p->Hq);
+  const size_t need = bwd_ws_total_bytes(p->B, p->T, p->Hq, p->Hkv);
   if (need > kStaticScratchBytes) return SWA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if ((rc = static_scratch(&scratch)) != SWA_OK) return rc;
@@ -303,7 +344,7 @@ int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
 
 size_t swa_bwd_workspace_size(const swa_params_t* p) {
   if (check_params(p, false) != SWA_OK) return 0;
-  return bwd_ws_da_bytes(p->B, p->T, p->Hq) + 2 * bwd_ws_d_bytes(p->B, p->T, p->Hq);
+  return bwd_ws_total_bytes(p->B, p->T, p->Hq, p->Hkv);
 }
 
 int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf16_t* v,

@@ -56,7 +56,7 @@ enum Site {
   kSiteKFull = 0x60, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteQFull, kSiteQEmpty, kSiteQReady,
   kSiteKReady, kSiteSFull, kSitePFull, kSiteAFull, kSiteDAFull, kSiteDPFull, kSiteDSFull,
   kSiteDQ0, kSiteDQFull, kSiteTFree, kSiteTables, kSiteDKVFull, kSiteKVEmpty, kSiteStaged,
-  kSiteMmaDone, kSiteForced, kSiteXchg, kSiteKVReady
+  kSiteMmaDone, kSiteForced, kSiteXchg, kSiteKVReady, kSiteVReady
 };
 
 // ---------------------------------------------------------------- helpers
@@ -87,14 +87,16 @@ __device__ __forceinline__ void st32B(void* p, const uint32_t (&r)[8]) {
                : "memory");
 }
 
-// Largest magnitude the fp16 staging of V and dA carries (the fp16 maximum).
-constexpr float kF16Max = 65504.0f;
+// bf16 magnitude bits of the largest value the fp16 staging of V carries:
+// 0x477F is 65280, and the next bf16 value, 65536, is past the fp16 maximum.
+constexpr uint32_t kF16MaxBits = 0x477Fu;
 
 // Row `row` of a [128 x 128] bf16 tile (two 128-byte-row halves) converted to
 // fp16 in place: every backward contraction runs fp16 x fp16, three more
-// mantissa bits than bf16.  Returns false if a value is beyond the fp16 range.
-__device__ __forceinline__ bool row_to_f16(uint8_t* tile, int row) {
-  bool ok = true;
+// mantissa bits than bf16.  Returns the row's largest magnitude as bf16 bits
+// (NaN compares above every finite value).
+__device__ __forceinline__ uint32_t row_to_f16(uint8_t* tile, int row) {
+  uint32_t m = 0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint4* p = reinterpret_cast<uint4*>(tile + h * kHalfBytes + row * 128);
@@ -105,15 +107,46 @@ __device__ __forceinline__ bool row_to_f16(uint8_t* tile, int row) {
       uint32_t o[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
+        m = __vmaxu2(m, w[e] & 0x7FFF7FFFu);
         const float2 f = bf2(w[e]);
-        ok &= fabsf(f.x) <= kF16Max && fabsf(f.y) <= kF16Max;
         o[e] = pack_f16x2(f.x, f.y);
       }
       p[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  return ok;
+  return max(m & 0xFFFFu, m >> 16);
 }
+
+// Scale exponents of the fp16 staging.  Every exponent lies in
+// [-kExpLimit, kExpLimit], so a sum of two is still a normal fp32 power of two.
+constexpr int kExpLimit = 62;
+__device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-126, 127]
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
+// Exponent e of a row of dA: 2^e max|dO| lies in [1, 2), so dA 2^e (|dA| <=
+// |dO|) keeps fp16's full precision whatever the gradient's scale.  `m` is
+// max|dO| as bf16 magnitude bits; an all-zero row takes the largest exponent,
+// which leaves every minimum over rows to the rows that carry a gradient.
+__device__ __forceinline__ int row_exponent(uint32_t m) {
+  const int E = static_cast<int>(m >> 7);  // biased bf16 exponent
+  if (E == 0) return kExpLimit;
+  return max(-kExpLimit, min(kExpLimit, 127 - E));
+}
+// Exponent k of dS for a query tile whose keys' values satisfy |v| <= vmax.
+// With |dA 2^e| <= 2: |dP| <= 2 D vmax and |D_i| <= 2 D vmax (A_i is a convex
+// combination of v rows), so |dS 2^(e+k)| <= scale 4 D vmax 2^k <= 2^15:
+// inside fp16's range by construction, and values of typical size land near
+// 1 rather than among fp16's subnormals when v is small.
+__device__ __forceinline__ int ds_exponent(float scale, uint32_t vmax_bits) {
+  const float bound = scale * (4.0f * kHeadDim) * __uint_as_float(vmax_bits << 16);
+  const uint32_t Eb = (__float_as_uint(bound) >> 23) & 0xFFu;
+  if (!(bound > 0.0f) || Eb == 0xFFu) return 0;  // zero, NaN or inf
+  if (Eb == 0) return kExpLimit;
+  return max(-kExpLimit, min(kExpLimit, 141 - static_cast<int>(Eb)));  // bound < 2^(Eb-126)
+}
+// Largest bf16 exponent field of dO the staging takes (|dO| < 2^63); beyond
+// it, short of inf or NaN, the call reports kDevErrRange.
+constexpr int kMaxDoExpField = 127 + kExpLimit;
 __device__ __forceinline__ float2 cmul(float2 x, float2 y) {
   return make_float2(x.x * y.x - x.y * y.y, x.x * y.y + x.y * y.x);
 }
@@ -286,9 +319,13 @@ struct alignas(1024) SmemQ {
   uint64_t qfull[2], qempty[2];
   uint64_t qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
   uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
-  // Row-sum exchanges between the two compute warpgroups (l, D, the dq dot).
+  // Row-sum exchanges between the two compute warpgroups (l with the dA row
+  // exponent, D, the dq dot).
   uint64_t xlb, xdb, xtb;
   float xl[2][kTile], xd[2][kTile], xt[2][kTile];
+  int xe[2][kTile];     // each half row's dA exponent (exchanged with l)
+  int xew[2][2][4];     // [head parity][warpgroup][warp]: minimum of those exponents
+  uint32_t vmax[2][4];  // per V slot and converting warp: largest |v| (bf16 bits)
   float rinvq[kTile];  // 1/rms of each Q row (cg 0 computes it; both use it)
   uint32_t tmem_base;
   int abort;
@@ -566,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t kpar = 0, vpar = 0;
     bool in_range = true;  // v and dO within the fp16 staging range
     int ndq0 = 0;
+    int kt = 0;  // dS exponent of the current query tile
     // Publish this warpgroup's partial of a row sum and add the partner's.
     auto exchange = [&](uint64_t* bar, float (*buf)[kTile], float v, uint32_t par, int site,
                         float& total) -> bool {
@@ -601,10 +639,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             ok = warp_wait(&sm.vfull[s], (vpar >> s) & 1u, abort, a.err, kSiteVFull);
             if (!ok) break;
-            in_range &= row_to_f16(sm.v[s], row);
+            const uint32_t m = row_to_f16(sm.v[s], row);
+            in_range &= m <= kF16MaxBits;
+            const uint32_t wm = __reduce_max_sync(0xffffffffu, m);
+            if (lane == 0) sm.vmax[s][wq4] = wm;
             fence_proxy_async_smem();
             mbar_arrive(&sm.vready[s]);
-            vpar ^= 1u << s;
           }
         }
         if (!ok) break;
@@ -677,8 +717,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // The row's dA exponent e: each warpgroup takes it from its 64 values of
+      // dO and the two are exchanged with l (the row takes the smaller).  Each
+      // warp's minimum goes to shared memory too, for the tile's minimum.
       float lsum;
-      if (!(ok = exchange(&sm.xlb, sm.xl, lsum2.x + lsum2.y, ph, kSiteXchg, lsum))) break;
+      int ei;
+      {
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m2 = __vmaxu2(m2, dc[i] & 0x7FFF7FFFu);
+        const uint32_t mh = max(m2 & 0xFFFFu, m2 >> 16);
+        const int ef = static_cast<int>(mh >> 7);
+        in_range &= !(ef > kMaxDoExpField && ef < 0xFF);
+        const int eh = row_exponent(mh);
+        const int ew = __reduce_min_sync(0xffffffffu, eh);
+        if (lane == 0) sm.xew[ph][cg][wq4] = ew;
+        sm.xl[cg][row] = lsum2.x + lsum2.y;
+        sm.xe[cg][row] = eh;
+        mbar_arrive(&sm.xlb);
+        if (!(ok = warp_wait(&sm.xlb, ph, abort, a.err, kSiteXchg))) break;
+        lsum = lsum2.x + lsum2.y + sm.xl[cg ^ 1][row];
+        ei = min(eh, sm.xe[cg ^ 1][row]);
+        if (cg == 0 && row == 0) {  // the key-major pass's common scale starts here
+          int mn = kExpLimit;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) mn = min(mn, sm.xew[ph][w >> 2][w & 3]);
+          a.ws_ee[(static_cast<long long>(c.b) * a.Hq + hq) * a.tiles_per_chain + c.t] = mn;
+        }
+      }
       {
         const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
                                      0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -705,7 +771,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // are renormalised to sum to exactly 1 under this pass's scores, and the
       // corrected normaliser goes to the key-major pass.
       const float inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
-      if (cg == 0 && valid_row) a.ws_lse[lrow] = a.lse[lrow] + __logf(lsum);
+      // in log2 units, with the row's exponent added (the key-major pass
+      // subtracts its common exponent and so scales P^T column by column)
+      if (cg == 0 && valid_row)
+        a.ws_lse[lrow] = (a.lse[lrow] + __logf(lsum)) * kLog2e + static_cast<float>(ei);
 
       // ---- A: dg, dA (smem and workspace) and D over this warpgroup's 64
       // columns (TMEM chunks 2 cg, 2 cg + 1)
@@ -713,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float2 dsum2 = make_float2(0.f, 0.f);
       const float2 il2 = make_float2(inv_l, inv_l);
-      float dmax = 0.f;  // largest |dO| of the row: fp16 staging range
+      const float2 si2 = make_float2(pow2f(ei), pow2f(ei));  // dA is staged as dA 2^e
       {
         uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim) + 128 * cg;
         uint8_t* darow = reinterpret_cast<uint8_t*>(a.ws_da + tok * kHeadDim) + 128 * cg;
@@ -731,12 +800,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 gg = bf2(gw), dd = bf2(dw);
             const float2 av = __fmul2_rn(
                 make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), il2);  // A / l
-            const float2 sg = make_float2(sigmoid_fast(gg.x), sigmoid_fast(gg.y));  // one MUFU op each
-            const float2 ds = __ffma2_rn(make_float2(-sg.x, -sg.y), sg, sg);      // s (1 - s)
+            float2 ds;                            // sigma (1 - sigma), without cancellation
+            const float2 sg = sigmoid2(gg, &ds);  // one MUFU op per element
             const float2 dgv = __fmul2_rn(__fmul2_rn(dd, av), ds);
             dgo[e] = pack_bf16x2(dgv.x, dgv.y);
-            dmax = fmaxf(dmax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
-            const float2 dav = __fmul2_rn(dd, sg);
+            const float2 dav = __fmul2_rn(__fmul2_rn(dd, sg), si2);
             dao[e] = pack_f16x2(dav.x, dav.y);
             dsum2 = __ffma2_rn(f16x2(dao[e]), av, dsum2);  // D uses the rounded dA the MMAs see
           }
@@ -763,7 +831,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&sm.dafull);
       }
-      in_range &= !(dmax > kF16Max);
       float dsum;
       if (!(ok = exchange(&sm.xdb, sm.xd, dsum2.x + dsum2.y, ph, kSiteXchg, dsum))) break;
       if (cg == 0 && valid_row) a.ws_d[lrow] = dsum;
@@ -780,9 +847,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) xq[i] = 0u;
       }
+      // dS exponent of this query tile, from the largest |v| of its key
+      // tiles: both warpgroups read the V conversion's maxima once per tile.
+      if (h == 0) {
+        for (int j = (c.t > 0 && c.u == 0) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+          const int s = j & 1;
+          ok = warp_wait(&sm.vready[s], (vpar >> s) & 1u, abort, a.err, kSiteVReady);
+          vpar ^= 1u << s;
+        }
+        if (!ok) break;
+        uint32_t vm = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          vm = max(vm, sm.vmax[sc][w]);
+          if (hp) vm = max(vm, sm.vmax[sc ^ 1][w]);
+        }
+        kt = ds_exponent(a.scale, vm);
+        if (cg == 0 && row == 0)
+          a.ws_ek[(static_cast<long long>(c.b) * a.Hkv + c.kvh) * a.tiles_per_chain + c.t] = kt;
+      }
       if (!(ok = warp_wait(&sm.dpfull, ph, abort, a.err, kSiteDPFull))) break;
       tc_fence_after();
-      const float2 sl2 = make_float2(a.scale * inv_l, a.scale * inv_l), nd2 = make_float2(-dsum, -dsum);
+      // dS 2^(e+k) = scale 2^k P / l (dP 2^e - D 2^e)
+      const float dsc = a.scale * inv_l * pow2f(kt);
+      const float2 sl2 = make_float2(dsc, dsc), nd2 = make_float2(-dsum, -dsum);
       for (int blk = hp ? 0 : 1; blk < 2 && ok; ++blk) {
         if (blk == 1 && hp) {  // the MMA has read dS of key tile t-1 from the slot
           if (!(ok = warp_wait(&sm.dq0, ndq0 & 1, abort, a.err, kSiteDQ0))) break;
@@ -829,10 +917,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(t_row + 128 + cg * 64, r);
           tmem_ld32(t_row + 128 + cg * 64 + 32, r2);
           tmem_wait_ld();
+          const float2 un2 = make_float2(pow2f(-(ei + kt)), pow2f(-(ei + kt)));  // undo 2^(e+k)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            y[i] = __uint_as_float(r[i]);
-            y[32 + i] = __uint_as_float(r2[i]);
+          for (int i = 0; i < 16; ++i) {
+            const float2 y0 = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]),
+                                                     __uint_as_float(r[2 * i + 1])), un2);
+            const float2 y1 = __fmul2_rn(make_float2(__uint_as_float(r2[2 * i]),
+                                                     __uint_as_float(r2[2 * i + 1])), un2);
+            y[2 * i] = y0.x;
+            y[2 * i + 1] = y0.y;
+            y[32 + 2 * i] = y1.x;
+            y[32 + 2 * i + 1] = y1.y;
           }
         }
         if (cg == 0) {  // RoPE^-1 on the rotated pairs, all in the first half
@@ -1131,6 +1226,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor c = cursor_at(a, u0);
     for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
       const long long kpos = static_cast<long long>(c.t) * kTile + row;  // this thread's key
+      // Common scale of this key tile's dV and dK accumulators: e_c, the
+      // smallest dA exponent among the (query tile, head) pairs it meets, and
+      // k_c, the smaller dS exponent of the two query tiles (their key tiles
+      // j-1 .. j+1 bound every D_i the pairs bring).  Column i of P^T and dS^T
+      // is scaled by 2^(e_c - e_i) <= 1 through its staged lse, so the
+      // accumulators hold dV 2^e_c and dK 2^(e_c + k_c).
+      int ec = kExpLimit, kc;
+      {
+        const bool next = c.t + 1 < a.tiles_per_chain;
+        const long long chain = static_cast<long long>(c.b) * a.Hkv + c.kvh;
+        kc = __ldg(a.ws_ek + chain * a.tiles_per_chain + c.t);
+        if (next) kc = min(kc, __ldg(a.ws_ek + chain * a.tiles_per_chain + c.t + 1));
+        for (int h2 = 0; h2 < a.G; ++h2) {
+          const int* e = a.ws_ee +
+                         (static_cast<long long>(c.b) * a.Hq + c.kvh * a.G + h2) * a.tiles_per_chain +
+                         c.t;
+          ec = min(ec, __ldg(e));
+          if (next) ec = min(ec, __ldg(e + 1));
+        }
+      }
       // ---- K'_j (cg 0) and V_j in fp16 (cg 1), published to the MMA by kvready
       // (kfull also publishes the tile's rotation tables, which both use)
       if (!(ok = warp_wait(&sm.kfull, it & 1, abort, a.err, kSiteKFull))) break;
@@ -1138,7 +1253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.rinvk[row] = norm_rope_row<kPairs>(sm.k, row, sm.wk, sm.rot_hi[it & 1][0], sm.rot, a.eps);
       } else {
         if (!(ok = warp_wait(&sm.vfull, it & 1, abort, a.err, kSiteVFull))) break;
-        in_range &= row_to_f16(sm.v, row);
+        in_range &= row_to_f16(sm.v, row) <= kF16MaxBits;
       }
       fence_proxy_async_smem();
       mbar_arrive(&sm.kvready);
@@ -1158,8 +1273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         norm_rope_row<kPairs>(sm.q[cg], row, sm.wq, sm.rot_hi[it & 1][dt], sm.rot, a.eps);
         float* l2 = sm.lse2[cg][ph];
         float* dd = sm.dd[cg][ph];
-        l2[row] = lse_i * kLog2e;
-        dd[row] = d_i;
+        l2[row] = lse_i - static_cast<float>(ec);  // log2 lse_i + e_i - e_c
+        dd[row] = d_i;                           // D_i 2^e_i
         fence_proxy_async_smem();
         mbar_arrive(&sm.qready[cg]);
         mbar_arrive(&sm.staged[cg]);  // lse2 / dd of this pair visible to the warpgroup
@@ -1173,7 +1288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  a.T - static_cast<long long>(c.t + dt) * kTile));
         const float2 kval2 = kpos < a.T ? make_float2(1.f, 1.f) : make_float2(0.f, 0.f);
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-        const float2 scale2 = make_float2(a.scale, a.scale);
+        const float dss = a.scale * pow2f(kc);  // dS^T 2^(e_c + k_c)
+        const float2 scale2 = make_float2(dss, dss);
 #pragma unroll 1
         for (int pc = 0; pc < 4; ++pc) {
           // query tile j keeps columns >= row, tile j+1 columns < row
@@ -1245,6 +1361,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (cg == 1 && !(ok = warp_wait(&sm.kvready, it & 1, abort, a.err, kSiteKVReady))) break;
         const float rinv = sm.rinvk[row];
         const float2 rinv2 = make_float2(rinv, rinv);
+        // dK 2^(e_c + k_c) and dV 2^e_c are unscaled in the epilogue: dk is
+        // linear in dK, so its factor goes into 1/rms (and the dwk sums)
+        const float unk = pow2f(-(ec + kc)), unv = pow2f(-ec);
+        const float2 rinvu2 = make_float2(rinv * unk, rinv * unk);
+        const float2 unv2 = make_float2(unv, unv);
+        // Edge rows (the first n_lo and the last n_hi keys of each sequence)
+        // also go out in fp32, [B, n, Hkv, {dk, dv}, D]: a caller that sums
+        // partial gradients of the same keys from two calls (sequence
+        // sharding) then rounds the sum once.
+        float* edge = nullptr;
+        if (kpos < a.n_lo)
+          edge = a.edge_lo +
+                 ((static_cast<long long>(c.b) * a.n_lo + kpos) * a.Hkv + c.kvh) * 2 * kHeadDim;
+        else if (kpos < a.T && kpos >= a.T - a.n_hi)
+          edge = a.edge_hi + ((static_cast<long long>(c.b) * a.n_hi + (kpos - (a.T - a.n_hi))) *
+                                  a.Hkv + c.kvh) * 2 * kHeadDim;
         float y[64];
         uint32_t dvw[32];
         {
@@ -1262,8 +1394,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            dvw[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-            dvw[16 + e] = pack_bf16x2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1]));
+            const float2 v0 = __fmul2_rn(
+                make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), unv2);
+            const float2 v1 = __fmul2_rn(
+                make_float2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1])), unv2);
+            dvw[e] = pack_bf16x2(v0.x, v0.y);
+            dvw[16 + e] = pack_bf16x2(v1.x, v1.y);
+            if (edge != nullptr) {
+              *reinterpret_cast<float2*>(edge + kHeadDim + 64 * cg + 2 * e) = v0;
+              *reinterpret_cast<float2*>(edge + kHeadDim + 64 * cg + 32 + 2 * e) = v1;
+            }
           }
         }
         tc_fence_before();
@@ -1308,8 +1448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int d = 64 * cg + 2 * i;
             const float2 yv = make_float2(y[2 * i], y[2 * i + 1]);
             const float2 g = __fmul2_rn(
-                rinv2, __ffma2_rn(xh, ndot2, __fmul2_rn(yv, make_float2(sm.wk[d], sm.wk[d + 1]))));
+                rinvu2, __ffma2_rn(xh, ndot2, __fmul2_rn(yv, make_float2(sm.wk[d], sm.wk[d + 1]))));
             o[e] = pack_bf16x2(g.x, g.y);
+            if (edge != nullptr) *reinterpret_cast<float2*>(edge + d) = g;
             const float2 cv = __fmul2_rn(yv, xh);  // dw contribution dy * xhat, in place
             y[2 * i] = cv.x;
             y[2 * i + 1] = cv.y;
@@ -1317,8 +1458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kpos < a.T) st32B(out + 32 * i4, o);
         }
         const float2 sw = warp_reduce_scatter64(y, lane);
-        atomicAdd(sm.dw + 64 * cg + 2 * lane, sw.x);
-        atomicAdd(sm.dw + 64 * cg + 2 * lane + 1, sw.y);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane, sw.x * unk);
+        atomicAdd(sm.dw + 64 * cg + 2 * lane + 1, sw.y * unk);
       }
     }
     if (!in_range) atomicCAS(a.err, 0, kDevErrRange);

@@ -25,25 +25,48 @@ struct BwdArgs {
   uint16_t* dg;
   float* dwq;
   float* dwk;
-  uint16_t* ws_da;  // workspace: dA = dO * sigmoid(g), [B, T, Hq, D] fp16
-  float* ws_d;      // workspace: D_i = dA_i . A_i, [B, Hq, T] fp32
-  float* ws_lse;    // workspace: lse renormalised to the backward's scores, [B, Hq, T] fp32
+  // Workspace.  Row i of dA is staged as dA_i 2^e_i, with e_i chosen from
+  // max|dO_i| so the row's largest value lies in [1, 2) (fp16 keeps its full
+  // precision there whatever the scale of the upstream gradient).
+  uint16_t* ws_da;  // dA_i 2^e_i, [B, T, Hq, D] fp16
+  float* ws_d;      // D_i 2^e_i = (dA_i 2^e_i) . A_i, [B, Hq, T] fp32
+  float* ws_lse;    // log2 of the renormalised softmax normaliser, plus e_i, [B, Hq, T] fp32
+  int* ws_ee;       // min of e_i over each query tile's rows, [B, Hq, tiles]
+  int* ws_ek;       // dS scale exponent of each query tile (from max|v|), [B, Hkv, tiles]
+  // Optional fp32 copies of dk and dv for the first n_lo and the last n_hi
+  // key rows of every sequence, [B, n, Hkv, 2, D] (dk, then dv); 0 and null
+  // when unused.
+  int n_lo, n_hi;
+  float* edge_lo;
+  float* edge_hi;
   int* err;
   double inv_freq[kMaxPairs];
 };
 
 // Device error code: a norm weight too large for the fp16 operands (|w| > 4096).
 constexpr int kDevErrBadWeights = 0x201;
-// Device error code: a value of v or dO beyond the fp16 range (|x| > 65504).
+// Device error code: a value the fp16 staging cannot carry: |v| > 65504, or
+// a finite |dO| >= 2^63 (beyond the per-row scaling's range).
 constexpr int kDevErrRange = 0x202;
 
-// Workspace layout: dA rows, then D, then the renormalised lse, each 256-byte
-// aligned (D and lse share the size bwd_ws_d_bytes).
+// Workspace layout, each part 256-byte aligned: dA rows, D, the renormalised
+// lse (D and lse share the size bwd_ws_d_bytes), then the two exponent records.
+inline size_t bwd_round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 inline size_t bwd_ws_da_bytes(long long B, long long T, int Hq) {
-  return ((static_cast<size_t>(B) * T * Hq * kHeadDim * 2) + 255) & ~static_cast<size_t>(255);
+  return bwd_round256(static_cast<size_t>(B) * T * Hq * kHeadDim * 2);
 }
 inline size_t bwd_ws_d_bytes(long long B, long long T, int Hq) {
-  return ((static_cast<size_t>(B) * T * Hq * 4) + 255) & ~static_cast<size_t>(255);
+  return bwd_round256(static_cast<size_t>(B) * T * Hq * 4);
+}
+inline size_t bwd_ws_ee_bytes(long long B, long long T, int Hq) {
+  return bwd_round256(static_cast<size_t>(B) * ((T + kTile - 1) / kTile) * Hq * 4);
+}
+inline size_t bwd_ws_ek_bytes(long long B, long long T, int Hkv) {
+  return bwd_round256(static_cast<size_t>(B) * ((T + kTile - 1) / kTile) * Hkv * 4);
+}
+inline size_t bwd_ws_total_bytes(long long B, long long T, int Hq, int Hkv) {
+  return bwd_ws_da_bytes(B, T, Hq) + 2 * bwd_ws_d_bytes(B, T, Hq) + bwd_ws_ee_bytes(B, T, Hq) +
+         bwd_ws_ek_bytes(B, T, Hkv);
 }
 
 int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,

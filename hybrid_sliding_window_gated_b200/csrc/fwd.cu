@@ -750,12 +750,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.lse[(static_cast<long long>(c.b) * a.Hq + hq) * a.T + pos] =
             (ms + __log2f(l)) * 0.6931471805599453f;
 
-      // ---- epilogue E(n): o = A/l * sigmoid(g) = (A * l^-1/2) * (1 + tanh(g/2)),
-      // written over g(n) in Q slot r, 32 columns per step.
+      // ---- epilogue E(n): o = A/l * sigmoid(g), written over g(n) in Q slot r,
+      // 32 columns per step.
       if (!mbar_wait_inl(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
       if (!mbar_wait_inl(&sm.gfull[qs], qph, abort, a.err, kSiteGFull)) { ok = false; break; }
       tc_fence_after();
-      const float2 hl2 = make_float2(0.5f / l, 0.5f / l);
+      const float2 il2 = make_float2(1.0f / l, 1.0f / l);
       {
         // Chunk ch: 32 columns of O, written over the same columns of g.
         auto gate = [&](const uint32_t(&ov)[32], int ch) {
@@ -768,12 +768,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ow[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 t =
-                  tanh2_f16(__fmul2_rn(bf16x2_to_f2(gw[e]), make_float2(0.5f, 0.5f)));
+              const float2 sg = sigmoid2(bf16x2_to_f2(gw[e]));
               const float2 acc = __fmul2_rn(make_float2(__uint_as_float(ov[8 * i + 2 * e]),
                                                         __uint_as_float(ov[8 * i + 2 * e + 1])),
-                                            hl2);
-              const float2 o2 = __ffma2_rn(acc, t, acc);
+                                            il2);
+              const float2 o2 = __fmul2_rn(acc, sg);
               ow[e] = pack_bf16x2(o2.x, o2.y);
             }
             *gp = make_uint4(ow[0], ow[1], ow[2], ow[3]);

@@ -16,22 +16,35 @@ only on the difference of the two positions, so the attention is the same.
 Backward: the same chunk, with dO = 0 on the halo rows and their lse set to
 log(i + 1), the exact normaliser of a zero query row over its i + 1 keys.  The
 halo keys' dk and dv (this rank's queries' share) go back to rank r - 1, which
-adds them to its last W - 1 rows; dq and dg need nothing from other ranks.
-dwq and dwk are sums over tokens, so they are all-reduced over the group.
+adds them to its own share of its last W - 1 rows; both shares come out of the
+kernel in fp32 (swa_bwd_edges), so the sum is rounded to bf16 once, as a
+single-GPU backward rounds it.  dq and dg need nothing from other ranks.  dwq
+and dwk are sums over tokens, so they are all-reduced over the group.
 
 Exchanges are point-to-point sends to the next (forward) or previous
-(backward) rank through torch.distributed (NCCL between GPUs).
+(backward) rank through torch.distributed (NCCL between GPUs).  One rank's
+step, given the halo it received, is :func:`rank_fwd` / :func:`rank_bwd`, which
+need no process group.
+
+Cost: the kernels take one contiguous [B, T, H, D] tensor per input, so each
+rank assembles its chunk by copying q, k, v and g (and dO in the backward)
+behind the halo rows, and copies o, lse, dq, dk, dv and dg out of the chunk
+again.  Those copies move about as many bytes as the forward kernel itself;
+the halo rows' own compute (W - 1 query rows per rank) is small beside them.
+Needs eps > 0: the halo query rows are zero.
 """
 import torch
 import torch.distributed as dist
 
 from . import bwd as _kernel_bwd
+from . import bwd_edges as _kernel_bwd_edges
 from . import fwd as _kernel_fwd
 
 # The per-rank computation: the library's kernels.  (The CPU tests of the
-# exchange logic replace these two with a host implementation.)
+# exchange logic replace these with a host implementation.)
 _local_fwd = _kernel_fwd
 _local_bwd = _kernel_bwd
+_local_bwd_edges = _kernel_bwd_edges
 
 
 def _ranks(group):
@@ -60,22 +73,26 @@ def _exchange(send, recv_like, to_next, group):
     return got
 
 
-def _halo_in(k, v, halo, group):
+def _halo_in(k, v, halo, eps, group):
     rank, world, _ = _ranks(group)
     if world == 1:
         return None
-    # Agreed by every rank before any exchange, so that all of them raise.
-    ok = torch.tensor([int(rank + 1 == world or k.shape[1] >= halo)], dtype=torch.int32,
-                      device=k.device)
+    # Both preconditions are agreed by every rank before any exchange, so
+    # that all of them raise together rather than one waiting on a send.
+    ok = torch.tensor([int(rank + 1 == world or k.shape[1] >= halo), int(eps > 0.0)],
+                      dtype=torch.int32, device=k.device)
     dist.all_reduce(ok, op=dist.ReduceOp.MIN, group=group)
-    if int(ok.item()) == 0:
+    if int(ok[0].item()) == 0:
         raise ValueError(f"every rank but the last must hold at least {halo} tokens")
+    _check_eps(eps if int(ok[1].item()) else 0.0)
     tails = [k[:, -halo:], v[:, -halo:]]
     return _exchange(tails, tails, True, group)
 
 
 def _with_halo(x, halo_rows):
-    """[B, T, H, D] -> [B, len + T, H, D] with `halo_rows` (or zeros) in front."""
+    """[B, T, H, D] -> [B, len + T, H, D] with `halo_rows` (or zeros) in front.
+    This copies x: the kernels take one contiguous [B, T, H, D] tensor per
+    input, so the chunk is assembled here."""
     return torch.cat([halo_rows, x], dim=1)
 
 
@@ -85,21 +102,79 @@ def halo_lse(B, Hq, n, device):
     return lse.to(device).view(1, 1, n).expand(B, Hq, n).contiguous()
 
 
+def _check_eps(eps):
+    # The halo query rows are zero: with eps = 0 their RMSNorm divides 0 by 0,
+    # and the NaN would reach the halo keys' dk and dv and, through the
+    # all-reduce, dwq and dwk on every rank.
+    if not eps > 0.0:
+        raise ValueError("sequence sharding needs eps > 0 (its halo query rows are zero)")
+
+
+def rank_fwd(q, k, v, g, wq, wk, halo, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
+             scale=0.0, want_lse=False):
+    """One rank's forward, given the halo it received: `halo` is (k, v) of the
+    previous rank's last W - 1 tokens, or None on the first rank."""
+    kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
+    if halo is None:
+        return _local_fwd(q, k, v, g, wq, wk, want_lse=want_lse, **kw)
+    _check_eps(eps)
+    hk, hv = halo
+    n = hk.shape[1]
+    zq = torch.zeros((q.shape[0], n) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
+    o, lse = _local_fwd(_with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv),
+                        _with_halo(g, zq), wq, wk, want_lse=True, **kw)
+    o = o[:, n:].contiguous()
+    return (o, lse[:, :, n:].contiguous()) if want_lse else o
+
+
+def rank_bwd(q, k, v, g, wq, wk, lse, dO, halo, *, tail=0, window=128, rot_dim=42,
+             rope_base=1e4, eps=1e-6, scale=0.0):
+    """One rank's backward, given the halo it received (as in :func:`rank_fwd`).
+    Returns (dq, dk, dv, dg, dwq, dwk, back, own): `back` is this rank's share
+    of the gradient of the halo keys, [B, W - 1, Hkv, 2, D] fp32 (dk, dv), which
+    belongs to the previous rank's last W - 1 rows (None on the first rank);
+    `own` is this rank's share of its own last `tail` keys in the same fp32
+    form (None when tail is 0), to which the next rank's `back` is added by
+    :func:`add_back`.  dwq and dwk are this rank's share."""
+    kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
+    n = 0 if halo is None else halo[0].shape[1]
+    if halo is None and tail == 0:
+        return tuple(_local_bwd(q, k, v, g, wq, wk, lse, dO, **kw)) + (None, None)
+    if halo is None:
+        grads, _, own = _local_bwd_edges(q, k, v, g, wq, wk, lse, dO, 0, tail, **kw)
+        return tuple(grads) + (None, own)
+    _check_eps(eps)
+    hk, hv = halo
+    B, Hq = q.shape[0], q.shape[2]
+    zq = torch.zeros((B, n) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
+    lse_c = torch.cat([halo_lse(B, Hq, n, lse.device).to(lse.dtype), lse], dim=2)
+    grads, back, own = _local_bwd_edges(
+        _with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv), _with_halo(g, zq), wq, wk,
+        lse_c, _with_halo(dO, zq), n, tail, **kw)
+    dq, dk, dv, dg, dwq, dwk = grads
+    dq, dk, dv, dg = (x[:, n:].contiguous() for x in (dq, dk, dv, dg))
+    return dq, dk, dv, dg, dwq, dwk, back, own
+
+
+def add_back(dk, dv, own, back):
+    """Write this rank's last W - 1 rows of dk and dv as the sum of its own
+    share (`own` from its :func:`rank_bwd`) and the next rank's share (`back`
+    from the next rank's :func:`rank_bwd`), both fp32: the sum is rounded to
+    dk's dtype once."""
+    n = back.shape[1]
+    acc = torch.promote_types(own.dtype, torch.float32)
+    tot = own.to(acc) + back.to(acc)
+    dk[:, -n:] = tot[:, :, :, 0].to(dk.dtype)
+    dv[:, -n:] = tot[:, :, :, 1].to(dv.dtype)
+
+
 def fwd(q, k, v, g, wq, wk, *, group=None, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
         scale=0.0, want_lse=False):
     """o (and lse [B, Hq, T_r]) for this rank's tokens.  q, g: [B, T_r, Hq, D];
     k, v: [B, T_r, Hkv, D]."""
-    halo = window - 1
-    kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
-    got = _halo_in(k, v, halo, group)
-    if got is None:
-        return _local_fwd(q, k, v, g, wq, wk, want_lse=want_lse, **kw)
-    hk, hv = got
-    zq = torch.zeros((q.shape[0], halo) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
-    o, lse = _local_fwd(_with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv),
-                        _with_halo(g, zq), wq, wk, want_lse=True, **kw)
-    o = o[:, halo:].contiguous()
-    return (o, lse[:, :, halo:].contiguous()) if want_lse else o
+    halo = _halo_in(k, v, window - 1, eps, group)
+    return rank_fwd(q, k, v, g, wq, wk, halo, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale, want_lse=want_lse)
 
 
 def bwd(q, k, v, g, wq, wk, lse, dO, *, group=None, window=128, rot_dim=42, rope_base=1e4,
@@ -107,33 +182,26 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, group=None, window=128, rot_dim=42, rope
     """(dq, dk, dv, dg, dwq, dwk) for this rank's tokens; lse is this rank's
     rows from :func:`fwd`.  dwq and dwk are the group's totals when
     ``reduce_weight_grads``, else this rank's share."""
-    halo = window - 1
+    halo_n = window - 1
     rank, world, _ = _ranks(group)
-    kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
-    got = _halo_in(k, v, halo, group)
-    if got is None:
-        dq, dk, dv, dg, dwq, dwk = _local_bwd(q, k, v, g, wq, wk, lse, dO, **kw)
-        back = []
-    else:
-        hk, hv = got
-        B, Hq = q.shape[0], q.shape[2]
-        zq = torch.zeros((B, halo) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
-        lse_c = torch.cat([halo_lse(B, Hq, halo, lse.device).to(lse.dtype), lse], dim=2)
-        dq, dk, dv, dg, dwq, dwk = _local_bwd(
-            _with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv), _with_halo(g, zq), wq, wk,
-            lse_c, _with_halo(dO, zq), **kw)
-        back = [dk[:, :halo], dv[:, :halo]]
-        dq, dk, dv, dg = (x[:, halo:].contiguous() for x in (dq, dk, dv, dg))
-    # the next rank's share of the gradient of this rank's last W - 1 keys
-    ret = _exchange(back, [k[:, -halo:], v[:, -halo:]], False, group) if world > 1 else None
-    if ret is not None:  # summed in at least fp32, rounded once
-        acc = torch.promote_types(dk.dtype, torch.float32)
-        dk[:, -halo:] = (dk[:, -halo:].to(acc) + ret[0].to(acc)).to(dk.dtype)
-        dv[:, -halo:] = (dv[:, -halo:].to(acc) + ret[1].to(acc)).to(dv.dtype)
+    halo = _halo_in(k, v, halo_n, eps, group)
+    tail = halo_n if rank + 1 < world else 0
+    dq, dk, dv, dg, dwq, dwk, back, own = rank_bwd(q, k, v, g, wq, wk, lse, dO, halo, tail=tail,
+                                                   window=window, rot_dim=rot_dim,
+                                                   rope_base=rope_base, eps=eps, scale=scale)
+    # the next rank's share of the gradient of this rank's last W - 1 keys,
+    # exchanged in fp32 (or wider, for wider inputs)
+    wide = torch.promote_types(k.dtype, torch.float32)
+    like = [torch.empty((k.shape[0], halo_n, k.shape[2], 2, k.shape[3]), dtype=wide,
+                        device=k.device)]
+    send = [] if back is None else [back.to(wide)]
+    ret = _exchange(send, like, False, group) if world > 1 else None
+    if ret is not None:
+        add_back(dk, dv, own, ret[0])
     if reduce_weight_grads and world > 1:
         dist.all_reduce(dwq, group=group)
         dist.all_reduce(dwk, group=group)
     return dq, dk, dv, dg, dwq, dwk
 
 
-__all__ = ["fwd", "bwd", "halo_lse"]
+__all__ = ["fwd", "bwd", "rank_fwd", "rank_bwd", "add_back", "halo_lse"]

@@ -111,15 +111,40 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
  * misaligned pointer returns SWA_ERR_INVALID_ARG before any launch.  The
  * chain rule covers the gate, the softmax, RoPE and the
  * RMSNorm (the weights included).  The contractions run on fp16 operands
- * (three more mantissa bits than bf16), so |v| and |dO| must stay within the
- * fp16 range (65504) and |wq|, |wk| <= 4096; values beyond are reported by
- * swa_get_last_device_error() as SWA_ERR_INVALID_ARG.
+ * (three more mantissa bits than bf16).  dA = dO sigma(g) and dS are staged
+ * with power-of-two scales -- per query row from max|dO| of the row, per
+ * 128-query tile from max|v| of its keys -- so a row whose largest |dO| lies
+ * in [2^-62, 2^63) keeps fp16's relative precision, however small the
+ * gradient; a finite |dO| >= 2^63, |v| > 65504 or |wq|, |wk| > 4096 is reported by
+ * swa_get_last_device_error() as SWA_ERR_INVALID_ARG.  v is staged in fp16
+ * as is: exact for |v| >= 2^-14, absolute error at most 2^-25 below that.
  */
 int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
             const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
             const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
             swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, void* workspace,
             size_t workspace_bytes, void* stream);
+
+/*
+ * swa_bwd that also writes, in fp32, dk and dv of the first n_lo and the last
+ * n_hi tokens of every sequence (0 <= n_lo, n_hi <= T): dkv_lo [B, n_lo, Hkv,
+ * 2, D] and dkv_hi [B, n_hi, Hkv, 2, D] (index 0 of the fourth axis is dk, 1
+ * is dv), 8-byte aligned, caller-owned device memory; a buffer may be NULL when
+ * its count is 0.  The bf16 dk and dv are written as by swa_bwd.  For callers
+ * that add the partial gradients of the same keys from two calls -- sequence
+ * sharding, where a chunk's first W - 1 keys are the previous chunk's last
+ * W - 1 -- and want the sum rounded to bf16 once.  The partial sums are
+ * linear in the incoming gradient (the RMSNorm Jacobian depends on k only),
+ * so they add exactly.  No counterpart in the pages beyond the window itself
+ * (a token sees the W - 1 before it: jaehun.me review, "How Gated SWA
+ * Behaves"), whose halo crosses a chunk boundary.
+ */
+int swa_bwd_edges(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                  const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                  const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                  swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, int64_t n_lo,
+                  float* dkv_lo, int64_t n_hi, float* dkv_hi, void* workspace,
+                  size_t workspace_bytes, void* stream);
 
 /* Bytes of scratch swa_bwd needs for these parameters (0 if unsupported). */
 size_t swa_bwd_workspace_size(const swa_params_t* p);

@@ -127,6 +127,24 @@ def test_bwd_host_checks(L):
     assert L.swa_bwd(ctypes.byref(_params(T=0)), *([nul] * 15), 0, nul) == swa.OK
 
 
+def test_bwd_edges_host_checks(L):
+    p = _params(B=1, T=256, Hq=4, Hkv=1)
+    need = L.swa_bwd_workspace_size(ctypes.byref(p))
+    good = ctypes.c_void_p(1 << 20)
+    nul = ctypes.c_void_p(0)
+    i64 = ctypes.c_int64
+
+    def call(n_lo, lo, n_hi, hi, params=p):
+        return L.swa_bwd_edges(ctypes.byref(params), *([good] * 14), i64(n_lo), lo, i64(n_hi), hi,
+                               good, need, None)
+    assert call(-1, good, 0, nul) == swa.ERR_INVALID_ARG      # negative count
+    assert call(0, nul, 257, good) == swa.ERR_INVALID_ARG     # more rows than T
+    assert call(5, nul, 0, nul) == swa.ERR_INVALID_ARG        # rows but no buffer
+    assert call(5, ctypes.c_void_p((1 << 20) + 4), 0, nul) == swa.ERR_INVALID_ARG  # fp32 pairs
+    assert L.swa_bwd_edges(ctypes.byref(_params(T=0)), *([nul] * 14), i64(0), nul, i64(0), nul,
+                           nul, 0, None) == swa.OK
+
+
 def test_prefill_to_ring_host_checks(L):
     nul = ctypes.c_void_p(0)
     good = ctypes.c_void_p(1 << 20)

@@ -48,6 +48,92 @@ def test_tiny_config_backward():
     check_bwd(workloads.TINY)
 
 
+def check_bwd_scaled(cfg, do_scale=None, v_scale=1.0, row_scale=None):
+    """The backward at other magnitudes of dO and v than N(0, 1).  dO and v are
+    rescaled in fp32 and rounded to bf16 again (the oracle reads the same
+    bits); dO either by one factor or by a factor per (token, head) row.
+    Every gradient is compared by relative Frobenius error (max-abs bounds
+    mean nothing at these scales) and by max-abs error relative to the
+    product of the input scales it carries."""
+    inp = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=True)
+    if do_scale is not None:
+        inp["dO"] = (inp["dO"].float() * do_scale).bfloat16()
+    if row_scale is not None:
+        inp["dO"] = (inp["dO"].float() * row_scale[..., None]).bfloat16()
+    inp["v"] = (inp["v"].float() * v_scale).bfloat16()
+    ref = oracle.bwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["wq"]),
+                     f64(inp["wk"]), f64(inp["dO"]), W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+    got = run_gpu({k: v.to(DEV) for k, v in inp.items()}, cfg)
+    s_do = 1.0 if do_scale is None else do_scale
+    carried = {"dq": s_do * v_scale, "dk": s_do * v_scale, "dv": s_do, "dg": s_do * v_scale}
+    for name, x, r in zip(["dq", "dk", "dv", "dg"], got[:4], ref[:4]):
+        x = to_f64(x)
+        assert np.all(np.isfinite(x)), name
+        ma, fro = errors(x, r)
+        assert fro <= REL_FRO, f"{name}: rel_fro={fro:.3e}"
+        if row_scale is None:
+            assert ma <= 2e-2 * carried[name], f"{name}: max_abs={ma:.3e}"
+    for name, x, r in zip(["dwq", "dwk"], got[4:], ref[4:]):
+        fro = errors(to_f64(x), r)[1]
+        assert fro <= REL_FRO, f"{name}: rel_fro={fro:.3e}"
+    return got, ref
+
+
+@pytest.mark.parametrize("do_scale", [1e-3, 1e-5, 1e-7, 1e-12, 1e3, 1e6])
+def test_backward_at_upstream_gradient_scales(do_scale):
+    """Upstream gradients of training are far below N(0, 1) per element; fp16
+    staging of dA and dS without a scale would sink them into its subnormals."""
+    check_bwd_scaled(workloads.custom_prefill(1, 700, 8, 2, seed=41, backward=True),
+                     do_scale=do_scale)
+
+
+@pytest.mark.parametrize("v_scale,do_scale", [(1e-3, None), (1e-3, 1e-5), (30.0, 1e-4),
+                                              (1e-4, 1.0)])
+def test_backward_at_value_scales(v_scale, do_scale):
+    """Small v makes dP and dS small too: dS is staged with a scale from max|v|.
+    (v itself is staged in fp16, exactly for |v| >= 2^-14; below, its absolute
+    error is at most 2^-25, which the smallest scale here keeps well inside
+    the bound.)"""
+    check_bwd_scaled(workloads.custom_prefill(1, 520, 4, 1, seed=42, backward=True),
+                     do_scale=do_scale, v_scale=v_scale)
+
+
+def test_backward_with_row_magnitudes_spanning_six_decades():
+    """dO rows (token, head) scaled by 10^-U(0, 6): each query row is staged
+    with its own scale, so the smallest rows' dq keeps its relative accuracy;
+    the key-major pass shares one scale per key tile."""
+    cfg = workloads.custom_prefill(2, 600, 8, 2, seed=43, backward=True)
+    gen = torch.Generator().manual_seed(44)
+    rs = 10.0 ** (-6.0 * torch.rand((cfg.B, cfg.T, cfg.Hq), generator=gen))
+    got, ref = check_bwd_scaled(cfg, row_scale=rs)
+    small = (rs < 1e-4).numpy()
+    assert small.sum() > 100
+    fro = errors(to_f64(got[0])[small], ref[0][small])[1]
+    assert fro <= REL_FRO, f"dq of the rows under 1e-4: rel_fro={fro:.3e}"
+
+
+@pytest.mark.parametrize("g_mean", [-8.0, 8.0])
+def test_backward_with_nearly_shut_or_open_gates(g_mean):
+    """Gate logits ~ N(+-8, 1): sigma or 1 - sigma is ~3e-4, where a sigmoid
+    formed as 1/2 + tanh/2 (or sigma (1 - sigma) formed by cancellation)
+    loses its relative accuracy; dA = dO sigma and dg = dO A sigma (1 - sigma)
+    are compared by relative Frobenius error."""
+    cfg = workloads.custom_prefill(1, 600, 8, 2, seed=45, backward=True)
+    inp = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=True)
+    inp["g"] = (inp["g"].float() + g_mean).bfloat16()
+    ref = oracle.bwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["wq"]),
+                     f64(inp["wk"]), f64(inp["dO"]), W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+    got = run_gpu({k: v.to(DEV) for k, v in inp.items()}, cfg)
+    for name, x, r in zip(["dq", "dk", "dv", "dg", "dwq", "dwk"], got, ref):
+        fro = errors(to_f64(x), r)[1]
+        assert fro <= REL_FRO, f"{name}: rel_fro={fro:.3e}"
+
+
+def test_training_shape_backward_at_gradient_scale_1e_6():
+    cfg = workloads.TRAIN
+    check_bwd_scaled(cfg, do_scale=1e-6)
+
+
 @pytest.mark.parametrize("B,T,Hq,Hkv", [
     (1, 1, 4, 1), (1, 127, 4, 1), (1, 128, 4, 1), (1, 129, 4, 1), (2, 300, 8, 2),
     (1, 520, 2, 2), (1, 700, 3, 1), (3, 257, 8, 8), (1, 1000, 32, 8),
@@ -114,13 +200,14 @@ def test_values_beyond_fp16_range_are_reported():
     assert swa.get_last_device_error()[0] == swa.OK  # cleared
 
 
-def test_upstream_gradient_beyond_fp16_range_is_reported():
-    """dA = dO * sigmoid(g) is staged in fp16 too: a dO past its range is refused."""
+def test_upstream_gradient_beyond_the_staging_range_is_reported():
+    """dA = dO * sigmoid(g) is staged in fp16 after a per-row power-of-two
+    scale; a finite |dO| >= 2^63 is beyond what that scale covers and is refused."""
     cfg, d = _small_inputs()
     o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], want_lse=True)
     torch.cuda.synchronize()
     assert swa.get_last_device_error()[0] == swa.OK
-    d["dO"][0, 150, 2, 100] = -2.0e5
+    d["dO"][0, 150, 2, 100] = -1.0e20
     swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"])
     assert swa.get_last_device_error()[0] == swa.ERR_INVALID_ARG
     assert swa.get_last_device_error()[0] == swa.OK
@@ -147,3 +234,30 @@ def test_forced_timeout_is_reported_and_context_survives():
     assert code == swa.ERR_DEVICE_TIMEOUT and site >= 0x100
     assert swa.get_last_device_error()[0] == swa.OK
     check_bwd(workloads.TINY)
+
+
+@pytest.mark.parametrize("n_lo,n_hi", [(127, 127), (0, 50), (300, 0), (1, 299)])
+def test_edge_rows_in_fp32(n_lo, n_hi):
+    """swa_bwd_edges: the fp32 copies of the first n_lo and last n_hi rows of dk
+    and dv round to exactly the bf16 rows the same call writes, and match the
+    oracle; the other outputs equal swa_bwd's bit for bit."""
+    cfg = workloads.custom_prefill(2, 300, 8, 2, seed=46, backward=True)
+    inp = workloads.prefill_inputs(cfg, device="cpu", with_grad_out=True)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    o, lse = swa.fwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], want_lse=True)
+    plain = swa.bwd(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"])
+    grads, lo, hi = swa.bwd_edges(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], lse, d["dO"],
+                                  n_lo, n_hi)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    for a, b in zip(grads[:4], plain[:4]):
+        assert torch.equal(a, b)
+    ref = oracle.bwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["wq"]),
+                     f64(inp["wk"]), f64(inp["dO"]), W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+    T = cfg.T
+    for buf, rows in ((lo, slice(0, n_lo)), (hi, slice(T - n_hi, T))):
+        if buf is None:
+            continue
+        for j, (name, full) in enumerate((("dk", grads[1]), ("dv", grads[2]))):
+            assert torch.equal(buf[:, :, :, j].to(torch.bfloat16), full[:, rows]), name
+            assert_parity(to_f64(buf[:, :, :, j]), ref[1 + j][:, rows], f"{name} edge rows")

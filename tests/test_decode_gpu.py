@@ -128,6 +128,15 @@ def test_saturated_gate_gives_zero():
     assert torch.count_nonzero(o).item() == 0
 
 
+def test_open_gate_gives_ungated_attention():
+    """g = +inf: sigmoid is exactly 1 and o is the plain attention over the ring."""
+    cfg = workloads.Decode("decode test", N=6, layers=1, Hq=8, Hkv=2, base=1e7, seed=15)
+    inp = workloads.decode_layer_inputs(cfg, layer=0)
+    inp["g"] = torch.full_like(inp["g"], float("inf"))
+    o, kc, vc, o_ref, kc_ref, vc_ref = run_both(inp, cfg.R, cfg.base)
+    assert_parity(to_f64(o), o_ref, "decode o with g = +inf")
+
+
 def test_forced_timeout_is_reported_and_context_survives():
     """A wait that nothing completes ends by its time limit; the kernel drains
     its copies, reports the site, and the next call computes correctly."""

@@ -48,13 +48,25 @@ def host_bwd(q, k, v, g, wq, wk, lse, dO, *, window, rot_dim, rope_base, eps, sc
     return tuple(torch.from_numpy(x) for x in grads)
 
 
+def host_bwd_edges(q, k, v, g, wq, wk, lse, dO, n_lo, n_hi, **kw):
+    grads = host_bwd(q, k, v, g, wq, wk, lse, dO, **kw)
+    dkv = torch.stack([grads[1], grads[2]], dim=3)  # [B, T, Hkv, 2, D]
+    T = q.shape[1]
+    return grads, (dkv[:, :n_lo] if n_lo else None), (dkv[:, T - n_hi:] if n_hi else None)
+
+
+def _use_host(seqpar):
+    seqpar._local_fwd, seqpar._local_bwd = host_fwd, host_bwd
+    seqpar._local_bwd_edges = host_bwd_edges
+
+
 def _rank_main(rank, world, port, out):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         from hybrid_sliding_window_gated_b200 import seqpar
-        seqpar._local_fwd, seqpar._local_bwd = host_fwd, host_bwd
+        _use_host(seqpar)
         x = _inputs()
         s0 = sum(LENGTHS[:rank])
         sl = {k: (v[:, s0:s0 + LENGTHS[rank]].contiguous() if v.dim() == 4 else v)
@@ -143,5 +155,74 @@ def test_the_product_path_calls_the_kernel_wrappers():
     import hybrid_sliding_window_gated_b200 as swa
     from hybrid_sliding_window_gated_b200 import seqpar
     assert seqpar._local_fwd is swa.fwd and seqpar._local_bwd is swa.bwd
+    assert seqpar._local_bwd_edges is swa.bwd_edges
     src = open(seqpar.__file__).read()
     assert "oracle" not in src
+
+
+def _eps_rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from hybrid_sliding_window_gated_b200 import seqpar
+        seqpar._local_fwd = host_fwd
+        x = {k: (v[:, :150].contiguous() if v.dim() == 4 else v) for k, v in _inputs().items()}
+        try:
+            seqpar.fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=W, rot_dim=R,
+                       eps=0.0)
+            out[rank] = "returned"
+        except ValueError:
+            out[rank] = "raised"
+    finally:
+        dist.destroy_process_group()
+
+
+def test_eps_zero_is_refused_on_every_rank():
+    """The halo query rows are zero, so eps = 0 would make their RMSNorm NaN,
+    and the NaN would spread to dk, dv and the all-reduced weight gradients."""
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_eps_rank_main, args=(2, _free_port(), out), nprocs=2, join=True)
+        assert dict(out) == {0: "raised", 1: "raised"}
+
+
+def test_rank_steps_without_a_process_group():
+    """rank_fwd / rank_bwd / add_back chained by hand over three chunks equal
+    the oracle on the whole sequences (the host computation standing in for
+    the kernels, as above)."""
+    from hybrid_sliding_window_gated_b200 import seqpar
+    old = seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges
+    _use_host(seqpar)
+    try:
+        x = _inputs()
+        kw = dict(window=W, rot_dim=R, rope_base=BASE, eps=EPS)
+        outs, halo, s0 = [], None, 0
+        for T in LENGTHS:
+            sl = {k: (v[:, s0:s0 + T].contiguous() if v.dim() == 4 else v) for k, v in x.items()}
+            o, lse = seqpar.rank_fwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["wq"], sl["wk"], halo,
+                                     want_lse=True, **kw)
+            outs.append((sl, halo, o, lse))
+            halo = (sl["k"][:, -(W - 1):], sl["v"][:, -(W - 1):])
+            s0 += T
+        grads = []
+        for r, (sl, halo, o, lse) in enumerate(outs):
+            tail = W - 1 if r + 1 < len(outs) else 0
+            grads.append(seqpar.rank_bwd(sl["q"], sl["k"], sl["v"], sl["g"], sl["wq"], sl["wk"],
+                                         lse, sl["dO"], halo, tail=tail, **kw))
+        for r in range(1, len(grads)):
+            seqpar.add_back(grads[r - 1][1], grads[r - 1][2], grads[r - 1][7], grads[r][6])
+    finally:
+        seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges = old
+    n = {k: v.numpy() for k, v in x.items()}
+    o_ref, _ = oracle.fwd(n["q"], n["k"], n["v"], n["g"], n["wq"], n["wk"], W=W, R=R, base=BASE,
+                          eps=EPS)
+    g_ref = oracle.bwd(n["q"], n["k"], n["v"], n["g"], n["wq"], n["wk"], n["dO"], W=W, R=R,
+                       base=BASE, eps=EPS)
+    np.testing.assert_allclose(np.concatenate([r[2].numpy() for r in outs], axis=1), o_ref,
+                               rtol=0, atol=1e-10)
+    for i, name in enumerate(["dq", "dk", "dv", "dg"]):
+        got = np.concatenate([gr[i].numpy() for gr in grads], axis=1)
+        np.testing.assert_allclose(got, g_ref[i], rtol=0, atol=1e-9, err_msg=name)
+    np.testing.assert_allclose(sum(gr[4].numpy() for gr in grads), g_ref[4], rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(sum(gr[5].numpy() for gr in grads), g_ref[5], rtol=1e-9, atol=1e-9)
