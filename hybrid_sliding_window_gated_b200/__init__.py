@@ -17,6 +17,7 @@ import os
 import torch
 
 __all__ = ["fwd", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
+           "global_fwd", "global_decode_step", "global_decode_workspace_size",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswa.so")
@@ -67,6 +68,13 @@ def lib():
         L.swa_decode_step.restype = ctypes.c_int
         L.swa_prefill_to_ring.argtypes = [P] + [_vp] * 6
         L.swa_prefill_to_ring.restype = ctypes.c_int
+        L.swa_global_fwd.argtypes = [P] + [_vp] * 9 + [ctypes.c_int64, _vp]
+        L.swa_global_fwd.restype = ctypes.c_int
+        L.swa_global_decode_workspace_size.argtypes = [P, ctypes.c_int64]
+        L.swa_global_decode_workspace_size.restype = ctypes.c_size_t
+        L.swa_global_decode_step.argtypes = [P] + [_vp] * 8 + [ctypes.c_int64, _vp, _vp,
+                                                               ctypes.c_size_t, _vp]
+        L.swa_global_decode_step.restype = ctypes.c_int
         L.swa_error_string.argtypes = [ctypes.c_int]
         L.swa_error_string.restype = ctypes.c_char_p
         L.swa_get_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int)]
@@ -280,6 +288,69 @@ def prefill_to_ring(k, v, wk, k_cache, v_cache, *, Hq, rot_dim=42, rope_base=1e7
     rc = lib().swa_prefill_to_ring(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(wk), _ptr(k_cache),
                                    _ptr(v_cache), _stream(stream))
     _check(rc, "swa_prefill_to_ring")
+
+
+def global_fwd(q, k, v, wq, wk, k_cache, v_cache, *, rot_dim=42, rope_base=1e4, eps=1e-6,
+               scale=0.0, out=None, lse=None, want_lse=False, flags=0, stream=None):
+    """Global causal GQA layer over positions 0..T-1 (swa_global_fwd): no window,
+    no gate.  q: [B,T,Hq,128]; k, v: [B,T,Hkv,128] bf16; wq, wk: [128] fp32.
+    Fills slots 0..T-1 of k_cache, v_cache [B,Hkv,cap,128] (cap >= T) with k'
+    and v and returns o (and lse [B,Hq,T] when asked)."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    cap = k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=0, rot_dim=rot_dim, rope_base=rope_base,
+                    eps=eps, scale=scale, flags=flags)
+    nq, nk = B * T * Hq * D, B * T * Hkv * D
+    nc = B * Hkv * cap * D if nq else 0
+    bf, f32 = torch.bfloat16, torch.float32
+    opt = {} if lse is None else {"lse": (lse, f32, B * Hq * T)}
+    _need("swa_global_fwd", q.device, q=(q, bf, nq), k=(k, bf, nk), v=(v, bf, nk),
+          wq=(wq, f32, D if nq else 0), wk=(wk, f32, D if nq else 0), out=(out, bf, nq),
+          k_cache=(k_cache, bf, nc), v_cache=(v_cache, bf, nc), **opt)
+    rc = lib().swa_global_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk),
+                              _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), cap,
+                              _stream(stream))
+    _check(rc, "swa_global_fwd")
+    return (out, lse) if lse is not None else out
+
+
+def global_decode_workspace_size(N, Hq, Hkv, cap, *, head_dim=128, rot_dim=42):
+    p = make_params(N, 1, Hq, Hkv, head_dim=head_dim, window=0, rot_dim=rot_dim)
+    return int(lib().swa_global_decode_workspace_size(ctypes.byref(p), cap))
+
+
+def global_decode_step(pos, q, k_new, v_new, wq, wk, k_cache, v_cache, *, rot_dim=42,
+                       rope_base=1e7, eps=1e-6, scale=0.0, out=None, workspace=None, flags=0,
+                       stream=None):
+    """One decode step of a global layer (swa_global_decode_step): writes k', v at
+    slot pos[n] of the [N,Hkv,cap,128] caches and returns o [N,Hq,128]."""
+    N, Hq, D = q.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    p = make_params(N, 1, Hq, Hkv, head_dim=D, window=0, rot_dim=rot_dim, rope_base=rope_base,
+                    eps=eps, scale=scale, flags=flags)
+    nbytes = int(lib().swa_global_decode_workspace_size(ctypes.byref(p), cap))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    nq, nk = N * Hq * D, N * Hkv * D
+    bf, f32 = torch.bfloat16, torch.float32
+    _need("swa_global_decode_step", q.device, pos=(pos, torch.int64, N), q=(q, bf, nq),
+          k_new=(k_new, bf, nk), v_new=(v_new, bf, nk), wq=(wq, f32, D if N else 0),
+          wk=(wk, f32, D if N else 0), k_cache=(k_cache, bf, nk * cap),
+          v_cache=(v_cache, bf, nk * cap), out=(out, bf, nq),
+          workspace=(workspace, torch.uint8, nbytes if N else 0))
+    rc = lib().swa_global_decode_step(ctypes.byref(p), _ptr(pos), _ptr(q), _ptr(k_new),
+                                      _ptr(v_new), _ptr(wq), _ptr(wk), _ptr(k_cache),
+                                      _ptr(v_cache), cap, _ptr(out), _ptr(workspace),
+                                      workspace.numel(), _stream(stream))
+    _check(rc, "swa_global_decode_step")
+    return out
 
 
 def get_last_device_error(stream=None):

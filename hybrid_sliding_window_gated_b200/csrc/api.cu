@@ -9,6 +9,7 @@
 
 #include "bwd_internal.h"
 #include "decode_internal.h"
+#include "global_internal.h"
 #include "swa_internal.h"
 
 namespace swa {
@@ -124,6 +125,14 @@ int check_params(const swa_params_t* p, bool decode) {
   // below (B T Hq 128 x 2 bytes < 2^60) and every tile count fits in int64.
   if (!decode && p->B * p->T > (1ll << 40)) return SWA_ERR_UNSUPPORTED;
   return SWA_OK;
+}
+
+// The global layers have no window: their parameter blocks carry window = 0.
+static int check_params_global(const swa_params_t* p, bool decode) {
+  if (p == nullptr || p->window != 0) return SWA_ERR_INVALID_ARG;
+  swa_params_t c = *p;
+  c.window = kWindow;
+  return check_params(&c, decode);
 }
 
 static float score_scale(const swa_params_t* p) {
@@ -419,6 +428,158 @@ int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t*
                            CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
   return launch_decode(tk, tv, a, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+extern "C" {
+
+int swa_global_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                   const swa_bf16_t* v, const float* wq, const float* wk, swa_bf16_t* o,
+                   float* lse, swa_bf16_t* k_cache, swa_bf16_t* v_cache, int64_t cache_cap,
+                   void* stream) {
+  int rc = check_params_global(p, false);
+  if (rc != SWA_OK) return rc;
+  if (cache_cap < p->T) return SWA_ERR_INVALID_ARG;
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  if (cache_cap > (1ll << 30) || p->B * cache_cap > (1ll << 40)) return SWA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !wq || !wk || !o || !k_cache || !v_cache) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(wq) ||
+      !aligned16(wk) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  int* err = nullptr;
+  if ((rc = device_error_word(&err)) != SWA_OK) return rc;
+
+  GlobalKvArgs kv{};
+  kv.B = static_cast<int>(p->B);
+  kv.T = static_cast<int>(p->T);
+  kv.Hkv = p->Hkv;
+  kv.half_rot = p->rot_dim / 2;
+  kv.eps = p->eps;
+  kv.cap = cache_cap;
+  kv.pos = nullptr;
+  kv.k = k;
+  kv.v = v;
+  kv.wk = wk;
+  kv.k_cache = k_cache;
+  kv.v_cache = v_cache;
+  kv.err = err;
+  fill_inv_freq(p, kv.inv_freq);
+
+  GlobalFwdArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.tiles = static_cast<int>((p->T + kTile - 1) / kTile);
+  a.pairs = (a.G + 1) / 2;
+  a.units = static_cast<long long>(a.tiles) * p->B * p->Hkv * a.pairs;
+  if (a.units > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
+  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.flags = p->flags;
+  a.wq = wq;
+  a.wk = wk;
+  a.lse = lse;
+  a.err = err;
+  fill_inv_freq(p, a.inv_freq);
+
+  // q and o in boxes of 128 tokens x 64 dims, as in swa_fwd; the caches
+  // [B, Hkv, cap, D] in boxes of 128 slots x 64 dims.
+  CUtensorMap tq, tk, tv, to;
+  const uint64_t D = kHeadDim, T = p->T, B = p->B, cap = cache_cap;
+  if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&to, o, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tk, k_cache, D, cap, p->Hkv, B, 64, kTile, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tv, v_cache, D, cap, p->Hkv, B, 64, kTile, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = p->B * (static_cast<long long>(a.tiles) * kTile);
+  if ((rc = launch_global_kv(kv, rows, st)) != SWA_OK) return rc;
+  return launch_global_fwd(p->rot_dim, tq, tk, tv, to, a, st);
+}
+
+size_t swa_global_decode_workspace_size(const swa_params_t* p, int64_t cache_cap) {
+  if (check_params_global(p, true) != SWA_OK || cache_cap <= 0) return 0;
+  return global_decode_ws_bytes(p->B, p->Hkv, p->Hq / p->Hkv, cache_cap);
+}
+
+int swa_global_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
+                           const swa_bf16_t* k_new, const swa_bf16_t* v_new, const float* wq,
+                           const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                           int64_t cache_cap, swa_bf16_t* o, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  int rc = check_params_global(p, true);
+  if (rc != SWA_OK) return rc;
+  if (cache_cap <= 0) return SWA_ERR_INVALID_ARG;
+  if (p->Hq / p->Hkv > kGlobalMaxGroup) return SWA_ERR_UNSUPPORTED;
+  if (cache_cap > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
+  if (p->B == 0) return SWA_OK;
+  if (!pos || !q || !k_new || !v_new || !wq || !wk || !k_cache || !v_cache || !o || !workspace)
+    return SWA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) || !aligned16(q) || !aligned16(k_new) ||
+      !aligned16(v_new) || !aligned16(wq) || !aligned16(wk) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(o) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SWA_ERR_INVALID_ARG;
+  const int G = p->Hq / p->Hkv;
+  if (workspace_bytes < global_decode_ws_bytes(p->B, p->Hkv, G, cache_cap))
+    return SWA_ERR_INVALID_ARG;
+  int* err = nullptr;
+  if ((rc = device_error_word(&err)) != SWA_OK) return rc;
+
+  GlobalKvArgs kv{};
+  kv.B = static_cast<int>(p->B);
+  kv.T = 1;
+  kv.Hkv = p->Hkv;
+  kv.half_rot = p->rot_dim / 2;
+  kv.eps = p->eps;
+  kv.cap = cache_cap;
+  kv.pos = pos;
+  kv.k = k_new;
+  kv.v = v_new;
+  kv.wk = wk;
+  kv.k_cache = k_cache;
+  kv.v_cache = v_cache;
+  kv.err = err;
+  fill_inv_freq(p, kv.inv_freq);
+
+  GlobalDecArgs a{};
+  a.N = static_cast<int>(p->B);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = G;
+  a.half_rot = p->rot_dim / 2;
+  a.chunks = static_cast<int>((cache_cap + kGlobalChunk - 1) / kGlobalChunk);
+  a.flags = p->flags;
+  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.cap = cache_cap;
+  a.pos = pos;
+  a.q = q;
+  a.wq = wq;
+  const size_t po = global_decode_ws_bytes(p->B, p->Hkv, G, cache_cap) -
+                    (((static_cast<size_t>(p->B) * p->Hkv * a.chunks * G * 2 * 4) + 255) &
+                     ~static_cast<size_t>(255));
+  a.part_o = static_cast<float*>(workspace);
+  a.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + po);
+  a.o = o;
+  a.err = err;
+  fill_inv_freq(p, a.inv_freq);
+
+  CUtensorMap tk, tv;
+  const uint64_t D = kHeadDim, cap = cache_cap, N = p->B;
+  if ((rc = encode_tmap_4d(&tk, k_cache, D, cap, p->Hkv, N, 64, kTile, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&tv, v_cache, D, cap, p->Hkv, N, 64, kTile, 1, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = launch_global_kv(kv, p->B, st)) != SWA_OK) return rc;
+  return launch_global_decode(tk, tv, a, st);
 }
 
 }  // extern "C"

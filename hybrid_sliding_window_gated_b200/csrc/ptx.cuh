@@ -352,13 +352,14 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 
 // Logistic function of two values with a small relative error everywhere
-// (about 1.2e-5, for either sign and any magnitude), and sigma (1 - sigma):
-//   e = 2^(-|g| log2(e)) in (0, 1]                 one MUFU operation each,
-//   r = 1 / (1 + e)                                 two Newton steps r <- r (2 - d r)
-//                                                   from the linear start (24 - 8 d)/17,
-//                                                   whose relative error 1/17 squares
-//                                                   at each step,
-//   sigma(g) = r for g >= 0, e r for g < 0,         sigma (1 - sigma) = e r^2.
+// (about 1e-4, for either sign and any magnitude), and sigma (1 - sigma):
+//   e = 2^(-|g| log2(e)) in (0, 1]          one MUFU operation each,
+//   r = 1 / (1 + e), d = 1 + e in (1, 2]     a quadratic start on [1, 2] with
+//                                            relative error 1.0e-2 (fitted for
+//                                            the minimax error of d r), then one
+//                                            Newton step r <- r (2 - d r), which
+//                                            squares it,
+//   sigma(g) = r for g >= 0, e r for g < 0,  sigma (1 - sigma) = e r^2.
 // Neither 1 - sigma nor 1 + tanh is ever formed, so a gate that is nearly
 // shut (sigma ~ e^g) keeps its relative accuracy.  g = -inf gives exactly 0,
 // +inf exactly 1.
@@ -366,13 +367,11 @@ __device__ __forceinline__ float2 sigmoid2(float2 g, float2* dsig = nullptr) {
   constexpr float kL2e = 1.4426950408889634f;
   const float2 e = make_float2(ex2_approx(-fabsf(g.x) * kL2e), ex2_approx(-fabsf(g.y) * kL2e));
   const float2 d = __fadd2_rn(e, make_float2(1.0f, 1.0f));
-  float2 r = __ffma2_rn(d, make_float2(-8.0f / 17.0f, -8.0f / 17.0f),
-                        make_float2(24.0f / 17.0f, 24.0f / 17.0f));
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float2 t = __ffma2_rn(make_float2(-d.x, -d.y), r, make_float2(1.0f, 1.0f));
-    r = __ffma2_rn(r, t, r);
-  }
+  float2 r = __ffma2_rn(d, make_float2(0.32286211f, 0.32286211f),
+                        make_float2(-1.45351115f, -1.45351115f));
+  r = __ffma2_rn(r, d, make_float2(2.12052006f, 2.12052006f));
+  const float2 t = __ffma2_rn(make_float2(-d.x, -d.y), r, make_float2(1.0f, 1.0f));
+  r = __ffma2_rn(r, t, r);
   const float2 er = __fmul2_rn(e, r);
   if (dsig != nullptr) *dsig = __fmul2_rn(er, r);
   return make_float2(g.x >= 0.0f ? r.x : er.x, g.y >= 0.0f ? r.y : er.y);

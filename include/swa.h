@@ -198,6 +198,50 @@ int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t*
 int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf16_t* v,
                         const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache, void* stream);
 
+/*
+ * Global causal GQA layers (no counterpart of the window: 5 of ZGCM-1's 32
+ * layers, at 6, 12, 18, 24 and 30, attend over the whole causal context with
+ * the same QK-RMSNorm, partial RoPE and GQA, and without the output gate --
+ * onedev.kr summary, "어떻게 동작하나"; jaehun.me review, "How Gated SWA
+ * Behaves"; they keep every token's K and V -- "Why the KV Cache Shrinks by
+ * 6.4x").  For these calls p->window must be 0 (no window).
+ *
+ * Prefill: o_i = softmax_j(scale q'_i . k'_j, j <= i) V for positions
+ * 0 .. T-1.  q [B,T,Hq,D], k, v [B,T,Hkv,D] bf16; wq, wk [D] fp32.  Writes o
+ * [B,T,Hq,D] bf16, lse [B,Hq,T] fp32 when lse != NULL, and the layer's
+ * full-length caches k_cache, v_cache [B, Hkv, cache_cap, D] bf16 (cache_cap
+ * >= T): slot t of (b, kv head) receives k' = RoPE_t(RMSNorm(k_t)) rounded to
+ * bf16 and v_t; the slots from T up to the end of T's 128-slot tile are
+ * zeroed, the rest are not touched.  The attention reads K' and V back from
+ * those caches.  Pointers 16-byte aligned.  Errors as swa_fwd.
+ */
+int swa_global_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                   const swa_bf16_t* v, const float* wq, const float* wk, swa_bf16_t* o,
+                   float* lse, swa_bf16_t* k_cache, swa_bf16_t* v_cache, int64_t cache_cap,
+                   void* stream);
+
+/* Bytes of scratch swa_global_decode_step needs (0 if unsupported). */
+size_t swa_global_decode_workspace_size(const swa_params_t* p, int64_t cache_cap);
+
+/*
+ * One decode step of a global layer for p->B sequences over their
+ * full-length caches [B, Hkv, cache_cap, D] (as swa_global_fwd writes them):
+ * slot pos[n] receives RoPE_pos(RMSNorm(k_new)) (bf16) and v_new, then q'
+ * attends over slots 0 .. pos[n].  pos: [B] int64 device array (8-byte
+ * aligned), 0 <= pos < cache_cap (else that sequence is skipped and
+ * swa_get_last_device_error returns SWA_ERR_INVALID_ARG); q [B,Hq,D], k_new,
+ * v_new [B,Hkv,D] bf16; writes o [B,Hq,D] bf16.  Slots past pos[n] may hold
+ * anything.  `workspace`: caller-owned device scratch of
+ * swa_global_decode_workspace_size bytes, 256-byte aligned.  Hq / Hkv <= 8
+ * (else SWA_ERR_UNSUPPORTED).  The step reads about 4 KiB of cache per key
+ * position at 8 KV heads: it is memory-bandwidth bound.
+ */
+int swa_global_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
+                           const swa_bf16_t* k_new, const swa_bf16_t* v_new, const float* wq,
+                           const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                           int64_t cache_cap, swa_bf16_t* o, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Static description of an error code. */
 const char* swa_error_string(int code);
 

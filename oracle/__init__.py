@@ -5,7 +5,9 @@ CPU-baseline / reference legs of ``bench.py`` may import this package.  It
 shares no code with the CUDA library and never imports it.
 
 The arithmetic lives in ``swa_oracle.c`` (plain C, IEEE fp64, OpenMP over
-independent rows); this module only marshals numpy arrays.  Definitions follow
+independent rows); this module marshals numpy arrays, and writes two steps
+out in numpy on top of the C norm/RoPE: the prefill -> ring handoff and the
+global layers' decode over a full-length cache.  Definitions follow
 the ZGCM-1 pages: "7.39B 오픈 모델로 256K 문맥의 … ZGCM-1" (onedev.kr), section
 "어떻게 동작하나", and "ZGCM-1: A Fully Open and Extremely Efficient Foundation
 Model …" (jaehun.me), sections "How Gated SWA Behaves" and "Why the KV Cache
@@ -228,6 +230,53 @@ def prefill_to_ring(k, v, wk, k_cache_bits, v_cache_bits, *, R, base, eps):
         kc[:, :, s, :] = bf16_round_array(kp)
         vc[:, :, s, :] = bf16_round_array(v[:, p])
     return kc, vc
+
+
+def global_decode(pos, q, k_new, v_new, wq, wk, k_cache_bits, v_cache_bits, *, R, base, eps,
+                  scale=0.0):
+    """One decode step of a global (full causal context, ungated) layer over
+    full-length caches.
+
+    The global layers attend over every earlier token and keep every token's
+    K and V (onedev.kr summary, "어떻게 동작하나": 5 global layers beside the
+    27 window layers; jaehun.me review, "How Gated SWA Behaves": global layers
+    skip the gate, and "Why the KV Cache Shrinks by 6.4x": they store the whole
+    sequence).  Slot s of a cache holds position s.  For sequence n at position
+    p = pos[n]: slot p first receives k' = RoPE_p(RMSNorm(k_new, wk)) rounded
+    to bf16 and v_new; then q' = RoPE_p(RMSNorm(q, wq)) attends over slots
+    0 .. p (query head h reads KV head h // (Hq / Hkv)): s_j = scale q'.k_j,
+    P = softmax(s), o = sum_j P_j v_j.
+
+    pos [N] int64; q [N, Hq, D], k_new, v_new [N, Hkv, D] (fp64 values of bf16
+    inputs); caches [N, Hkv, cap, D] as uint16 bf16 bits (copied, not
+    modified).  Returns (o [N, Hq, D] fp64, k_cache_bits', v_cache_bits').
+    """
+    pos = np.asarray(pos, dtype=np.int64)
+    q = np.asarray(q, dtype=np.float64)
+    k_new = np.asarray(k_new, dtype=np.float64)
+    v_new = np.asarray(v_new, dtype=np.float64)
+    kc = np.array(k_cache_bits, dtype=np.uint16, copy=True, order="C")
+    vc = np.array(v_cache_bits, dtype=np.uint16, copy=True, order="C")
+    N, Hq, D = q.shape
+    Hkv = kc.shape[1]
+    group = Hq // Hkv
+    sc = _scale(D, scale)
+    o = np.empty_like(q)
+    for n in range(N):
+        p = int(pos[n])
+        at = np.array([float(p)])
+        kp = norm_rope(k_new[n][None], wk, at, R, base, eps)[0]  # [Hkv, D]
+        kc[n, :, p, :] = bf16_round_array(kp)
+        vc[n, :, p, :] = bf16_round_array(v_new[n])
+        qp = norm_rope(q[n][None], wq, at, R, base, eps)[0]      # [Hq, D]
+        for h in range(Hq):
+            kvh = h // group
+            keys = bf16_bits_to_f64(kc[n, kvh, :p + 1])          # slots 0 .. p
+            vals = bf16_bits_to_f64(vc[n, kvh, :p + 1])
+            s = sc * (keys @ qp[h])
+            e = np.exp(s - s.max())
+            o[n, h] = (e / e.sum()) @ vals
+    return o, kc, vc
 
 
 def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, bytes_per_elt: int) -> int:

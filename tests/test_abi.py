@@ -226,3 +226,36 @@ def test_binding_passes_empty_problems_through():
 
 class _NullStream:
     cuda_stream = 0
+
+
+def test_global_layer_host_checks(L):
+    good = ctypes.c_void_p(1 << 20)
+    nul = ctypes.c_void_p(0)
+    i64 = ctypes.c_int64
+    p = _params(B=1, T=256, Hq=8, Hkv=2, window=0)
+
+    def fwd(params, cap, lse=nul, q=good):
+        return L.swa_global_fwd(ctypes.byref(params), q, good, good, good, good, good, lse,
+                                good, good, i64(cap), None)
+    assert fwd(_params(B=1, T=256, Hq=8, Hkv=2), 256) == swa.ERR_INVALID_ARG  # window must be 0
+    assert fwd(p, 255) == swa.ERR_INVALID_ARG                               # cache shorter than T
+    assert fwd(p, 256, q=ctypes.c_void_p((1 << 20) + 8)) == swa.ERR_INVALID_ARG
+    assert fwd(p, 256, lse=ctypes.c_void_p((1 << 20) + 2)) == swa.ERR_INVALID_ARG
+    assert fwd(_params(B=1, T=0, Hq=8, Hkv=2, window=0), 0) == swa.OK
+    assert fwd(_params(B=1, T=256, Hq=8, Hkv=2, window=0, head_dim=64), 256) == swa.ERR_UNSUPPORTED
+
+    pd = _params(B=4, T=1, Hq=8, Hkv=2, window=0)
+    need = L.swa_global_decode_workspace_size(ctypes.byref(pd), i64(5000))
+    assert need >= 4 * 2 * 3 * 4 * 128 * 4   # 3 chunks of 2048 slots x 4 heads x 128 dims fp32
+    assert L.swa_global_decode_workspace_size(ctypes.byref(pd), i64(0)) == 0
+
+    def dec(params, cap, ws_bytes, ws=good, pos=good):
+        # pos, then q, k_new, v_new, wq, wk, k_cache, v_cache
+        return L.swa_global_decode_step(ctypes.byref(params), pos, *([good] * 7), i64(cap), good,
+                                        ws, ws_bytes, None)
+    assert dec(pd, 5000, need - 1) == swa.ERR_INVALID_ARG
+    assert dec(pd, 5000, need, ws=ctypes.c_void_p((1 << 20) + 16)) == swa.ERR_INVALID_ARG
+    assert dec(pd, 5000, need, pos=ctypes.c_void_p((1 << 20) + 4)) == swa.ERR_INVALID_ARG
+    assert dec(_params(B=4, T=1, Hq=32, Hkv=2, window=0), 5000, need) == swa.ERR_UNSUPPORTED
+    assert dec(pd, 0, need) == swa.ERR_INVALID_ARG
+    assert dec(_params(B=0, T=1, Hq=8, Hkv=2, window=0), 5000, 0) == swa.OK

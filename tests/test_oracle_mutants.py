@@ -80,6 +80,16 @@ PY_MUTANTS = [
      [("np.full(B, float(p))", "np.full(B, float(s))")]),
     ("fwd_rows_keys_start_one_late", "fwd_rows",
      [("kb = max(0, t0 - W + 1)", "kb = max(0, t0 - W + 2)")]),
+    ("global_decode_skips_new_key", "global_decode",
+     [("kc[n, kvh, :p + 1]", "kc[n, kvh, :p]"), ("vc[n, kvh, :p + 1]", "vc[n, kvh, :p]")]),
+    ("global_decode_gqa_mapping", "global_decode", [("kvh = h // group", "kvh = h % Hkv")]),
+    ("global_decode_query_position", "global_decode",
+     [("qp = norm_rope(q[n][None], wq, at,", "qp = norm_rope(q[n][None], wq, at + 1,")]),
+    ("global_decode_caches_k_as_v", "global_decode",
+     [("vc[n, :, p, :] = bf16_round_array(v_new[n])",
+       "vc[n, :, p, :] = bf16_round_array(k_new[n])")]),
+    ("global_decode_scale_dropped", "global_decode",
+     [("s = sc * (keys @ qp[h])", "s = keys @ qp[h]")]),
 ]
 
 PINS = (
@@ -99,6 +109,11 @@ PINS = (
        for p in (0, 5, 127, 128, 300)]
     + [(f"prefill_to_ring({T})", pins.test_prefill_to_ring_equals_sequential_decode, (T,))
        for T in (1, 131)]
+    + [("global_decode_dense", pins.test_global_decode_matches_dense_over_cache_contents, ())]
+    + [(f"global_decode_ring({p})", pins.test_global_decode_equals_ring_decode_inside_the_window,
+        (p,)) for p in (0, 77)]
+    + [(f"global_decode_prefill({p})", pins.test_global_decode_equals_causal_prefill_row, (p,))
+       for p in (5, 200)]
 )
 
 
@@ -161,7 +176,8 @@ def test_unmodified_copy_passes_every_pin(tmp_path):
     pass all the pins."""
     with oracle_library(build_variant(tmp_path, [])):
         assert failing_pins(stop_at_first=False) == []
-    with oracle_function("prefill_to_ring", []), oracle_function("fwd_rows", []):
+    with oracle_function("prefill_to_ring", []), oracle_function("fwd_rows", []), \
+            oracle_function("global_decode", []):
         assert failing_pins(stop_at_first=False) == []
 
 

@@ -373,6 +373,90 @@ def test_decode_matches_dense_over_ring_contents():
             np.testing.assert_allclose(o[n, h], ref.numpy(), rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------ global-layer decode
+
+def _global_caches(k, v, wk, p, cap, R, base, eps, rng):
+    """Full-length caches whose slots 0 .. p-1 hold the prefill's bf16 k' and
+    v (positions = slots), the rest noise."""
+    B, Hkv, D = k.shape[0], k.shape[2], k.shape[3]
+    kc = oracle.bf16_round_array(rng.standard_normal((B, Hkv, cap, D)) * 50)
+    vc = oracle.bf16_round_array(rng.standard_normal((B, Hkv, cap, D)) * 50)
+    for t in range(p):
+        kp = oracle.norm_rope(k[:, t], wk, np.full(B, float(t)), R, base, eps)
+        kc[:, :, t] = oracle.bf16_round_array(kp)
+        vc[:, :, t] = oracle.bf16_round_array(v[:, t])
+    return kc, vc
+
+
+def test_global_decode_matches_dense_over_cache_contents():
+    """Global decode = a dense softmax over slots 0 .. p of the cache after
+    the new key is written (brute-force norm/RoPE, torch softmax)."""
+    R, base, eps, Hq, Hkv, D, N, cap = 42, 1e7, 1e-6, 8, 2, 128, 3, 700
+    rng = np.random.default_rng(80)
+    bf = lambda x: oracle.bf16_bits_to_f64(oracle.bf16_round_array(x))
+    q = bf(rng.standard_normal((N, Hq, D)))
+    kn, vn = bf(rng.standard_normal((N, Hkv, D))), bf(rng.standard_normal((N, Hkv, D)))
+    wq, wk = 1 + 0.1 * rng.standard_normal(D), 1 + 0.1 * rng.standard_normal(D)
+    kc = oracle.bf16_round_array(rng.standard_normal((N, Hkv, cap, D)))
+    vc = oracle.bf16_round_array(rng.standard_normal((N, Hkv, cap, D)))
+    pos = np.array([699, 0, 130])
+    o, kc2, vc2 = oracle.global_decode(pos, q, kn, vn, wq, wk, kc, vc, R=R, base=base, eps=eps)
+    for n in range(N):
+        p = int(pos[n])
+        qp = brute_norm_rope(q[n][None, None], wq, np.array([p], float), R, base, eps)[0, 0]
+        kpn = brute_norm_rope(kn[n][None, None], wk, np.array([p], float), R, base, eps)[0, 0]
+        keys = torch.tensor(oracle.bf16_bits_to_f64(kc[n]))
+        vals = torch.tensor(oracle.bf16_bits_to_f64(vc[n]))
+        keys[:, p] = torch.tensor(bf(kpn.numpy()))   # the new token's slot
+        vals[:, p] = torch.tensor(vn[n])
+        for h in range(Hq):
+            s_ = keys[h // (Hq // Hkv), :p + 1] @ qp[h] / math.sqrt(D)
+            ref = torch.softmax(s_, 0) @ vals[h // (Hq // Hkv), :p + 1]
+            np.testing.assert_allclose(o[n, h], ref.numpy(), rtol=0, atol=1e-12)
+        others = [i for i in range(cap) if i != p]
+        assert np.array_equal(kc2[n][:, others], kc[n][:, others])
+        assert np.array_equal(vc2[n][:, others], vc[n][:, others])
+        assert np.array_equal(vc2[n][:, p], oracle.bf16_round_array(vn[n]))
+
+
+@pytest.mark.parametrize("p", [0, 1, 77, 126])
+def test_global_decode_equals_ring_decode_inside_the_window(p):
+    """Below position 127 a 128-slot ring holds exactly slots 0 .. p, so the
+    global decode equals the window layer's decode with the gate open
+    (g = +inf gives sigmoid 1), through the C oracle's own decode."""
+    R, base, eps, Hq, Hkv, D, N, cap = 42, 1e4, 1e-6, 4, 1, 128, 2, 300
+    q, k, v, g, wq, wk = rand_inputs(N, p + 1, Hq, Hkv, D, seed=90 + p)
+    rng = np.random.default_rng(91 + p)
+    kc, vc = _global_caches(k, v, wk, p, cap, R, base, eps, rng)
+    o, kc2, vc2 = oracle.global_decode(np.full(N, p), q[:, p], k[:, p], v[:, p], wq, wk, kc, vc,
+                                       R=R, base=base, eps=eps)
+    ginf = np.full((N, Hq, D), np.inf)
+    o_ring, kr, vr = oracle.decode(np.full(N, p), q[:, p], k[:, p], v[:, p], ginf, wq, wk,
+                                   kc[:, :, :128], vc[:, :, :128], R=R, base=base, eps=eps)
+    np.testing.assert_allclose(o, o_ring, rtol=0, atol=1e-12)
+    assert np.array_equal(kc2[:, :, :128], kr) and np.array_equal(vc2[:, :, :128], vr)
+    if p == 0:  # one key: the output is v_new itself
+        np.testing.assert_allclose(o, np.repeat(v[:, 0], Hq // Hkv, axis=1), rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("p", [5, 200, 600])
+def test_global_decode_equals_causal_prefill_row(p):
+    """Decoding position p over a cache filled by the prefill gives row p of
+    the forward with a window past the sequence (full causal attention,
+    pinned against SDPA above) and the gate open; cached keys are bf16, so
+    the agreement is to bf16 precision."""
+    R, base, eps, Hq, Hkv, D, cap = 42, 1e7, 1e-6, 4, 2, 128, 700
+    q, k, v, g, wq, wk = rand_inputs(1, p + 1, Hq, Hkv, D, seed=100 + p)
+    rng = np.random.default_rng(101 + p)
+    kc, vc = _global_caches(k, v, wk, p, cap, R, base, eps, rng)
+    o_dec, _, _ = oracle.global_decode(np.array([p]), q[:, p], k[:, p], v[:, p], wq, wk, kc, vc,
+                                       R=R, base=base, eps=eps)
+    o_pre, _ = oracle.fwd(q, k, v, np.full_like(g, np.inf), wq, wk, W=p + 10, R=R, base=base,
+                          eps=eps)
+    np.testing.assert_allclose(o_dec[0], o_pre[0, p], rtol=0, atol=2e-2)
+    assert np.abs(o_dec[0] - o_pre[0, p]).mean() < 2e-3
+
+
 # ---------------------------------------------------- rounding and footprint
 
 def test_bf16_rounding_matches_torch_rne():
