@@ -410,7 +410,82 @@ def secondary(swa, args, world, device, stream, peaks):
     out["train_fwd_bwd"] = train_bench(swa, args, world, device, stream, peaks)
     out["decode_step"] = decode_bench(swa, args, world, device, stream, peaks)
     out["prefill_to_ring"] = ring_bench(swa, args, world, device, stream, peaks)
+    out["global_prefill"] = global_prefill_bench(swa, args, world, device, stream, peaks)
+    out["global_decode_step"] = global_decode_bench(swa, args, world, device, stream, peaks)
     return out
+
+
+def global_fwd_flops(c):
+    """QK^T and PV over the causal triangle: 4 D Hq sum_i (i + 1) per sequence."""
+    return 4 * c.D * c.Hq * c.T * (c.T + 1) // 2 * c.B
+
+
+def global_prefill_bench(swa, args, world, device, stream, peaks):
+    """A global layer's causal prefill (swa_global_fwd: cache writer + tcgen05
+    attention) on 1 x 16384, 32 / 8 heads.  Tensor-bound: 2.2e12 band FLOPs
+    against 0.3 GB of traffic."""
+    cfg = workloads.GLOBAL_PREFILL
+    d = workloads.prefill_inputs(cfg, device=device, with_grad_out=False)
+    kc = torch.empty((cfg.B, cfg.Hkv, cfg.T, cfg.D), dtype=torch.bfloat16, device=device)
+    vc = torch.empty_like(kc)
+    o = torch.empty_like(d["q"])
+
+    def step():
+        swa.global_fwd(d["q"], d["k"], d["v"], d["wq"], d["wk"], kc, vc, rot_dim=cfg.R,
+                       rope_base=cfg.base, eps=cfg.eps, out=o)
+    steps = max(3, min(args.steps, 10))
+    ms, _, _, _ = timed_loop([step], steps, 3, stream, world)
+    fl = global_fwd_flops(cfg)
+    tf = fl / (ms / steps / 1e3) / 1e12
+    res = {"workload": cfg.name,
+           "tokens_per_s": round(cfg.B * cfg.T * world / (ms / steps / 1e3), 1),
+           "ms_per_step": round(ms / steps, 4),
+           "algorithmic_flops_per_step": fl,
+           "achieved_TFLOPs": round(tf, 1),
+           "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
+           "frac_of_measured_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+           "bound": "tensor", "launches_per_step": 2}
+    del d, kc, vc, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def global_decode_bench(swa, args, world, device, stream, peaks):
+    """A decode step of the 5 global layers: one swa_global_decode_step per
+    layer over its own [64, 8, 32768, 128] K and V caches (8.6 GB each), at
+    positions uniform in [1, 32768).  HBM-bound: the K and V of positions
+    0 .. pos, plus q, k, v, o rows."""
+    cfg = workloads.GLOBAL_DECODE
+    layers = [workloads.global_decode_layer_inputs(cfg, l, device=device)
+              for l in range(cfg.layers)]
+    outs = [torch.empty_like(x["q"]) for x in layers]
+    ws = torch.empty(swa.global_decode_workspace_size(cfg.N, cfg.Hq, cfg.Hkv, cfg.cap),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        for x, o in zip(layers, outs):
+            swa.global_decode_step(x["pos"], x["q"], x["k"], x["v"], x["wq"], x["wk"],
+                                   x["k_cache"], x["v_cache"], rot_dim=cfg.R, rope_base=cfg.base,
+                                   eps=cfg.eps, out=o, workspace=ws)
+    steps = max(3, min(args.steps, 10))
+    ms, _, _, _ = timed_loop([step], steps, 3, stream, world)
+    kv_row = cfg.Hkv * cfg.D * 2
+    b = 0
+    for x in layers:  # keys 0..pos read from both caches; new k, v written; q read, o written
+        b += int((x["pos"] + 1).sum().item()) * kv_row * 2 + cfg.N * (2 * kv_row + 2 * kv_row
+                                                                     + 2 * cfg.Hq * cfg.D * 2)
+    gbs = b / (ms / steps / 1e3) / 1e9
+    res = {"workload": cfg.name,
+           "tokens_per_s": round(cfg.N * world / (ms / steps / 1e3), 1),
+           "ms_per_step": round(ms / steps, 4),
+           "algorithmic_bytes_per_step": b,
+           "achieved_GBps": round(gbs, 1),
+           "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4),
+           "launches_per_step": 3 * cfg.layers,
+           "note": "positions fixed across steps: each step rewrites the same cache slots"}
+    del layers, outs, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def train_bench(swa, args, world, device, stream, peaks):
@@ -528,7 +603,8 @@ def run_profile(args, device):
     profiler sees a short, predictable launch list: `fwd` on the layer-shape
     workload, `decode` on one layer of the decode workload, `bwd` (with the
     forward that produces its lse) on the training shape, `ring` on the
-    prefill -> ring handoff of the decode batch."""
+    prefill -> ring handoff of the decode batch, `gfwd` on the global-layer
+    prefill, `gdec` on 16 sequences of one global layer's decode."""
     import hybrid_sliding_window_gated_b200 as swa
     which = args.profile
     if which == "fwd":
@@ -541,6 +617,22 @@ def run_profile(args, device):
         fns = [lambda: swa.decode_step(x["pos"], x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"],
                                        x["k_cache"], x["v_cache"], rot_dim=cfg.R,
                                        rope_base=cfg.base, eps=cfg.eps, out=o)]
+    elif which == "gfwd":
+        cfg = workloads.GLOBAL_PREFILL
+        d = workloads.prefill_inputs(cfg, device=device, with_grad_out=False)
+        kc = torch.empty((cfg.B, cfg.Hkv, cfg.T, cfg.D), dtype=torch.bfloat16, device=device)
+        vc = torch.empty_like(kc)
+        fns = [lambda: swa.global_fwd(d["q"], d["k"], d["v"], d["wq"], d["wk"], kc, vc,
+                                      rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps)]
+    elif which == "gdec":
+        # 16 of the 64 sequences (2.1 GB of caches), so a full capture stays small
+        cfg = workloads.GLOBAL_DECODE
+        x = workloads.global_decode_layer_inputs(cfg, 0, device=device)
+        x = {k: (v[:16].contiguous() if v.dim() > 1 or k == "pos" else v) for k, v in x.items()}
+        o = torch.empty_like(x["q"])
+        fns = [lambda: swa.global_decode_step(x["pos"], x["q"], x["k"], x["v"], x["wq"], x["wk"],
+                                              x["k_cache"], x["v_cache"], rot_dim=cfg.R,
+                                              rope_base=cfg.base, eps=cfg.eps, out=o)]
     elif which == "ring":
         cfg = workloads.custom_prefill(256, 256, 32, 8, base=1e7, seed=7)
         gen = torch.Generator(device="cpu").manual_seed(7)
@@ -608,7 +700,8 @@ def main():
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "decode", "bwd", "ring"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "decode", "bwd", "ring", "gfwd", "gdec"],
+                    default=None,
                     help="only warmup + steps calls of one entry point (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:

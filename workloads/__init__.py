@@ -13,6 +13,9 @@ not used here; these synthetic tensors stand in for it):
     for the training shape.
   * Decode: both rings ~N(0,1) (bf16), new q, k, v, g ~N(0,1), positions
     uniform in [128, 262144), drawn after the rings.
+  * Global layers: the prefill draws q, k, v as above (its g is unused); the
+    decode draws [N, Hkv, cap, D] caches ~N(0,1), then q, k, v, the norm
+    weights and positions uniform in [1, cap).
 """
 from dataclasses import dataclass, field
 
@@ -75,6 +78,49 @@ DECODE = Decode("decode step, 256 sequences x 27 gated-SWA layers, 128-slot ring
                 layers=27, Hq=32, Hkv=8, base=1e7, seed=4)
 
 PREFILL_CONFIGS = {"tiny": TINY, "layer": LAYER, "train": TRAIN, "long": LONG}
+
+# The global causal layers (5 of the 32): no window and no gate, so only q, k
+# and v are drawn (g and the gate's std unused).
+GLOBAL_PREFILL = Prefill("global-layer causal prefill 1x16384, 32q/8kv", B=1, T=16384, Hq=32,
+                         Hkv=8, base=1e4, g_std=1.0, seed=6)
+
+
+@dataclass(frozen=True)
+class GlobalDecode:
+    name: str
+    N: int
+    layers: int
+    Hq: int
+    Hkv: int
+    cap: int
+    base: float
+    seed: int
+    D: int = HEAD_DIM
+    R: int = ROT_DIM
+    eps: float = EPS
+
+
+GLOBAL_DECODE = GlobalDecode("global-layer decode step, 64 sequences x 5 layers, 32K-slot caches",
+                             N=64, layers=5, Hq=32, Hkv=8, cap=32768, base=1e7, seed=7)
+
+
+def global_decode_layer_inputs(cfg: GlobalDecode, layer: int, device="cpu"):
+    """One global layer's decode inputs: [N, Hkv, cap, D] K and V caches ~N(0,1),
+    new q, k, v ~N(0,1), norm weights, positions uniform in [1, cap)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg.seed * 1000 + layer)
+    N, Hq, Hkv, D = cfg.N, cfg.Hq, cfg.Hkv, cfg.D
+    out = {
+        "k_cache": _randn((N, Hkv, cfg.cap, D), gen, device),
+        "v_cache": _randn((N, Hkv, cfg.cap, D), gen, device),
+        "q": _randn((N, Hq, D), gen, device),
+        "k": _randn((N, Hkv, D), gen, device),
+        "v": _randn((N, Hkv, D), gen, device),
+    }
+    out["wq"] = 1.0 + 0.1 * torch.randn((D,), generator=gen, device=device)
+    out["wk"] = 1.0 + 0.1 * torch.randn((D,), generator=gen, device=device)
+    out["pos"] = torch.randint(1, cfg.cap, (N,), generator=gen, device=device, dtype=torch.int64)
+    return out
 
 
 def _randn(shape, gen, device, std=1.0):
