@@ -410,9 +410,44 @@ def secondary(swa, args, world, device, stream, peaks):
     out["train_fwd_bwd"] = train_bench(swa, args, world, device, stream, peaks)
     out["decode_step"] = decode_bench(swa, args, world, device, stream, peaks)
     out["prefill_to_ring"] = ring_bench(swa, args, world, device, stream, peaks)
+    out["fp8_fwd"] = fp8_fwd_bench(swa, args, world, device, stream, peaks)
     out["global_prefill"] = global_prefill_bench(swa, args, world, device, stream, peaks)
     out["global_decode_step"] = global_decode_bench(swa, args, world, device, stream, peaks)
     return out
+
+
+def FP8_FWD_BYTES_PER_TOKEN(c):
+    """The forward with E4M3 q, k, v: one byte each for q, k, v; g and o bf16."""
+    return (c.Hq + 2 * c.Hkv) * c.D + 2 * c.Hq * c.D * 2
+
+
+def fp8_fwd_bench(swa, args, world, device, stream, peaks):
+    """swa_fwd_fp8 on the layer shape (4 x 4096): q, k, v in E4M3 with one factor
+    each; two rotating input sets (> L2)."""
+    cfg = workloads.LAYER
+    sets = []
+    for s in range(2):
+        x = workloads.fp8_prefill_inputs(cfg, device=device, seed=cfg.seed + 100 * s)
+        x["o"] = torch.empty(x["g"].shape, dtype=torch.bfloat16, device=device)
+        sets.append(x)
+
+    def mk(x):
+        return lambda: swa.fwd_fp8(x["q8"], x["k8"], x["v8"], x["qkv_scale"], x["g"], x["wq"],
+                                   x["wk"], rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps,
+                                   out=x["o"])
+    steps = max(5, min(args.steps, 20))
+    ms, _, _, _ = timed_loop([mk(x) for x in sets], steps, 3, stream, world)
+    b = FP8_FWD_BYTES_PER_TOKEN(cfg) * cfg.B * cfg.T
+    gbs = b / (ms / steps / 1e3) / 1e9
+    res = {"workload": cfg.name + ", q/k/v in FP8 E4M3",
+           "tokens_per_s": round(cfg.B * cfg.T * world / (ms / steps / 1e3), 1),
+           "ms_per_step": round(ms / steps, 5),
+           "algorithmic_bytes_per_step": b,
+           "achieved_GBps": round(gbs, 1),
+           "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    del sets
+    torch.cuda.empty_cache()
+    return res
 
 
 def global_fwd_flops(c):

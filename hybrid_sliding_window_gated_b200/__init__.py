@@ -16,7 +16,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
+__all__ = ["fwd", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
            "global_fwd", "global_decode_step", "global_decode_workspace_size",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
@@ -55,6 +55,8 @@ def lib():
         P = ctypes.POINTER(Params)
         L.swa_fwd.argtypes = [P] + [_vp] * 9
         L.swa_fwd.restype = ctypes.c_int
+        L.swa_fwd_fp8.argtypes = [P] + [_vp] * 10
+        L.swa_fwd_fp8.restype = ctypes.c_int
         L.swa_bwd.argtypes = [P] + [_vp] * 15 + [ctypes.c_size_t, _vp]
         L.swa_bwd.restype = ctypes.c_int
         L.swa_bwd_edges.argtypes = [P] + [_vp] * 14 + [ctypes.c_int64, _vp, ctypes.c_int64, _vp,
@@ -150,6 +152,34 @@ def fwd(q, k, v, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6, 
     rc = lib().swa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
                        _ptr(out), _ptr(lse), _stream(stream))
     _check(rc, "swa_fwd")
+    return (out, lse) if lse is not None else out
+
+
+def fwd_fp8(q8, k8, v8, qkv_scale, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4,
+            eps=1e-6, scale=0.0, out=None, lse=None, want_lse=False, flags=0, stream=None):
+    """:func:`fwd` with q, k, v in FP8 E4M3 (swa_fwd_fp8): q8 [B,T,Hq,128], k8,
+    v8 [B,T,Hkv,128] as torch.float8_e4m3fn or uint8 bytes; qkv_scale [3] fp32
+    (CUDA) with the values q = q8 * qkv_scale[0], k = k8 * qkv_scale[1],
+    v = v8 * qkv_scale[2]; g, wq, wk as in :func:`fwd`."""
+    B, T, Hq, D = q8.shape
+    Hkv = k8.shape[2]
+    if out is None:
+        out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q8.device)
+    byte = lambda t: t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+    q8, k8, v8 = byte(q8), byte(k8), byte(v8)
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale, flags=flags)
+    nq, nk = B * T * Hq * D, B * T * Hkv * D
+    bf, f32, u8 = torch.bfloat16, torch.float32, torch.uint8
+    opt = {} if lse is None else {"lse": (lse, f32, B * Hq * T)}
+    _need("swa_fwd_fp8", q8.device, q=(q8, u8, nq), k=(k8, u8, nk), v=(v8, u8, nk),
+          qkv_scale=(qkv_scale, f32, 3 if nq else 0), g=(g, bf, nq),
+          wq=(wq, f32, D if nq else 0), wk=(wk, f32, D if nq else 0), out=(out, bf, nq), **opt)
+    rc = lib().swa_fwd_fp8(ctypes.byref(p), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qkv_scale),
+                           _ptr(g), _ptr(wq), _ptr(wk), _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc, "swa_fwd_fp8")
     return (out, lse) if lse is not None else out
 
 

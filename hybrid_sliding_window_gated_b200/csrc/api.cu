@@ -84,7 +84,7 @@ int device_error_word(int** ptr) {
 
 int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                    uint64_t d3, uint32_t box0, uint32_t box1, uint32_t box2, uint32_t box3,
-                   CUtensorMapSwizzle swizzle) {
+                   CUtensorMapSwizzle swizzle, bool bytes) {
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (g_encode == nullptr) {
@@ -98,10 +98,12 @@ int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
     }
   }
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};  // bytes, dims 1..3
+  const cuuint64_t eb = bytes ? 1 : 2;
+  const cuuint64_t strides[3] = {d0 * eb, d0 * d1 * eb, d0 * d1 * d2 * eb};  // bytes, dims 1..3
   const cuuint32_t box[4] = {box0, box1, box2, box3};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = g_encode(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        4, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SWA_OK : SWA_ERR_CUDA;
@@ -146,6 +148,60 @@ static void fill_inv_freq(const swa_params_t* p, double* out) {
 
 }  // namespace swa
 
+namespace swa {
+
+// swa_fwd, and swa_fwd_fp8 when qkv_scale is set (q, k, v then point at E4M3 bytes).
+static int fwd_impl(const swa_params_t* p, const void* q, const void* k, const void* v,
+                    const float* qkv_scale, const swa_bf16_t* g, const float* wq, const float* wk,
+                    swa_bf16_t* o, float* lse, void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  if (p->B == 0 || p->T == 0) return SWA_OK;
+  if (!q || !k || !v || !g || !wq || !wk || !o) return SWA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o) ||
+      !aligned16(wq) || !aligned16(wk) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+
+  FwdArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.tiles_per_chain = static_cast<int>((p->T + kTile - 1) / kTile);
+  a.total_tiles = static_cast<long long>(a.tiles_per_chain) * p->B * p->Hkv;
+  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
+  a.eps = p->eps;
+  a.flags = p->flags;
+  a.wq = wq;
+  a.wk = wk;
+  a.qkv_scale = qkv_scale;
+  a.g = g;
+  a.o = o;
+  a.lse = lse;
+  rc = device_error_word(&a.err);
+  if (rc != SWA_OK) return rc;
+  fill_inv_freq(p, a.inv_freq);
+
+  // Every bf16 tensor moves in boxes of 128 rows x 64 dims (128-byte rows,
+  // 128B swizzle): the MMA operand layout for q, k, v, and the same layout for
+  // the gate and output tiles that pass through a Q slot.  FP8 q, k, v move
+  // in boxes of 128 rows x 128 one-byte dims, expanded in shared memory.
+  CUtensorMap tq, tk, tv, tg, to;
+  const uint64_t D = kHeadDim, T = p->T, B = p->B;
+  const bool f8 = qkv_scale != nullptr;
+  const uint32_t bx = f8 ? 128 : 64;
+  if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, bx, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B, f8)) ||
+      (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, bx, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B, f8)) ||
+      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, bx, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B, f8)) ||
+      (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (rc = encode_tmap_4d(&to, o, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  return launch_fwd(p, tq, tk, tv, tg, to, a, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace swa
+
 using namespace swa;
 
 extern "C" {
@@ -182,46 +238,16 @@ int swa_get_last_device_error(void* stream, int* site) {
 int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
             const swa_bf16_t* g, const float* wq, const float* wk, swa_bf16_t* o, float* lse,
             void* stream) {
-  int rc = check_params(p, false);
-  if (rc != SWA_OK) return rc;
-  if (p->B == 0 || p->T == 0) return SWA_OK;
-  if (!q || !k || !v || !g || !wq || !wk || !o) return SWA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o) ||
-      !aligned16(wq) || !aligned16(wk) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+  return fwd_impl(p, q, k, v, nullptr, g, wq, wk, o, lse, stream);
+}
+
+int swa_fwd_fp8(const swa_params_t* p, const uint8_t* q, const uint8_t* k, const uint8_t* v,
+                const float* qkv_scale, const swa_bf16_t* g, const float* wq, const float* wk,
+                swa_bf16_t* o, float* lse, void* stream) {
+  if (p != nullptr && p->B > 0 && p->T > 0 &&
+      (qkv_scale == nullptr || (reinterpret_cast<uintptr_t>(qkv_scale) & 3u)))
     return SWA_ERR_INVALID_ARG;
-
-  FwdArgs a{};
-  a.B = static_cast<int>(p->B);
-  a.T = static_cast<int>(p->T);
-  a.Hq = p->Hq;
-  a.Hkv = p->Hkv;
-  a.G = p->Hq / p->Hkv;
-  a.tiles_per_chain = static_cast<int>((p->T + kTile - 1) / kTile);
-  a.total_tiles = static_cast<long long>(a.tiles_per_chain) * p->B * p->Hkv;
-  a.scale_log2 = score_scale(p) * 1.4426950408889634f;
-  a.eps = p->eps;
-  a.flags = p->flags;
-  a.wq = wq;
-  a.wk = wk;
-  a.g = g;
-  a.o = o;
-  a.lse = lse;
-  rc = device_error_word(&a.err);
-  if (rc != SWA_OK) return rc;
-  fill_inv_freq(p, a.inv_freq);
-
-  // Every tensor moves in boxes of 128 rows x 64 dims (128-byte rows, 128B
-  // swizzle): the MMA operand layout for q, k, v, and the same layout for the
-  // gate and output tiles that pass through a Q slot.
-  CUtensorMap tq, tk, tv, tg, to;
-  const uint64_t D = kHeadDim, T = p->T, B = p->B;
-  if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&to, o, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)))
-    return rc;
-  return launch_fwd(p, tq, tk, tv, tg, to, a, static_cast<cudaStream_t>(stream));
+  return fwd_impl(p, q, k, v, qkv_scale, g, wq, wk, o, lse, stream);
 }
 
 }  // extern "C"

@@ -72,6 +72,8 @@
 // instructions are refetched all the time; when they miss the instruction
 // cache, every SM fetches from L2 while L2 is busiest.  The chunk loops of the
 // softmax and the epilogue therefore stay rolled, with one register buffer.
+#include <cuda_fp8.h>
+
 #include "launch.cuh"
 #include "ptx.cuh"
 #include "swa_internal.h"
@@ -98,8 +100,9 @@ struct alignas(1024) Smem {
   float2 rot_tile[2][kMaxPairs];  // rot(128 j * w_p) of the K tile in each slot
   float wq[kHeadDim];
   float wk[kHeadDim];
+  float sc[3];  // FP8 inputs: dequantisation factors of q, k, v
   uint64_t kfull[2], kready[2], kempty[2];
-  uint64_t vfull[2], vempty[2];
+  uint64_t vfull[2], vempty[2], vready[2];  // vready: FP8 V expanded to bf16
   uint64_t qfull[3], qready[2];
   uint64_t sfull[2], pfull[2], ofull[2], tfree[2];
   uint64_t gfull[3], ostore[2];  // gate tile landed (per slot) / o written (per region)
@@ -294,6 +297,157 @@ __device__ __forceinline__ float transform_q_row(uint8_t* tile, int row, const S
   return rinv;
 }
 
+// ------------------------------------------------------- FP8 (E4M3) inputs
+//
+// An FP8 tile (128 rows x 128 one-byte dims, 128B-swizzled in 16-byte chunks
+// of 16 dims) is loaded by TMA into the upper half of its 32 KiB slot.  Each
+// thread expands its own row into the slot's two bf16 halves: it reads the
+// whole 128-byte row first, so writing half 1 (the same bytes) is safe.
+// Every E4M3 value is exact in bf16, and the per-tensor factor s (x = e4m3 *
+// s) folds into per-row factors, so the operands carry no rounding that the
+// bf16 path does not.
+
+// Dims 16 c .. 16 c + 15 of an FP8 row, exactly, as floats.
+__device__ __forceinline__ void e4m3x16_to_f32(const uint4& u, float (&x)[16]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * h)), __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r));
+      x[4 * i + 2 * h] = f.x;
+      x[4 * i + 2 * h + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void load_row_fp8(const uint8_t* tile, int row, uint4 (&u)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    u[c] = *reinterpret_cast<const uint4*>(tile + kHalfBytes + sw_off(row, c));
+}
+
+__device__ __forceinline__ float row_sumsq_fp8(const uint4 (&u)[8]) {
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float x[16];
+    e4m3x16_to_f32(u[c], x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = make_float2(x[2 * i], x[2 * i + 1]);
+      acc[i & 1] = __ffma2_rn(f, f, acc[i & 1]);
+    }
+  }
+  const float2 s2 = __fadd2_rn(acc[0], acc[1]);
+  return s2.x + s2.y;
+}
+
+// Write dims [64 h, 64 h + 64) of a row, given as floats, as bf16 half h.
+__device__ __forceinline__ void store_half_bf16(uint8_t* tile, int row, int h, const float* x) {
+  uint8_t* hp = tile + h * kHalfBytes;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(hp + sw_off(row, c)) = pack8(x + 8 * c);
+}
+
+// The factor that takes an FP8 row x8 to RMSNorm's x / rms(x) for x = s x8:
+// s / sqrt(s^2 mean(x8^2) + eps).
+__device__ __forceinline__ float fp8_row_factor(float sumsq8, float s, float eps) {
+  return s * rsqrtf(s * s * sumsq8 * (1.0f / kHeadDim) + eps);
+}
+
+// K row from FP8: k'' as transform_k_row writes it, from x8 and the factor.
+template <int kPairs>
+__device__ __forceinline__ void transform_k_row_fp8(uint8_t* tile, int row, const Smem& sm,
+                                                    int kslot, const RowRot<kPairs>& rr,
+                                                    float eps) {
+  uint4 u[8];
+  load_row_fp8(tile, row, u);
+  const float f = fp8_row_factor(row_sumsq_fp8(u), sm.sc[1], eps);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float y[16];
+      e4m3x16_to_f32(u[4 * h + c], y);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int d = 64 * h + 16 * c + i;
+        x[16 * c + i] = d < 2 * kPairs ? y[i] * f * sm.wk[d] : y[i] * f * sm.wk[d] * sm.wq[d];
+      }
+    }
+    if (h == 0) {
+#pragma unroll
+      for (int p = 0; p < kPairs; ++p) {
+        const float2 t = cmul(sm.rot_tile[kslot][p], rr.r[p]);
+        const float a0 = x[p], b0 = x[p + kPairs];
+        x[p] = a0 * t.x - b0 * t.y;
+        x[p + kPairs] = b0 * t.x + a0 * t.y;
+      }
+    }
+    store_half_bf16(tile, row, h, x);
+  }
+}
+
+// Q row from FP8: q'' = [RoPE(x8 * wq) on the rotated dims; x8 elsewhere],
+// both exact in bf16 but for the rotation; returns the row's factor, which
+// the softmax applies in place of 1/rms(q).
+template <int kPairs>
+__device__ __forceinline__ float transform_q_row_fp8(uint8_t* tile, int row, const Smem& sm,
+                                                     int kslot, const RowRot<kPairs>& rr,
+                                                     float eps) {
+  uint4 u[8];
+  load_row_fp8(tile, row, u);
+  const float f = fp8_row_factor(row_sumsq_fp8(u), sm.sc[0], eps);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float y[16];
+      e4m3x16_to_f32(u[4 * h + c], y);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int d = 64 * h + 16 * c + i;
+        x[16 * c + i] = d < 2 * kPairs ? y[i] * sm.wq[d] : y[i];
+      }
+    }
+    if (h == 0) {
+#pragma unroll
+      for (int p = 0; p < kPairs; ++p) {
+        const float2 t = cmul(sm.rot_tile[kslot][p], rr.r[p]);
+        const float a0 = x[p], b0 = x[p + kPairs];
+        x[p] = a0 * t.x - b0 * t.y;
+        x[p + kPairs] = b0 * t.x + a0 * t.y;
+      }
+    }
+    store_half_bf16(tile, row, h, x);
+  }
+  return f;
+}
+
+// V row from FP8: x8 exactly as bf16 (the factor s_v enters with 1/l).
+__device__ __forceinline__ void expand_v_row_fp8(uint8_t* tile, int row) {
+  uint4 u[8];
+  load_row_fp8(tile, row, u);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float y[16];
+      e4m3x16_to_f32(u[4 * h + c], y);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[16 * c + i] = y[i];
+    }
+    store_half_bf16(tile, row, h, x);
+  }
+}
+
 // K-major operand descriptor for k-step kk (16 elements) of a 128 x 128 tile.
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
   return make_desc_sw128(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
@@ -318,7 +472,7 @@ struct Ring {
   }
 };
 
-template <int kPairs>
+template <int kPairs, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -345,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kempty[i], 1);
       mbar_init(&sm.vfull[i], 1);
       mbar_init(&sm.vempty[i], 1);
+      mbar_init(&sm.vready[i], 128);
       mbar_init(&sm.qready[i], 128);
       mbar_init(&sm.sfull[i], 1);
       mbar_init(&sm.pfull[i], 128);
@@ -383,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.wq[tid] = wq;
     sm.wk[tid] = wk;
   }
+  if (tid < 3) sm.sc[tid] = kFp8 ? a.qkv_scale[tid] : 1.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -405,9 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j & 1;
         if (kr.was_used(s) && !wait0(&sm.kempty[s], kr.parity(s) ^ 1u, kSiteKEmpty)) return false;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.kfull[s], kTileBytes);
-          tma_load_4d(sm.k[s], &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
-          tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 64, c.kvh, j * kTile, c.b);
+          if (kFp8) {  // one 16 KiB box of bytes, into the slot's upper half
+            mbar_arrive_expect_tx(&sm.kfull[s], kHalfBytes);
+            tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
+          } else {
+            mbar_arrive_expect_tx(&sm.kfull[s], kTileBytes);
+            tma_load_4d(sm.k[s], &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
+            tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 64, c.kvh, j * kTile, c.b);
+          }
         }
         // rot(128 j w_p) for this tile, then the second arrive on kfull.
         if (lane < kPairs) {
@@ -435,9 +596,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) {
             const int hq = c.kvh * a.G + h;
-            mbar_arrive_expect_tx(&sm.qfull[qs], kTileBytes);
-            tma_load_4d(sm.q[qs], &tm_q, &sm.qfull[qs], 0, hq, c.t * kTile, c.b);
-            tma_load_4d(sm.q[qs] + kHalfBytes, &tm_q, &sm.qfull[qs], 64, hq, c.t * kTile, c.b);
+            if (kFp8) {
+              mbar_arrive_expect_tx(&sm.qfull[qs], kHalfBytes);
+              tma_load_4d(sm.q[qs] + kHalfBytes, &tm_q, &sm.qfull[qs], 0, hq, c.t * kTile, c.b);
+            } else {
+              mbar_arrive_expect_tx(&sm.qfull[qs], kTileBytes);
+              tma_load_4d(sm.q[qs], &tm_q, &sm.qfull[qs], 0, hq, c.t * kTile, c.b);
+              tma_load_4d(sm.q[qs] + kHalfBytes, &tm_q, &sm.qfull[qs], 64, hq, c.t * kTile, c.b);
+            }
             tma_prefetch_4d(&tm_g, 0, hq, c.t * kTile, c.b);  // warm L2 for the gate tile
             tma_prefetch_4d(&tm_g, 64, hq, c.t * kTile, c.b);
           }
@@ -466,9 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (vr.was_used(s) &&
               !(ok = mbar_wait_inl(&sm.vempty[s], vr.parity(s) ^ 1u, abort, a.err, kSiteVEmpty)))
             break;
-          mbar_arrive_expect_tx(&sm.vfull[s], kTileBytes);
-          tma_load_4d(sm.v[s], &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
-          tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 64, c.kvh, j * kTile, c.b);
+          if (kFp8) {
+            mbar_arrive_expect_tx(&sm.vfull[s], kHalfBytes);
+            tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
+          } else {
+            mbar_arrive_expect_tx(&sm.vfull[s], kTileBytes);
+            tma_load_4d(sm.v[s], &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
+            tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 64, c.kvh, j * kTile, c.b);
+          }
           vr.advance(s);
         }
       }
@@ -519,11 +690,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t cnt = static_cast<uint32_t>(m >> 1);
           const int sp = (cp.t + 1) & 1, sc = cp.t & 1;
           if (cp.h == 0) {
+            // FP8 V is read once a region warpgroup has expanded it to bf16
+            uint64_t* vb = kFp8 ? sm.vready : sm.vfull;
             if (need_prev(cp)) {
-              if (!mbar_wait_inl(&sm.vfull[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
+              if (!mbar_wait_inl(&vb[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
               vr.advance(sp);
             }
-            if (!mbar_wait_inl(&sm.vfull[sc], vr.parity(sc), abort, a.err, kSiteVFull)) { ok = false; break; }
+            if (!mbar_wait_inl(&vb[sc], vr.parity(sc), abort, a.err, kSiteVFull)) { ok = false; break; }
             vr.advance(sc);
           }
           if (!mbar_wait_inl(&sm.pfull[r], cnt & 1, abort, a.err, kSitePFull)) { ok = false; break; }
@@ -596,9 +769,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = j & 1;
           if (transform_last && acct == upto) {
             if (!mbar_wait_inl(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
-            transform_k_row<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
+            if constexpr (kFp8)
+              transform_k_row_fp8<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
+            else
+              transform_k_row<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
             fence_proxy_async_smem();
             mbar_arrive(&sm.kready[s]);
+            if constexpr (kFp8) {  // V of the same tile (vfull has the K ring's phase)
+              if (!mbar_wait_inl(&sm.vfull[s], kr.parity(s), abort, a.err, kSiteVFull)) return false;
+              expand_v_row_fp8(sm.v[s], row);
+              fence_proxy_async_smem();
+              mbar_arrive(&sm.vready[s]);
+            }
           } else if (acct == upto && j == kc.t) {
             // The Q rows of this tile use its rotation table, which the
             // producer publishes with kfull.  The slot cannot be refilled
@@ -635,7 +817,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // after every QK^T of tile t+1.
       if (!account(c.u, c.h == 0)) { ok = false; break; }
       if (!mbar_wait_inl(&sm.qfull[qs], qph, abort, a.err, kSiteQFull)) { ok = false; break; }
-      const float rinv = transform_q_row<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
+      float rinv;
+      if constexpr (kFp8)
+        rinv = transform_q_row_fp8<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
+      else
+        rinv = transform_q_row<kPairs>(sm.q[qs], row, sm, c.t & 1, rr, a.eps);
       fence_proxy_async_smem();
       mbar_arrive(&sm.qready[r]);
 
@@ -755,7 +941,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_inl(&sm.ofull[r], cnt & 1, abort, a.err, kSiteOFull)) { ok = false; break; }
       if (!mbar_wait_inl(&sm.gfull[qs], qph, abort, a.err, kSiteGFull)) { ok = false; break; }
       tc_fence_after();
-      const float2 il2 = make_float2(1.0f / l, 1.0f / l);
+      const float il = sm.sc[2] / l;  // FP8 V: its factor s_v enters here
+      const float2 il2 = make_float2(il, il);
       {
         // Chunk ch: 32 columns of O, written over the same columns of g.
         auto gate = [&](const uint32_t(&ov)[32], int ch) {
@@ -826,7 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kPairs>
+template <int kPairs, bool kFp8>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
                 cudaStream_t stream) {
@@ -838,17 +1025,30 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
     // The register split (setmaxnreg) assumes the kernel was built with the
     // full launch budget per thread; refuse to launch otherwise.
     cudaFuncAttributes attr;
-    cudaError_t e = cudaFuncGetAttributes(&attr, swa_fwd_kernel<kPairs>);
+    cudaError_t e = cudaFuncGetAttributes(&attr, swa_fwd_kernel<kPairs, kFp8>);
     if (e != cudaSuccess) return map_cuda_error(e);
     if (attr.numRegs != kRegsLaunch) return SWA_ERR_UNSUPPORTED;
-    e = cudaFuncSetAttribute(swa_fwd_kernel<kPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = cudaFuncSetAttribute(swa_fwd_kernel<kPairs, kFp8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return map_cuda_error(e);
     configured_device = dev;
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
-  return launch_dependent(swa_fwd_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem,
-                          stream, tq, tk, tv, tg, to, a);
+  return launch_dependent(swa_fwd_kernel<kPairs, kFp8>, static_cast<unsigned>(grid), kThreads,
+                          smem, stream, tq, tk, tv, tg, to, a);
+}
+
+template <bool kFp8>
+int launch_rot(int rot_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
+               cudaStream_t stream) {
+  switch (rot_dim) {
+    case 0: return launch_impl<0, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
+    case 32: return launch_impl<16, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
+    case 42: return launch_impl<21, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
+    case 48: return launch_impl<24, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
+    default: return SWA_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace fwd
@@ -860,13 +1060,9 @@ int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& 
   int rc = current_device_info(&di);
   if (rc != SWA_OK) return rc;
   if (a.total_tiles > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
-  switch (p->rot_dim) {
-    case 0: return fwd::launch_impl<0>(tq, tk, tv, tg, to, a, di.num_sms, stream);
-    case 32: return fwd::launch_impl<16>(tq, tk, tv, tg, to, a, di.num_sms, stream);
-    case 42: return fwd::launch_impl<21>(tq, tk, tv, tg, to, a, di.num_sms, stream);
-    case 48: return fwd::launch_impl<24>(tq, tk, tv, tg, to, a, di.num_sms, stream);
-    default: return SWA_ERR_UNSUPPORTED;
-  }
+  return a.qkv_scale != nullptr
+             ? fwd::launch_rot<true>(p->rot_dim, tq, tk, tv, tg, to, a, di.num_sms, stream)
+             : fwd::launch_rot<false>(p->rot_dim, tq, tk, tv, tg, to, a, di.num_sms, stream);
 }
 
 }  // namespace swa

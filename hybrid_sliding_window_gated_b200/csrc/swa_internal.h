@@ -22,6 +22,7 @@ struct FwdArgs {
   int flags;         // SWA_FLAG_* debug bits (0 in normal use)
   const float* wq;
   const float* wk;
+  const float* qkv_scale;  // FP8 (E4M3) q, k, v: their dequantisation factors; null for bf16
   const uint16_t* g;
   uint16_t* o;
   float* lse;
@@ -37,10 +38,11 @@ struct DeviceInfo {
 // Current device and its SM count (cached per device).
 int current_device_info(DeviceInfo* info);
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// cuTensorMapEncodeTiled through the runtime's driver entry point: bf16
+// elements, or single bytes when `bytes` is set.
 int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                    uint64_t d3, uint32_t box0, uint32_t box1, uint32_t box2, uint32_t box3,
-                   CUtensorMapSwizzle swizzle);
+                   CUtensorMapSwizzle swizzle, bool bytes = false);
 
 int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, const CUtensorMap& tg, const CUtensorMap& to,

@@ -101,6 +101,24 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
             swa_bf16_t* o, float* lse, void* stream);
 
 /*
+ * swa_fwd with q, k and v in FP8 E4M3 (one byte per element, the OCP E4M3
+ * encoding: bias 7, no infinities), each with one fp32 dequantisation factor:
+ * the values are q = q8 * qkv_scale[0], k = k8 * qkv_scale[1], v = v8 *
+ * qkv_scale[2].  qkv_scale is a [3] fp32 DEVICE array (4-byte aligned), so a
+ * caller that keeps delayed-scaling factors on the device passes them as
+ * they are.  q, k, v: [B,T,H,D] bytes, 16-byte aligned; g, wq, wk, o, lse as
+ * in swa_fwd.  Every E4M3 value is exact in bf16, and the factors fold into
+ * per-row factors, so the result has the accuracy of swa_fwd on the
+ * dequantised inputs; q, k, v move at half the bytes.  Source: the training
+ * recipe's FP8 forward (onedev.kr summary, "무엇과 다른가": Transformer Engine
+ * hybrid FP8, E4M3 forward); one factor per tensor is what delayed scaling
+ * keeps.
+ */
+int swa_fwd_fp8(const swa_params_t* p, const uint8_t* q, const uint8_t* k, const uint8_t* v,
+                const float* qkv_scale, const swa_bf16_t* g, const float* wq, const float* wk,
+                swa_bf16_t* o, float* lse, void* stream);
+
+/*
  * Backward of swa_fwd given the upstream gradient dO [B,T,Hq,D] and the lse
  * that swa_fwd wrote.  Writes dq, dg [B,T,Hq,D] and dk, dv [B,T,Hkv,D]
  * (bf16) and ADDS the weight gradients into dwq, dwk [D] (fp32; the caller

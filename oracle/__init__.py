@@ -96,6 +96,19 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
+def e4m3_to_f64(b):
+    """Values of FP8 E4M3 bytes (the OCP 8-bit format with 4 exponent bits, bias
+    7, and 3 mantissa bits; no infinities, S.1111.111 is NaN), from the
+    encoding's definition: normal (1 + m/8) 2^(e-7), subnormal m 2^-9."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
 def norm_rope(x, w, pos, R, base, eps):
     """RoPE(RMSNorm(x, w), pos) for x [rows, H, D] (fp64), pos [rows]."""
     x, px = _f64(x)

@@ -457,6 +457,22 @@ def test_global_decode_equals_causal_prefill_row(p):
     assert np.abs(o_dec[0] - o_pre[0, p]).mean() < 2e-3
 
 
+# ---------------------------------------------------------------- FP8 inputs
+
+def test_e4m3_decoding_matches_torch_and_the_encoding():
+    """Every one of the 256 byte patterns against torch.float8_e4m3fn, and the
+    encoding's fixed points: 1.0, the largest normal 448, the smallest
+    subnormal 2^-9, the smallest normal 2^-6, NaN."""
+    b = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_to_f64(b)
+    ref = torch.from_numpy(b).view(torch.float8_e4m3fn).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and nan.sum() == 2
+    assert np.array_equal(mine[~nan], ref[~nan])
+    assert mine[0x38] == 1.0 and mine[0x7E] == 448.0 and mine[0xFE] == -448.0
+    assert mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6 and mine[0x80] == 0.0
+
+
 # ---------------------------------------------------- rounding and footprint
 
 def test_bf16_rounding_matches_torch_rne():

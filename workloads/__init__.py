@@ -148,6 +148,24 @@ def prefill_inputs(cfg: Prefill, device="cpu", seed=None, with_grad_out=None):
     return out
 
 
+def fp8_prefill_inputs(cfg: Prefill, device="cpu", seed=None):
+    """The inputs of :func:`prefill_inputs` with q, k and v quantised to FP8
+    E4M3, one factor per tensor (its largest magnitude over 448, the E4M3
+    maximum): q8, k8, v8 (torch.float8_e4m3fn) with qkv_scale [3] fp32, so that
+    q ~ q8 * qkv_scale[0] etc.  g, wq, wk as there.  The quantisation only
+    builds inputs: the library and the oracle both read the same bytes."""
+    x = prefill_inputs(cfg, device=device, seed=seed, with_grad_out=False)
+    out = {"g": x["g"], "wq": x["wq"], "wk": x["wk"]}
+    scales = []
+    for name in ("q", "k", "v"):
+        t = x[name].float()
+        s = float(t.abs().max()) / 448.0
+        out[name + "8"] = (t / s).to(torch.float8_e4m3fn)
+        scales.append(s)
+    out["qkv_scale"] = torch.tensor(scales, dtype=torch.float32, device=device)
+    return out
+
+
 def decode_layer_inputs(cfg: Decode, layer: int, device="cpu", N=None):
     """Inputs of one layer's decode step: rings, new token tensors, positions."""
     N = cfg.N if N is None else N
