@@ -16,7 +16,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring",
+__all__ = ["fwd", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring", "prefill_to_ring_varlen",
            "global_fwd", "global_decode_step", "global_decode_workspace_size",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
@@ -70,6 +70,8 @@ def lib():
         L.swa_decode_step.restype = ctypes.c_int
         L.swa_prefill_to_ring.argtypes = [P] + [_vp] * 6
         L.swa_prefill_to_ring.restype = ctypes.c_int
+        L.swa_prefill_to_ring_varlen.argtypes = [P] + [_vp] * 9
+        L.swa_prefill_to_ring_varlen.restype = ctypes.c_int
         L.swa_global_fwd.argtypes = [P] + [_vp] * 9 + [ctypes.c_int64, _vp]
         L.swa_global_fwd.restype = ctypes.c_int
         L.swa_global_decode_workspace_size.argtypes = [P, ctypes.c_int64]
@@ -381,6 +383,30 @@ def global_decode_step(pos, q, k_new, v_new, wq, wk, k_cache, v_cache, *, rot_di
                                       workspace.numel(), _stream(stream))
     _check(rc, "swa_global_decode_step")
     return out
+
+
+def prefill_to_ring_varlen(k, v, wk, k_cache, v_cache, starts, lens, pos0=None, *, Hq,
+                           rot_dim=42, rope_base=1e7, eps=1e-6, stream=None):
+    """The ring handoff for a ragged or continued prefill (swa_prefill_to_ring_varlen):
+    k, v [T, Hkv, 128] rows (packed, or a padded batch flattened); sequence b's
+    lens[b] tokens start at row starts[b], at position pos0[b] (0 if None);
+    rings [B, Hkv, 128, 128]."""
+    T, Hkv, D = k.shape
+    B, W = k_cache.shape[0], k_cache.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=W, rot_dim=rot_dim, rope_base=rope_base,
+                    eps=eps)
+    i64, bf = torch.int64, torch.bfloat16
+    nk = T * Hkv * D
+    nr = B * Hkv * W * D
+    extra = {} if pos0 is None else {"pos0": (pos0, i64, B)}
+    _need("swa_prefill_to_ring_varlen", k_cache.device, starts=(starts, i64, B),
+          lens=(lens, i64, B), k=(k, bf, nk), v=(v, bf, nk),
+          wk=(wk, torch.float32, D if B else 0), k_cache=(k_cache, bf, nr),
+          v_cache=(v_cache, bf, nr), **extra)
+    rc = lib().swa_prefill_to_ring_varlen(ctypes.byref(p), _ptr(starts), _ptr(lens), _ptr(pos0),
+                                          _ptr(k), _ptr(v), _ptr(wk), _ptr(k_cache),
+                                          _ptr(v_cache), _stream(stream))
+    _check(rc, "swa_prefill_to_ring_varlen")
 
 
 def get_last_device_error(stream=None):

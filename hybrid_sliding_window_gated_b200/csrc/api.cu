@@ -406,6 +406,38 @@ int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf
   return launch_prefill_ring(a, static_cast<cudaStream_t>(stream));
 }
 
+int swa_prefill_to_ring_varlen(const swa_params_t* p, const int64_t* starts, const int64_t* lens,
+                               const int64_t* pos0, const swa_bf16_t* k, const swa_bf16_t* v,
+                               const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                               void* stream) {
+  int rc = check_params(p, false);
+  if (rc != SWA_OK) return rc;
+  if (p->B == 0) return SWA_OK;
+  if (!starts || !lens || !wk || !k_cache || !v_cache || (p->T > 0 && (!k || !v)))
+    return SWA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(starts) & 7u) || (reinterpret_cast<uintptr_t>(lens) & 7u) ||
+      (reinterpret_cast<uintptr_t>(pos0) & 7u) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(wk) || !aligned16(k_cache) || !aligned16(v_cache))
+    return SWA_ERR_INVALID_ARG;
+  RingArgs a{};
+  a.B = static_cast<int>(p->B);
+  a.T = static_cast<int>(p->T);
+  a.Hkv = p->Hkv;
+  a.half_rot = p->rot_dim / 2;
+  a.eps = p->eps;
+  a.k = k;
+  a.v = v;
+  a.wk = wk;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.starts = starts;
+  a.lens = lens;
+  a.pos0 = pos0;
+  if ((rc = device_error_word(&a.err)) != SWA_OK) return rc;
+  fill_inv_freq(p, a.inv_freq);
+  return launch_prefill_ring(a, static_cast<cudaStream_t>(stream));
+}
+
 int swa_decode_step(const swa_params_t* p, const int64_t* pos, const swa_bf16_t* q,
                     const swa_bf16_t* k_new, const swa_bf16_t* v_new, const swa_bf16_t* g,
                     const float* wq, const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,

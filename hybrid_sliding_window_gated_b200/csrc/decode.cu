@@ -345,12 +345,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Prefill -> ring handoff.  Slot s of ring (b, kv head h) takes the latest
-// prefill position p <= T-1 with p = s (mod W): k' = RoPE_p(RMSNorm(k_p))
-// rounded to bf16, exactly as a decode step writes its new token, and v_p as
-// it is.  Slots that no position reaches (s > T-1) keep their contents.  One
-// warp per (sequence, slot): the slot's rotation is computed once for all KV
-// heads, whose rows lie next to each other; 4 dims per lane, so each 256-byte
-// row is one coalesced access.
+// position p of the sequence's tokens with p = s (mod W): k' = RoPE_p(RMSNorm
+// (k_p)) rounded to bf16, exactly as a decode step writes its new token, and
+// v_p as it is.  Slots that no position reaches keep their contents.  One warp
+// per (sequence, slot): the slot's rotation is computed once for all KV heads,
+// whose rows lie next to each other; 4 dims per lane, so each 256-byte row is
+// one coalesced access.  Dense form: tokens 0 .. T-1 of row b at positions
+// 0 .. T-1.  Varlen form: lens[b] tokens from row starts[b] at positions
+// pos0[b] ..; a sequence whose numbers do not fit the rows (or are negative)
+// is reported and skipped.
 __global__ void __launch_bounds__(128) swa_prefill_ring_kernel(const RingArgs a) {
   __shared__ __align__(16) float scratch[4][kHeadDim];
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -358,12 +361,29 @@ __global__ void __launch_bounds__(128) swa_prefill_ring_kernel(const RingArgs a)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;
   const int b = static_cast<int>(gw / kWindow), s = static_cast<int>(gw % kWindow);
-  if (b >= a.B || s > a.T - 1) return;  // warp-uniform
-  const long long p = (a.T - 1) - ((a.T - 1 - s) % kWindow);
+  if (b >= a.B) return;  // warp-uniform
+  long long first = 0, len = a.T, p0 = 0;  // row of token 0, tokens, position of token 0
+  if (a.lens != nullptr) {
+    first = a.starts[b];
+    len = a.lens[b];
+    p0 = a.pos0 != nullptr ? a.pos0[b] : 0;
+    if (first < 0 || len < 0 || p0 < 0 || len > a.T || first > a.T - len) {
+      if (s == 0 && lane == 0) atomicCAS(a.err, 0, kDevErrBadPosition);
+      return;
+    }
+  } else {
+    first = static_cast<long long>(b) * a.T;
+  }
+  if (len == 0) return;
+  // the latest position p in [p0, p0 + len) with p = s (mod W)
+  const long long last = p0 + len - 1;
+  const long long p = last - (((last - s) % kWindow) + kWindow) % kWindow;
+  if (p < p0) return;  // no position of this sequence reaches slot s
+  const long long row_tok = first + (p - p0);
   float cs = 1.0f, sn = 0.0f;
   if (lane < a.half_rot) rope_cos_sin(static_cast<double>(p), a.inv_freq[lane], &cs, &sn);
   for (int h = 0; h < a.Hkv; ++h) {
-    const long long row = ((static_cast<long long>(b) * a.T + p) * a.Hkv + h) * kHeadDim;
+    const long long row = (row_tok * a.Hkv + h) * kHeadDim;
     float x[4];
     load4(a.k + row + 4 * lane, x);
     const uint2 vv = *reinterpret_cast<const uint2*>(a.v + row + 4 * lane);

@@ -32,16 +32,23 @@ constexpr int kDevErrBadPosition = 0x200;
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecArgs& a,
                   cudaStream_t stream);
 
-// Prefill -> ring handoff (see swa_prefill_to_ring).
+// Prefill -> ring handoff (see swa_prefill_to_ring and its varlen form).
 struct RingArgs {
   int B, T, Hkv;
   int half_rot;
   float eps;
-  const uint16_t* k;  // [B, T, Hkv, D]
+  const uint16_t* k;  // [B, T, Hkv, D], or [T, Hkv, D] rows for the varlen form
   const uint16_t* v;
   const float* wk;
   uint16_t* k_cache;  // [B, Hkv, W, D]
   uint16_t* v_cache;
+  // Varlen form (null for the dense one): sequence b's token i is row
+  // starts[b] + i of k and v, at position pos0[b] + i (pos0 may be null: 0),
+  // for i < lens[b].
+  const int64_t* starts;
+  const int64_t* lens;
+  const int64_t* pos0;
+  int* err;
   double inv_freq[kMaxPairs];
 };
 

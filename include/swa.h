@@ -217,6 +217,28 @@ int swa_prefill_to_ring(const swa_params_t* p, const swa_bf16_t* k, const swa_bf
                         const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache, void* stream);
 
 /*
+ * The prefill -> ring handoff for ragged batches and continued prefills.  p->B
+ * sequences; sequence b's lens[b] tokens are rows starts[b] .. starts[b] +
+ * lens[b] - 1 of k, v [p->T, Hkv, D] (a packed batch: starts = cumulative
+ * lengths; or a padded [B, Tmax] batch: starts[b] = b Tmax, p->T = B Tmax),
+ * at positions pos0[b] .. pos0[b] + lens[b] - 1 (pos0 NULL: 0).  Slot s of
+ * ring b receives the latest of those positions p with p = s (mod W), as
+ * swa_prefill_to_ring writes it; other slots keep their contents (so a
+ * continued prefill, pos0 > 0, keeps the earlier chunk's slots it does not
+ * reach).  starts, lens, pos0: [B] int64 DEVICE arrays, 8-byte aligned; a
+ * sequence with a negative value or rows past p->T is skipped and reported
+ * by swa_get_last_device_error as SWA_ERR_INVALID_ARG.  A padded batch's
+ * prefill runs through swa_fwd unchanged: causal attention makes each valid
+ * row independent of the padding after it.  Source: the serving view of the
+ * window layers, which keep only their last W tokens (jaehun.me review,
+ * "Why the KV Cache Shrinks by 6.4x").
+ */
+int swa_prefill_to_ring_varlen(const swa_params_t* p, const int64_t* starts, const int64_t* lens,
+                               const int64_t* pos0, const swa_bf16_t* k, const swa_bf16_t* v,
+                               const float* wk, swa_bf16_t* k_cache, swa_bf16_t* v_cache,
+                               void* stream);
+
+/*
  * Global causal GQA layers (no counterpart of the window: 5 of ZGCM-1's 32
  * layers, at 6, 12, 18, 24 and 30, attend over the whole causal context with
  * the same QK-RMSNorm, partial RoPE and GQA, and without the output gate --

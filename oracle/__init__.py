@@ -5,9 +5,9 @@ CPU-baseline / reference legs of ``bench.py`` may import this package.  It
 shares no code with the CUDA library and never imports it.
 
 The arithmetic lives in ``swa_oracle.c`` (plain C, IEEE fp64, OpenMP over
-independent rows); this module marshals numpy arrays, and writes two steps
-out in numpy on top of the C norm/RoPE: the prefill -> ring handoff and the
-global layers' decode over a full-length cache.  Definitions follow
+independent rows); this module marshals numpy arrays, and writes a few steps
+out in numpy on top of the C norm/RoPE: the prefill -> ring handoff (dense
+and ragged) and the global layers' decode over a full-length cache.  Definitions follow
 the ZGCM-1 pages: "7.39B 오픈 모델로 256K 문맥의 … ZGCM-1" (onedev.kr), section
 "어떻게 동작하나", and "ZGCM-1: A Fully Open and Extremely Efficient Foundation
 Model …" (jaehun.me), sections "How Gated SWA Behaves" and "Why the KV Cache
@@ -242,6 +242,31 @@ def prefill_to_ring(k, v, wk, k_cache_bits, v_cache_bits, *, R, base, eps):
         kp = norm_rope(k[:, p], wk, np.full(B, float(p)), R, base, eps)  # [B, Hkv, D]
         kc[:, :, s, :] = bf16_round_array(kp)
         vc[:, :, s, :] = bf16_round_array(v[:, p])
+    return kc, vc
+
+
+def prefill_to_ring_varlen(k, v, wk, k_cache_bits, v_cache_bits, starts, lens, pos0, *, R, base,
+                           eps):
+    """Decode rings after ragged or continued prefills.
+
+    Sequence b's lens[b] tokens are rows starts[b] .. of k, v [rows, Hkv, D]
+    (fp64 values of bf16 inputs), at positions pos0[b] + i.  As in
+    :func:`prefill_to_ring`, slot s of ring b takes the latest of those
+    positions p with p = s (mod W): k' = RoPE_p(RMSNorm(k, wk)) rounded to bf16,
+    and v.  Slots no position reaches keep their bits.  Returns the new bits.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    kc = np.array(k_cache_bits, dtype=np.uint16, copy=True, order="C")
+    vc = np.array(v_cache_bits, dtype=np.uint16, copy=True, order="C")
+    W = kc.shape[2]
+    for b in range(kc.shape[0]):
+        n, first, p0 = int(lens[b]), int(starts[b]), int(pos0[b])
+        for p in range(max(p0, p0 + n - W), p0 + n):  # the last W positions
+            row = first + (p - p0)
+            kp = norm_rope(k[row][None], wk, np.array([float(p)]), R, base, eps)[0]
+            kc[b, :, p % W, :] = bf16_round_array(kp)
+            vc[b, :, p % W, :] = bf16_round_array(v[row])
     return kc, vc
 
 

@@ -206,3 +206,88 @@ def test_prefill_then_decode_continues_the_sequence():
     assert swa.get_last_device_error()[0] == swa.OK
     assert_parity(to_f64(o_pre), o_ref[:, :T], "prefill rows")
     assert_parity(to_f64(o_dec), o_ref[:, T], "decode row after the ring handoff")
+
+
+def _varlen_case(lens, pos0, seed, Hkv=2):
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+    rows = int(sum(lens))
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    k = torch.randn((max(rows, 1), Hkv, 128), generator=gen).bfloat16()
+    v = torch.randn((max(rows, 1), Hkv, 128), generator=gen).bfloat16()
+    wk = 1 + 0.1 * torch.randn(128, generator=gen)
+    B = len(lens)
+    kc0 = (torch.randn((B, Hkv, 128, 128), generator=gen) * 50).bfloat16()
+    vc0 = (torch.randn((B, Hkv, 128, 128), generator=gen) * 50).bfloat16()
+    return starts, k, v, wk, kc0, vc0
+
+
+@pytest.mark.parametrize("pos0", [None, [5, 0, 1000, 130, 7, 0, 64]])
+def test_prefill_to_ring_varlen_matches_oracle(pos0):
+    """Ragged lengths below, at and above the window, packed in one row array,
+    optionally continuing at positions > 0: V slots bit-exact, K' slots within
+    one bf16 step, unreached slots untouched (they keep the noise)."""
+    lens = [0, 1, 77, 127, 128, 129, 300]
+    starts, k, v, wk, kc0, vc0 = _varlen_case(lens, pos0, seed=41)
+    dev = lambda t: t.to(DEV)
+    i64 = lambda x: torch.tensor(x, dtype=torch.int64, device=DEV)
+    kc, vc = dev(kc0), dev(vc0)
+    swa.prefill_to_ring_varlen(dev(k), dev(v), dev(wk), kc, vc, i64(starts), i64(lens),
+                               None if pos0 is None else i64(pos0), Hq=8, rope_base=1e7)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    kr, vr = oracle.prefill_to_ring_varlen(f64(k), f64(v), f64(wk), bits(kc0), bits(vc0), starts,
+                                           lens, [0] * 7 if pos0 is None else pos0, R=42,
+                                           base=1e7, eps=1e-6)
+    assert np.array_equal(bits(vc), vr)
+    gk, rk = oracle.bf16_bits_to_f64(bits(kc)), oracle.bf16_bits_to_f64(kr)
+    assert np.all(np.abs(gk - rk) <= np.abs(rk) * 2.0 ** -7 + 1e-6)
+    same = bits(kc0) == kr  # slots the oracle left alone are bit-identical on the GPU too
+    assert np.array_equal(bits(kc)[same], kr[same])
+
+
+def test_padded_ragged_batch_prefill_handoff_then_decode():
+    """A serving batch padded to Tmax = 300 with true lengths 50, 300, 129:
+    swa_fwd on the padded batch (causal rows do not see the padding after
+    them), the varlen handoff with each sequence's true length, then one
+    decode step per sequence at its own next position, against the oracle's
+    forward over that sequence's len + 1 tokens."""
+    lens, Tmax, Hq, Hkv = [50, 300, 129], 300, 8, 2
+    cfg = workloads.custom_prefill(3, Tmax + 1, Hq, Hkv, base=1e7, g_std=1.0, seed=43)
+    inp = workloads.prefill_inputs(cfg)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    pre = {x: d[x][:, :Tmax].contiguous() for x in ("q", "k", "v", "g")}
+    o_pre = swa.fwd(pre["q"], pre["k"], pre["v"], pre["g"], d["wq"], d["wk"], rot_dim=cfg.R,
+                    rope_base=cfg.base, eps=cfg.eps)
+    kc = torch.zeros((3, Hkv, 128, 128), dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    i64 = lambda x: torch.tensor(x, dtype=torch.int64, device=DEV)
+    swa.prefill_to_ring_varlen(pre["k"].view(-1, Hkv, 128), pre["v"].view(-1, Hkv, 128), d["wk"],
+                               kc, vc, i64([0, Tmax, 2 * Tmax]), i64(lens), Hq=Hq, rot_dim=cfg.R,
+                               rope_base=cfg.base, eps=cfg.eps)
+    # each sequence's next token is row len[b] of its inputs
+    idx = torch.tensor(lens, device=DEV)
+    nxt = {x: d[x][torch.arange(3, device=DEV), idx].contiguous() for x in ("q", "k", "v", "g")}
+    o_dec = swa.decode_step(i64(lens), nxt["q"], nxt["k"], nxt["v"], nxt["g"], d["wq"], d["wk"],
+                            kc, vc, rot_dim=cfg.R, rope_base=cfg.base, eps=cfg.eps)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    for b, n in enumerate(lens):
+        sl = {x: f64(inp[x][b:b + 1, :n + 1]) for x in ("q", "k", "v", "g")}
+        o_ref, _ = oracle.fwd(sl["q"], sl["k"], sl["v"], sl["g"], f64(inp["wq"]), f64(inp["wk"]),
+                              W=cfg.W, R=cfg.R, base=cfg.base, eps=cfg.eps)
+        assert_parity(to_f64(o_pre[b:b + 1, :n]), o_ref[:, :n], f"padded prefill rows, seq {b}")
+        assert_parity(to_f64(o_dec[b]), o_ref[0, n], f"decode after the ragged handoff, seq {b}")
+
+
+def test_prefill_to_ring_varlen_bad_lengths_are_reported():
+    lens = [10, 20]
+    starts, k, v, wk, kc0, vc0 = _varlen_case(lens, None, seed=44)
+    i64 = lambda x: torch.tensor(x, dtype=torch.int64, device=DEV)
+    kc, vc = kc0.to(DEV), vc0.to(DEV)
+    swa.prefill_to_ring_varlen(k.to(DEV), v.to(DEV), wk.to(DEV), kc, vc, i64([0, 25]), i64(lens),
+                               Hq=4)  # rows 25 .. 44 of 30: past the end
+    code, _ = swa.get_last_device_error()
+    assert code == swa.ERR_INVALID_ARG
+    assert swa.get_last_device_error()[0] == swa.OK
+    assert torch.equal(kc[1], kc0[1].to(DEV)) and torch.equal(vc[1], vc0[1].to(DEV))
+    assert not torch.equal(kc[0], kc0[0].to(DEV))  # the valid sequence was written

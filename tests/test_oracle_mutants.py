@@ -90,6 +90,10 @@ PY_MUTANTS = [
        "vc[n, :, p, :] = bf16_round_array(k_new[n])")]),
     ("global_decode_scale_dropped", "global_decode",
      [("s = sc * (keys @ qp[h])", "s = keys @ qp[h]")]),
+    ("ring_varlen_position_offset_dropped", "prefill_to_ring_varlen",
+     [("np.array([float(p)])", "np.array([float(p - p0)])")]),
+    ("ring_varlen_drops_oldest", "prefill_to_ring_varlen",
+     [("range(max(p0, p0 + n - W), p0 + n)", "range(max(p0, p0 + n - W + 1), p0 + n)")]),
     ("e4m3_bias_8", "e4m3_to_f64", [("e.astype(np.float64) - 7.0", "e.astype(np.float64) - 8.0")]),
     ("e4m3_subnormal_scale", "e4m3_to_f64", [("m * 2.0 ** -9", "m * 2.0 ** -10")]),
 ]
@@ -113,6 +117,8 @@ PINS = (
        for T in (1, 131)]
     + [("global_decode_dense", pins.test_global_decode_matches_dense_over_cache_contents, ())]
     + [("e4m3_decoding", pins.test_e4m3_decoding_matches_torch_and_the_encoding, ())]
+    + [(f"ring_varlen({c})", pins.test_prefill_to_ring_varlen_equals_sequential_decode, (c,))
+       for c in ("ragged", "continued")]
     + [(f"global_decode_ring({p})", pins.test_global_decode_equals_ring_decode_inside_the_window,
         (p,)) for p in (0, 77)]
     + [(f"global_decode_prefill({p})", pins.test_global_decode_equals_causal_prefill_row, (p,))
@@ -180,7 +186,8 @@ def test_unmodified_copy_passes_every_pin(tmp_path):
     with oracle_library(build_variant(tmp_path, [])):
         assert failing_pins(stop_at_first=False) == []
     with oracle_function("prefill_to_ring", []), oracle_function("fwd_rows", []), \
-            oracle_function("global_decode", []), oracle_function("e4m3_to_f64", []):
+            oracle_function("global_decode", []), oracle_function("e4m3_to_f64", []), \
+            oracle_function("prefill_to_ring_varlen", []):
         assert failing_pins(stop_at_first=False) == []
 
 

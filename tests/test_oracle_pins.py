@@ -347,6 +347,45 @@ def test_prefill_to_ring_equals_sequential_decode(T):
         assert np.array_equal(vr[:, :, T:], vc0[:, :, T:])
 
 
+@pytest.mark.parametrize("case", ["ragged", "continued"])
+def test_prefill_to_ring_varlen_equals_sequential_decode(case):
+    """Ragged sequences (lengths 0, 1, 77, 127, 128, 129, 300) packed in one
+    row array, some continuing at positions > 0: each ring equals what
+    decode steps at that sequence's positions leave behind, from the same
+    noise; with every length T and positions from 0 it is the dense handoff."""
+    W, R, base, eps, Hq, Hkv, D = 128, 42, 1e7, 1e-6, 4, 2, 128
+    lens = [0, 1, 77, 127, 128, 129, 300]
+    pos0 = [0] * 7 if case == "ragged" else [5, 0, 1000, 130, 7, 0, 64]
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    rows = int(sum(lens))
+    rng = np.random.default_rng(70)
+    bf = lambda x: oracle.bf16_bits_to_f64(oracle.bf16_round_array(x))
+    k, v = bf(rng.standard_normal((rows, Hkv, D))), bf(rng.standard_normal((rows, Hkv, D)))
+    q, g = bf(rng.standard_normal((rows, Hq, D))), bf(rng.standard_normal((rows, Hq, D)))
+    wq, wk = 1 + 0.1 * rng.standard_normal(D), 1 + 0.1 * rng.standard_normal(D)
+    B = len(lens)
+    kc0 = oracle.bf16_round_array(rng.standard_normal((B, Hkv, W, D)) * 50)
+    vc0 = oracle.bf16_round_array(rng.standard_normal((B, Hkv, W, D)) * 50)
+    kr, vr = oracle.prefill_to_ring_varlen(k, v, wk, kc0, vc0, starts, lens, pos0, R=R, base=base,
+                                           eps=eps)
+    for b in range(B):
+        kc, vc = kc0[b:b + 1], vc0[b:b + 1]
+        for i in range(lens[b]):
+            r = starts[b] + i
+            _, kc, vc = oracle.decode(np.array([pos0[b] + i]), q[r][None], k[r][None], v[r][None],
+                                      g[r][None], wq, wk, kc, vc, R=R, base=base, eps=eps)
+        assert np.array_equal(kr[b:b + 1], kc) and np.array_equal(vr[b:b + 1], vc), b
+    # every length T from position 0 in a padded layout: the dense handoff
+    T = 140
+    kd = bf(rng.standard_normal((3, T, Hkv, D)))
+    vd = bf(rng.standard_normal((3, T, Hkv, D)))
+    ka, va = oracle.prefill_to_ring(kd, vd, wk, kc0[:3], vc0[:3], R=R, base=base, eps=eps)
+    kb, vb = oracle.prefill_to_ring_varlen(kd.reshape(-1, Hkv, D), vd.reshape(-1, Hkv, D), wk,
+                                           kc0[:3], vc0[:3], [0, T, 2 * T], [T] * 3, [0] * 3,
+                                           R=R, base=base, eps=eps)
+    assert np.array_equal(ka, kb) and np.array_equal(va, vb)
+
+
 def test_decode_matches_dense_over_ring_contents():
     """Decode output = dense softmax over the ring's keys (positions known)."""
     W, R, base, eps, Hq, Hkv, D, N = 128, 42, 1e7, 1e-6, 8, 2, 128, 3
