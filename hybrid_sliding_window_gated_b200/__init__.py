@@ -16,7 +16,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring", "prefill_to_ring_varlen",
+__all__ = ["fwd", "fwd_halo", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring", "prefill_to_ring_varlen",
            "global_fwd", "global_decode_step", "global_decode_workspace_size",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
@@ -55,6 +55,8 @@ def lib():
         P = ctypes.POINTER(Params)
         L.swa_fwd.argtypes = [P] + [_vp] * 9
         L.swa_fwd.restype = ctypes.c_int
+        L.swa_fwd_halo.argtypes = [P] + [_vp] * 8 + [ctypes.c_int64, _vp, _vp, _vp]
+        L.swa_fwd_halo.restype = ctypes.c_int
         L.swa_fwd_fp8.argtypes = [P] + [_vp] * 10
         L.swa_fwd_fp8.restype = ctypes.c_int
         L.swa_bwd.argtypes = [P] + [_vp] * 15 + [ctypes.c_size_t, _vp]
@@ -154,6 +156,33 @@ def fwd(q, k, v, g, wq, wk, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6, 
     rc = lib().swa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
                        _ptr(out), _ptr(lse), _stream(stream))
     _check(rc, "swa_fwd")
+    return (out, lse) if lse is not None else out
+
+
+def fwd_halo(q, k, v, g, wq, wk, k_halo, v_halo, pos0, *, window=128, rot_dim=42, rope_base=1e4,
+             eps=1e-6, scale=0.0, out=None, lse=None, want_lse=False, flags=0, stream=None):
+    """:func:`fwd` for a chunk starting at position pos0 whose previous 127 tokens
+    are k_halo, v_halo [B,127,Hkv,128] (swa_fwd_halo); both None: no history."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale, flags=flags)
+    nq, nk, nh = B * T * Hq * D, B * T * Hkv * D, B * (window - 1) * Hkv * D
+    bf, f32 = torch.bfloat16, torch.float32
+    opt = {} if lse is None else {"lse": (lse, f32, B * Hq * T)}
+    if k_halo is not None or v_halo is not None:
+        opt["k_halo"] = (k_halo, bf, nh if nq else 0)
+        opt["v_halo"] = (v_halo, bf, nh if nq else 0)
+    _need("swa_fwd_halo", q.device, q=(q, bf, nq), k=(k, bf, nk), v=(v, bf, nk), g=(g, bf, nq),
+          wq=(wq, f32, D if nq else 0), wk=(wk, f32, D if nq else 0), out=(out, bf, nq), **opt)
+    rc = lib().swa_fwd_halo(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
+                            _ptr(wk), _ptr(k_halo), _ptr(v_halo), int(pos0), _ptr(out), _ptr(lse),
+                            _stream(stream))
+    _check(rc, "swa_fwd_halo")
     return (out, lse) if lse is not None else out
 
 

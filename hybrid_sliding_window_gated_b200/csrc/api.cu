@@ -150,16 +150,23 @@ static void fill_inv_freq(const swa_params_t* p, double* out) {
 
 namespace swa {
 
-// swa_fwd, and swa_fwd_fp8 when qkv_scale is set (q, k, v then point at E4M3 bytes).
+// swa_fwd, swa_fwd_fp8 when qkv_scale is set (q, k, v then point at E4M3
+// bytes), and swa_fwd_halo when k_halo / v_halo are set.
 static int fwd_impl(const swa_params_t* p, const void* q, const void* k, const void* v,
                     const float* qkv_scale, const swa_bf16_t* g, const float* wq, const float* wk,
-                    swa_bf16_t* o, float* lse, void* stream) {
+                    swa_bf16_t* o, float* lse, const swa_bf16_t* k_halo,
+                    const swa_bf16_t* v_halo, int64_t pos0, void* stream) {
   int rc = check_params(p, false);
   if (rc != SWA_OK) return rc;
+  const bool halo = k_halo != nullptr || v_halo != nullptr;
+  if (pos0 < 0 || (halo && (!k_halo || !v_halo || pos0 < kWindow - 1)) ||
+      pos0 > (1ll << 40))
+    return SWA_ERR_INVALID_ARG;
   if (p->B == 0 || p->T == 0) return SWA_OK;
   if (!q || !k || !v || !g || !wq || !wk || !o) return SWA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o) ||
-      !aligned16(wq) || !aligned16(wk) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+      !aligned16(wq) || !aligned16(wk) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (halo && (!aligned16(k_halo) || !aligned16(v_halo))))
     return SWA_ERR_INVALID_ARG;
 
   FwdArgs a{};
@@ -176,6 +183,8 @@ static int fwd_impl(const swa_params_t* p, const void* q, const void* k, const v
   a.wq = wq;
   a.wk = wk;
   a.qkv_scale = qkv_scale;
+  a.halo = halo ? 1 : 0;
+  a.pos0 = pos0;
   a.g = g;
   a.o = o;
   a.lse = lse;
@@ -197,7 +206,15 @@ static int fwd_impl(const swa_params_t* p, const void* q, const void* k, const v
       (rc = encode_tmap_4d(&tg, g, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       (rc = encode_tmap_4d(&to, o, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
-  return launch_fwd(p, tq, tk, tv, tg, to, a, static_cast<cudaStream_t>(stream));
+  // The halo's W-1 rows per (sequence, KV head), loaded as key tile -1 from row -1.
+  CUtensorMap tkh = tk, tvh = tv;
+  if (halo &&
+      ((rc = encode_tmap_4d(&tkh, k_halo, D, p->Hkv, kWindow - 1, B, 64, 1, kTile, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) ||
+       (rc = encode_tmap_4d(&tvh, v_halo, D, p->Hkv, kWindow - 1, B, 64, 1, kTile, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B))))
+    return rc;
+  return launch_fwd(p, tq, tk, tv, tg, to, tkh, tvh, a, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace swa
@@ -238,7 +255,14 @@ int swa_get_last_device_error(void* stream, int* site) {
 int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, const swa_bf16_t* v,
             const swa_bf16_t* g, const float* wq, const float* wk, swa_bf16_t* o, float* lse,
             void* stream) {
-  return fwd_impl(p, q, k, v, nullptr, g, wq, wk, o, lse, stream);
+  return fwd_impl(p, q, k, v, nullptr, g, wq, wk, o, lse, nullptr, nullptr, 0, stream);
+}
+
+int swa_fwd_halo(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                 const swa_bf16_t* k_halo, const swa_bf16_t* v_halo, int64_t pos0, swa_bf16_t* o,
+                 float* lse, void* stream) {
+  return fwd_impl(p, q, k, v, nullptr, g, wq, wk, o, lse, k_halo, v_halo, pos0, stream);
 }
 
 int swa_fwd_fp8(const swa_params_t* p, const uint8_t* q, const uint8_t* k, const uint8_t* v,
@@ -247,7 +271,7 @@ int swa_fwd_fp8(const swa_params_t* p, const uint8_t* q, const uint8_t* k, const
   if (p != nullptr && p->B > 0 && p->T > 0 &&
       (qkv_scale == nullptr || (reinterpret_cast<uintptr_t>(qkv_scale) & 3u)))
     return SWA_ERR_INVALID_ARG;
-  return fwd_impl(p, q, k, v, qkv_scale, g, wq, wk, o, lse, stream);
+  return fwd_impl(p, q, k, v, qkv_scale, g, wq, wk, o, lse, nullptr, nullptr, 0, stream);
 }
 
 }  // extern "C"

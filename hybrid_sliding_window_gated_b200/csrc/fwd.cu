@@ -153,9 +153,15 @@ __device__ __forceinline__ void next_head(Cursor& c, const FwdArgs& a) {
     next_tile(c, a);
   }
 }
-// Key tile t-1 exists / must be loaded at this tile (first tile of a run).
-__device__ __forceinline__ bool has_prev(const Cursor& c) { return c.t > 0; }
-__device__ __forceinline__ bool need_prev(const Cursor& c) { return c.t > 0 && c.u == 0; }
+// Key tile t-1 exists (chain tile 0 has one when the previous chunk's halo
+// is given: key tile -1) / must be loaded at this tile (the first tile of a
+// run, or chain tile 0 with a halo, whose ring slot held another chain's tile).
+__device__ __forceinline__ bool has_prev(const Cursor& c, const FwdArgs& a) {
+  return c.t > 0 || a.halo;
+}
+__device__ __forceinline__ bool need_prev(const Cursor& c, const FwdArgs& a) {
+  return has_prev(c, a) && (c.u == 0 || c.t == 0);
+}
 // Last tile of the run on its chain: its K/V tile is released after use.
 __device__ __forceinline__ bool seg_last(const Cursor& c, const FwdArgs& a, int n_tiles) {
   return c.u == n_tiles - 1 || c.t == a.tiles_per_chain - 1;
@@ -476,7 +482,8 @@ template <int kPairs, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
+                   const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_kh,
+                   const __grid_constant__ CUtensorMap tm_vh, const FwdArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];  // 128B-swizzled tiles need 1 KiB
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -523,6 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_g);
     prefetch_tensormap(&tm_o);
+    if (a.halo) {
+      prefetch_tensormap(&tm_kh);
+      prefetch_tensormap(&tm_vh);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -565,15 +576,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.kfull[s], kHalfBytes);
             tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
           } else {
+            // key tile -1: the halo's 127 rows, from row -1 (zero-filled, never in the band)
+            const CUtensorMap* map = j < 0 ? &tm_kh : &tm_k;
+            const int y = j < 0 ? -1 : j * kTile;
             mbar_arrive_expect_tx(&sm.kfull[s], kTileBytes);
-            tma_load_4d(sm.k[s], &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
-            tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 64, c.kvh, j * kTile, c.b);
+            tma_load_4d(sm.k[s], map, &sm.kfull[s], 0, c.kvh, y, c.b);
+            tma_load_4d(sm.k[s] + kHalfBytes, map, &sm.kfull[s], 64, c.kvh, y, c.b);
           }
         }
         // rot(128 j w_p) for this tile, then the second arrive on kfull.
         if (lane < kPairs) {
           float cv, sv;
-          rope_cos_sin(static_cast<double>(j) * kTile, a.inv_freq[lane], &cv, &sv);
+          rope_cos_sin(static_cast<double>(a.pos0 + static_cast<long long>(j) * kTile),
+                       a.inv_freq[lane], &cv, &sv);
           sm.rot_tile[s][lane] = make_float2(cv, sv);
         }
         __syncwarp();
@@ -586,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nq = 0;  // Q loads issued
       Cursor c = cursor_at(a, u0);
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
-        if (need_prev(c)) ok = load_kv(true, c.t - 1, c);  // first tile of a run: key tile t-1 too
+        if (need_prev(c, a)) ok = load_kv(true, c.t - 1, c);  // first tile of a run: key tile t-1 too
         ok = ok && load_kv(true, c.t, c);
         for (int h = 0; h < a.G && ok; ++h) {
           const int qs = nq % 3;
@@ -627,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       Cursor c = cursor_at(a, u0);
       for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
-        for (int j = need_prev(c) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+        for (int j = need_prev(c, a) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
           const int s = j & 1;
           if (vr.was_used(s) &&
               !(ok = mbar_wait_inl(&sm.vempty[s], vr.parity(s) ^ 1u, abort, a.err, kSiteVEmpty)))
@@ -636,9 +651,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&sm.vfull[s], kHalfBytes);
             tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
           } else {
+            const CUtensorMap* map = j < 0 ? &tm_vh : &tm_v;
+            const int y = j < 0 ? -1 : j * kTile;
             mbar_arrive_expect_tx(&sm.vfull[s], kTileBytes);
-            tma_load_4d(sm.v[s], &tm_v, &sm.vfull[s], 0, c.kvh, j * kTile, c.b);
-            tma_load_4d(sm.v[s] + kHalfBytes, &tm_v, &sm.vfull[s], 64, c.kvh, j * kTile, c.b);
+            tma_load_4d(sm.v[s], map, &sm.vfull[s], 0, c.kvh, y, c.b);
+            tma_load_4d(sm.v[s] + kHalfBytes, map, &sm.vfull[s], 64, c.kvh, y, c.b);
           }
           vr.advance(s);
         }
@@ -660,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t cnt = static_cast<uint32_t>(m >> 1);
           const int sp = (cq.t + 1) & 1, sc = cq.t & 1;
           if (cq.h == 0) {
-            if (need_prev(cq)) {
+            if (need_prev(cq, a)) {
               if (!mbar_wait_inl(&sm.kready[sp], kr.parity(sp), abort, a.err, kSiteKReady)) { ok = false; break; }
               kr.advance(sp);
             }
@@ -671,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cnt > 0 && !mbar_wait_inl(&sm.tfree[r], (cnt - 1) & 1, abort, a.err, kSiteTFree)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s_base = tmem + r * 256;
-          const bool hp = has_prev(cq);
+          const bool hp = has_prev(cq, a);
           for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
             const uint8_t* kt = sm.k[blk == 0 ? sp : sc];
 #pragma unroll
@@ -692,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cp.h == 0) {
             // FP8 V is read once a region warpgroup has expanded it to bf16
             uint64_t* vb = kFp8 ? sm.vready : sm.vfull;
-            if (need_prev(cp)) {
+            if (need_prev(cp, a)) {
               if (!mbar_wait_inl(&vb[sp], vr.parity(sp), abort, a.err, kSiteVFull)) { ok = false; break; }
               vr.advance(sp);
             }
@@ -702,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait_inl(&sm.pfull[r], cnt & 1, abort, a.err, kSitePFull)) { ok = false; break; }
           tc_fence_after();
           const uint32_t p_base = tmem + r * 256;
-          const bool hp = has_prev(cp);
+          const bool hp = has_prev(cp, a);
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
             const uint8_t* vt = sm.v[blk == 0 ? sp : sc];
@@ -765,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor kc = cursor_at(a, u0);
     auto account = [&](int upto, bool transform_last) -> bool {
       while (acct <= upto) {
-        for (int j = need_prev(kc) ? kc.t - 1 : kc.t; j <= kc.t; ++j) {
+        for (int j = need_prev(kc, a) ? kc.t - 1 : kc.t; j <= kc.t; ++j) {
           const int s = j & 1;
           if (transform_last && acct == upto) {
             if (!mbar_wait_inl(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
@@ -838,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // The MMA saw unnormalised q rows; 1/rms(q) enters with the softmax scale.
       const float rs = sl2 * rinv;
-      const bool hp = has_prev(c);
+      const bool hp = has_prev(c, a);
       float ms = bound;
       if (exact) {
         // Row maximum over the band: key tile t-1 gives columns c > row, key
@@ -1015,8 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int kPairs, bool kFp8>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
-                cudaStream_t stream) {
+                const CUtensorMap& tg, const CUtensorMap& to, const CUtensorMap& tkh,
+                const CUtensorMap& tvh, const FwdArgs& a, int num_sms, cudaStream_t stream) {
   const size_t smem = sizeof(Smem);
   static int configured_device = -1;
   int dev = 0;
@@ -1035,18 +1052,18 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
   return launch_dependent(swa_fwd_kernel<kPairs, kFp8>, static_cast<unsigned>(grid), kThreads,
-                          smem, stream, tq, tk, tv, tg, to, a);
+                          smem, stream, tq, tk, tv, tg, to, tkh, tvh, a);
 }
 
 template <bool kFp8>
 int launch_rot(int rot_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& tg, const CUtensorMap& to, const FwdArgs& a, int num_sms,
-               cudaStream_t stream) {
+               const CUtensorMap& tg, const CUtensorMap& to, const CUtensorMap& tkh,
+               const CUtensorMap& tvh, const FwdArgs& a, int num_sms, cudaStream_t stream) {
   switch (rot_dim) {
-    case 0: return launch_impl<0, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
-    case 32: return launch_impl<16, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
-    case 42: return launch_impl<21, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
-    case 48: return launch_impl<24, kFp8>(tq, tk, tv, tg, to, a, num_sms, stream);
+    case 0: return launch_impl<0, kFp8>(tq, tk, tv, tg, to, tkh, tvh, a, num_sms, stream);
+    case 32: return launch_impl<16, kFp8>(tq, tk, tv, tg, to, tkh, tvh, a, num_sms, stream);
+    case 42: return launch_impl<21, kFp8>(tq, tk, tv, tg, to, tkh, tvh, a, num_sms, stream);
+    case 48: return launch_impl<24, kFp8>(tq, tk, tv, tg, to, tkh, tvh, a, num_sms, stream);
     default: return SWA_ERR_UNSUPPORTED;
   }
 }
@@ -1055,14 +1072,18 @@ int launch_rot(int rot_dim, const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, const CUtensorMap& tg, const CUtensorMap& to,
-               const FwdArgs& a, cudaStream_t stream) {
+               const CUtensorMap& tkh, const CUtensorMap& tvh, const FwdArgs& a,
+               cudaStream_t stream) {
   DeviceInfo di;
   int rc = current_device_info(&di);
   if (rc != SWA_OK) return rc;
   if (a.total_tiles > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
+  if (a.qkv_scale != nullptr && a.halo) return SWA_ERR_UNSUPPORTED;  // FP8 takes no halo
   return a.qkv_scale != nullptr
-             ? fwd::launch_rot<true>(p->rot_dim, tq, tk, tv, tg, to, a, di.num_sms, stream)
-             : fwd::launch_rot<false>(p->rot_dim, tq, tk, tv, tg, to, a, di.num_sms, stream);
+             ? fwd::launch_rot<true>(p->rot_dim, tq, tk, tv, tg, to, tkh, tvh, a, di.num_sms,
+                                     stream)
+             : fwd::launch_rot<false>(p->rot_dim, tq, tk, tv, tg, to, tkh, tvh, a, di.num_sms,
+                                      stream);
 }
 
 }  // namespace swa

@@ -20,6 +20,8 @@ struct FwdArgs {
   float scale_log2;  // softmax scale * log2(e)
   float eps;
   int flags;         // SWA_FLAG_* debug bits (0 in normal use)
+  int halo;          // 1: the previous chunk's last W-1 tokens precede row 0 (key tile -1)
+  long long pos0;    // position of row 0
   const float* wq;
   const float* wk;
   const float* qkv_scale;  // FP8 (E4M3) q, k, v: their dequantisation factors; null for bf16
@@ -44,9 +46,12 @@ int encode_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                    uint64_t d3, uint32_t box0, uint32_t box1, uint32_t box2, uint32_t box3,
                    CUtensorMapSwizzle swizzle, bool bytes = false);
 
+// tkh, tvh: tensor maps of the halo K and V [B, W-1, Hkv, D] (used only when
+// a.halo is set; any valid map otherwise).
 int launch_fwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, const CUtensorMap& tg, const CUtensorMap& to,
-               const FwdArgs& a, cudaStream_t stream);
+               const CUtensorMap& tkh, const CUtensorMap& tvh, const FwdArgs& a,
+               cudaStream_t stream);
 
 int map_cuda_error(cudaError_t e);
 

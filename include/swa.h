@@ -101,6 +101,25 @@ int swa_fwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
             swa_bf16_t* o, float* lse, void* stream);
 
 /*
+ * swa_fwd for one chunk of longer sequences: row 0 of q, k, v, g is at
+ * position pos0, and the W - 1 = 127 tokens before it -- the previous
+ * chunk's last ones, positions pos0 - 127 .. pos0 - 1 -- are given as k_halo,
+ * v_halo [B, 127, Hkv, D] bf16 (raw k and v, as the previous chunk received
+ * them), so every query row sees its whole window.  pos0 >= 127 (with a
+ * halo, every halo row is a real token); k_halo and v_halo both set or both
+ * NULL (then pos0 only shifts the positions: a chunk without history).
+ * Other arguments and results as swa_fwd: o, lse [B, Hq, T] for the chunk's
+ * own rows.  For sequence sharding (a rank holds a contiguous slice of every
+ * sequence) and continued prefills: the halo crosses the chunk boundary
+ * because a token sees the W - 1 before it (jaehun.me review, "How Gated SWA
+ * Behaves").
+ */
+int swa_fwd_halo(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                 const swa_bf16_t* k_halo, const swa_bf16_t* v_halo, int64_t pos0, swa_bf16_t* o,
+                 float* lse, void* stream);
+
+/*
  * swa_fwd with q, k and v in FP8 E4M3 (one byte per element, the OCP E4M3
  * encoding: bias 7, no infinities), each with one fp32 dequantisation factor:
  * the values are q = q8 * qkv_scale[0], k = k8 * qkv_scale[1], v = v8 *
