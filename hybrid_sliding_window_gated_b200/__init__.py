@@ -16,7 +16,7 @@ import os
 
 import torch
 
-__all__ = ["fwd", "fwd_halo", "fwd_fp8", "bwd", "bwd_edges", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring", "prefill_to_ring_varlen",
+__all__ = ["fwd", "fwd_halo", "fwd_fp8", "bwd", "bwd_edges", "bwd_halo", "bwd_noalloc", "bwd_workspace_size", "decode_step", "prefill_to_ring", "prefill_to_ring_varlen",
            "global_fwd", "global_decode_step", "global_decode_workspace_size",
            "get_last_device_error", "SwaError", "Params", "lib", "LIB_PATH"]
 
@@ -64,6 +64,9 @@ def lib():
         L.swa_bwd_edges.argtypes = [P] + [_vp] * 14 + [ctypes.c_int64, _vp, ctypes.c_int64, _vp,
                                                        _vp, ctypes.c_size_t, _vp]
         L.swa_bwd_edges.restype = ctypes.c_int
+        L.swa_bwd_halo.argtypes = [P] + [_vp] * 16 + [ctypes.c_int64, _vp, ctypes.c_int64, _vp,
+                                                      _vp, ctypes.c_size_t, _vp]
+        L.swa_bwd_halo.restype = ctypes.c_int
         L.swa_bwd_noalloc.argtypes = [P] + [_vp] * 15
         L.swa_bwd_noalloc.restype = ctypes.c_int
         L.swa_bwd_workspace_size.argtypes = [P]
@@ -288,6 +291,41 @@ def bwd_edges(q, k, v, g, wq, wk, lse, dO, n_lo, n_hi, *, window=128, rot_dim=42
                              _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "swa_bwd_edges")
     return grads, lo, hi
+
+
+def bwd_halo(q, k, v, g, wq, wk, lse, dO, k_halo, v_halo, pos0, n_hi=0, *, window=128,
+             rot_dim=42, rope_base=1e4, eps=1e-6, scale=0.0, workspace=None, grads=None,
+             stream=None):
+    """The backward of :func:`fwd_halo` (swa_bwd_halo).  Returns (grads, dkv_halo,
+    dkv_hi): this chunk's fp32 share of the halo keys' dk, dv [B,127,Hkv,2,128],
+    and its own last n_hi rows' dk, dv in fp32 (None when n_hi is 0)."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    p = make_params(B, T, Hq, Hkv, head_dim=D, window=window, rot_dim=rot_dim,
+                    rope_base=rope_base, eps=eps, scale=scale)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g),
+                 torch.zeros(D, dtype=torch.float32, device=q.device),
+                 torch.zeros(D, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dg, dwq, dwk = grads
+    nbytes = int(lib().swa_bwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    halo = torch.empty((B, window - 1, Hkv, 2, D), dtype=torch.float32, device=q.device)
+    hi = torch.empty((B, n_hi, Hkv, 2, D), dtype=torch.float32, device=q.device) if n_hi else None
+    nh = B * (window - 1) * Hkv * D
+    extra = {"workspace": (workspace, torch.uint8, nbytes),
+             "k_halo": (k_halo, torch.bfloat16, nh), "v_halo": (v_halo, torch.bfloat16, nh)}
+    if hi is not None:
+        extra["dkv_hi"] = (hi, torch.float32, hi.numel())
+    _need_bwd("swa_bwd_halo", q, k, v, g, wq, wk, lse, dO, grads, **extra)
+    rc = lib().swa_bwd_halo(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
+                            _ptr(wk), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                            _ptr(dwq), _ptr(dwk), _ptr(k_halo), _ptr(v_halo), int(pos0),
+                            _ptr(halo), n_hi, _ptr(hi), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    _check(rc, "swa_bwd_halo")
+    return grads, halo, hi
 
 
 def bwd_noalloc(q, k, v, g, wq, wk, lse, dO, *, window=128, rot_dim=42, rope_base=1e4,

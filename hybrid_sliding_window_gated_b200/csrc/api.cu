@@ -288,10 +288,16 @@ static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
                     const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
                     const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
                     swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk, int64_t n_lo,
-                    float* edge_lo, int64_t n_hi, float* edge_hi, void* workspace,
+                    float* edge_lo, int64_t n_hi, float* edge_hi, const swa_bf16_t* k_halo,
+                    const swa_bf16_t* v_halo, int64_t pos0, float* dkv_halo, void* workspace,
                     size_t workspace_bytes, void* stream) {
   int rc = check_params(p, false);
   if (rc != SWA_OK) return rc;
+  const bool halo = k_halo != nullptr || v_halo != nullptr || dkv_halo != nullptr;
+  if (pos0 < 0 || pos0 > (1ll << 40) ||
+      (halo && (!k_halo || !v_halo || !dkv_halo || pos0 < kWindow - 1 || !aligned32(k_halo) ||
+                !aligned16(v_halo) || (reinterpret_cast<uintptr_t>(dkv_halo) & 7u))))
+    return SWA_ERR_INVALID_ARG;
   if (n_lo < 0 || n_hi < 0 || n_lo > p->T || n_hi > p->T || (n_lo > 0 && edge_lo == nullptr) ||
       (n_hi > 0 && edge_hi == nullptr) || (reinterpret_cast<uintptr_t>(edge_lo) & 7u) ||
       (reinterpret_cast<uintptr_t>(edge_hi) & 7u))
@@ -346,6 +352,12 @@ static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
   a.ws_ek = reinterpret_cast<int*>(ws + da_bytes + 2 * d_bytes + ee_bytes);
   a.n_lo = static_cast<int>(n_lo);
   a.n_hi = static_cast<int>(n_hi);
+  a.halo = halo ? 1 : 0;
+  a.pos0 = pos0;
+  a.kv_tiles = a.tiles_per_chain + a.halo;
+  a.kv_total_tiles = static_cast<long long>(a.kv_tiles) * p->B * p->Hkv;
+  a.k_halo = k_halo;
+  a.dkv_halo = dkv_halo;
   a.edge_lo = n_lo > 0 ? edge_lo : nullptr;
   a.edge_hi = n_hi > 0 ? edge_hi : nullptr;
   rc = device_error_word(&a.err);
@@ -361,7 +373,14 @@ static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
       (rc = encode_tmap_4d(&tda, a.ws_da, D, p->Hq, T, B, 64, 1, kTile, 1,
                            CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
-  return launch_bwd(p, tq, tk, tv, tda, a, static_cast<cudaStream_t>(stream));
+  CUtensorMap tkh = tk, tvh = tv;
+  if (halo &&
+      ((rc = encode_tmap_4d(&tkh, k_halo, D, p->Hkv, kWindow - 1, B, 64, 1, kTile, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) ||
+       (rc = encode_tmap_4d(&tvh, v_halo, D, p->Hkv, kWindow - 1, B, 64, 1, kTile, 1,
+                            CU_TENSOR_MAP_SWIZZLE_128B))))
+    return rc;
+  return launch_bwd(p, tq, tk, tv, tda, tkh, tvh, a, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace swa
@@ -373,7 +392,7 @@ int swa_bwd(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k, con
             const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk, swa_bf16_t* dv, swa_bf16_t* dg,
             float* dwq, float* dwk, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, 0, nullptr, 0, nullptr,
-                  workspace, workspace_bytes, stream);
+                  nullptr, nullptr, 0, nullptr, workspace, workspace_bytes, stream);
 }
 
 int swa_bwd_edges(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
@@ -383,7 +402,18 @@ int swa_bwd_edges(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* 
                   float* dkv_lo, int64_t n_hi, float* dkv_hi, void* workspace,
                   size_t workspace_bytes, void* stream) {
   return bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, n_lo, dkv_lo, n_hi,
-                  dkv_hi, workspace, workspace_bytes, stream);
+                  dkv_hi, nullptr, nullptr, 0, nullptr, workspace, workspace_bytes, stream);
+}
+
+int swa_bwd_halo(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                 const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                 swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk,
+                 const swa_bf16_t* k_halo, const swa_bf16_t* v_halo, int64_t pos0,
+                 float* dkv_halo, int64_t n_hi, float* dkv_hi, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  return bwd_impl(p, q, k, v, g, wq, wk, lse, dO, dq, dk, dv, dg, dwq, dwk, 0, nullptr, n_hi,
+                  dkv_hi, k_halo, v_halo, pos0, dkv_halo, workspace, workspace_bytes, stream);
 }
 
 int swa_bwd_noalloc(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,

@@ -291,6 +291,44 @@ __device__ __forceinline__ void next_tile(Cursor& c, const BwdArgs& a) {
     }
   }
 }
+// Key tile t-1 exists (chain tile 0 has one with a halo: key tile -1) / must
+// be loaded (the first tile of a run, or chain tile 0 with a halo).
+__device__ __forceinline__ bool has_prev(const Cursor& c, const BwdArgs& a) {
+  return c.t > 0 || a.halo;
+}
+__device__ __forceinline__ bool need_prev(const Cursor& c, const BwdArgs& a) {
+  return has_prev(c, a) && (c.u == 0 || c.t == 0);
+}
+// The key-major pass walks key tiles -halo .. tiles-1 of each chain.
+__device__ __forceinline__ Cursor cursor_at_kv(const BwdArgs& a, int u0) {
+  Cursor c;
+  const int chain = u0 / a.kv_tiles;
+  c.t = u0 - chain * a.kv_tiles - a.halo;
+  c.b = chain / a.Hkv;
+  c.kvh = chain - c.b * a.Hkv;
+  c.u = 0;
+  return c;
+}
+__device__ __forceinline__ void next_tile_kv(Cursor& c, const BwdArgs& a) {
+  ++c.u;
+  if (++c.t == a.tiles_per_chain) {
+    c.t = -a.halo;
+    if (++c.kvh == a.Hkv) {
+      c.kvh = 0;
+      ++c.b;
+    }
+  }
+}
+// TMA of key tile j of a chain: tile -1 is the halo's rows from row -1 (that
+// row zero-filled and never in the band).
+__device__ __forceinline__ void load_key_tile(uint8_t* dst, const CUtensorMap* map,
+                                              const CUtensorMap* map_halo, uint64_t* bar, int j,
+                                              int kvh, int b) {
+  const CUtensorMap* m = j < 0 ? map_halo : map;
+  const int y = j < 0 ? -1 : j * kTile;
+  tma_load_4d(dst, m, bar, 0, kvh, y, b);
+  tma_load_4d(dst + kHalfBytes, m, bar, 64, kvh, y, b);
+}
 
 // Rotation table rot((128 j + 16 a) w_p), a = 0..7, computed by a warp.
 template <int kPairs>
@@ -298,7 +336,8 @@ __device__ __forceinline__ void fill_rot_hi(float2 (*hi)[8], int j, const BwdArg
   for (int e = lane; e < kPairs * 8; e += 32) {
     const int p = e >> 3, ai = e & 7;
     float cv, sv;
-    rope_cos_sin(static_cast<double>(j) * kTile + 16.0 * ai, a.inv_freq[p], &cv, &sv);
+    rope_cos_sin(static_cast<double>(a.pos0 + static_cast<long long>(j) * kTile) + 16.0 * ai,
+                 a.inv_freq[p], &cv, &sv);
     hi[p][ai] = make_float2(cv, sv);
   }
 }
@@ -335,7 +374,9 @@ static_assert(sizeof(SmemQ) + 1024 <= 232448, "pass 1 shared memory");
 template <int kPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_kh,
+                     const __grid_constant__ CUtensorMap tm_vh, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   SmemQ& sm = *reinterpret_cast<SmemQ*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~static_cast<uintptr_t>(1023));
@@ -430,10 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return false;
       if (lane == 0) {
         uint8_t* dst = is_k ? sm.k[s] : sm.v[s];
-        const CUtensorMap* map = is_k ? &tm_k : &tm_v;
         mbar_arrive_expect_tx(full, kTileBytes);
-        tma_load_4d(dst, map, full, 0, c.kvh, j * kTile, c.b);
-        tma_load_4d(dst + kHalfBytes, map, full, 64, c.kvh, j * kTile, c.b);
+        load_key_tile(dst, is_k ? &tm_k : &tm_v, is_k ? &tm_kh : &tm_vh, full, j, c.kvh, c.b);
       }
       if (is_k) {
         fill_rot_hi<kPairs>(sm.rot_hi[s], j, a, lane);
@@ -446,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     Cursor c = cursor_at(a, u0);
     for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
-      if (c.t > 0 && c.u == 0)
+      if (need_prev(c, a))
         ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
       ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
       for (int h = 0; h < a.G && ok; ++h, ++nq) {
@@ -486,10 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
       for (int n = 0; n < n_heads && ok; ++n) {
         const uint32_t ph = n & 1;
-        const bool hp = c.t > 0;
+        const bool hp = has_prev(c, a);
         const int sp = (c.t + 1) & 1, sc = c.t & 1;
         if (h == 0) {
-          if (c.t > 0 && c.u == 0) {
+          if (need_prev(c, a)) {
             if (!W(&sm.kready[sp], (kpar >> sp) & 1u, kSiteKReady)) break;
             kpar ^= 1u << sp;
           }
@@ -507,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    desc_kmajor(sm.k[blk ? sc : sp], kk), kIdescKK16, kk > 0);
         mma_commit(&sm.sfull);
         if (h == 0) {
-          if (c.t > 0 && c.u == 0) {
+          if (need_prev(c, a)) {
             if (!W(&sm.vready[sp], (vpar >> sp) & 1u, kSiteVFull)) break;
             vpar ^= 1u << sp;
           }
@@ -617,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int h = 0;
     for (int n = 0; n < n_heads && ok; ++n) {
       const uint32_t ph = n & 1;
-      const bool hp = c.t > 0;
+      const bool hp = has_prev(c, a);
       const int sc = c.t & 1;
       const int hq = c.kvh * a.G + h;
       const long long pos = static_cast<long long>(c.t) * kTile + row;
@@ -627,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- K' (cg 0) and V in fp16 (cg 1) of this tile's new key tiles
       if (h == 0) {
-        for (int j = (c.t > 0 && c.u == 0) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+        for (int j = need_prev(c, a) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
           const int s = j & 1;
           if (cg == 0) {
             ok = warp_wait(&sm.kfull[s], (kpar >> s) & 1u, abort, a.err, kSiteKFull);
@@ -850,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dS exponent of this query tile, from the largest |v| of its key
       // tiles: both warpgroups read the V conversion's maxima once per tile.
       if (h == 0) {
-        for (int j = (c.t > 0 && c.u == 0) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
+        for (int j = need_prev(c, a) ? c.t - 1 : c.t; j <= c.t && ok; ++j) {
           const int s = j & 1;
           ok = warp_wait(&sm.vready[s], (vpar >> s) & 1u, abort, a.err, kSiteVReady);
           vpar ^= 1u << s;
@@ -1023,13 +1062,14 @@ template <int kPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
-                      const BwdArgs a) {
+                      const __grid_constant__ CUtensorMap tm_kh,
+                      const __grid_constant__ CUtensorMap tm_vh, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                           ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u0 = static_cast<int>(a.total_tiles * blockIdx.x / gridDim.x);
-  const int u1 = static_cast<int>(a.total_tiles * (blockIdx.x + 1) / gridDim.x);
+  const int u0 = static_cast<int>(a.kv_total_tiles * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(a.kv_total_tiles * (blockIdx.x + 1) / gridDim.x);
   int n_tiles = u1 - u0;
 
   if (tid < kHeadDim) sm.dw[tid] = 0.f;
@@ -1087,8 +1127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       n_tiles = 0;
     }
   }
-  // (query tiles, heads) a key tile meets: tiles j and j+1 (if it exists) x G
-  auto n_iters = [&](const Cursor& c) { return (c.t + 1 < a.tiles_per_chain ? 2 : 1) * a.G; };
+  // (query tiles, heads) a key tile meets: tiles j and j+1 (when they exist) x G;
+  // the halo's key tile -1 meets only query tile 0
+  auto n_iters = [&](const Cursor& c) {
+    return ((c.t >= 0 ? 1 : 0) + (c.t + 1 < a.tiles_per_chain ? 1 : 0)) * a.G;
+  };
+  auto dt0 = [&](const Cursor& c) { return c.t < 0 ? 1 : 0; };  // first query tile j + dt0
 
   if (warp < 4) regs_dec<kRegsControl>();
   if (warp == 0) {
@@ -1100,17 +1144,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) w = mbar_wait_inl(bar, par, abort, a.err, site);
       return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
     };
-    Cursor c = cursor_at(a, u0);
-    for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+    Cursor c = cursor_at_kv(a, u0);
+    for (int it = 0; it < n_tiles && ok; ++it, next_tile_kv(c, a)) {
       if (it > 0 && !(ok = wait0(&sm.kvempty, (it - 1) & 1, kSiteKVEmpty))) break;
       ++nkv;
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.kfull, kTileBytes);
-        tma_load_4d(sm.k, &tm_k, &sm.kfull, 0, c.kvh, c.t * kTile, c.b);
-        tma_load_4d(sm.k + kHalfBytes, &tm_k, &sm.kfull, 64, c.kvh, c.t * kTile, c.b);
+        load_key_tile(sm.k, &tm_k, &tm_kh, &sm.kfull, c.t, c.kvh, c.b);
         mbar_arrive_expect_tx(&sm.vfull, kTileBytes);
-        tma_load_4d(sm.v, &tm_v, &sm.vfull, 0, c.kvh, c.t * kTile, c.b);
-        tma_load_4d(sm.v + kHalfBytes, &tm_v, &sm.vfull, 64, c.kvh, c.t * kTile, c.b);
+        load_key_tile(sm.v, &tm_v, &tm_vh, &sm.vfull, c.t, c.kvh, c.b);
       }
       fill_rot_hi<kPairs>(sm.rot_hi[it & 1][0], c.t, a, lane);
       fill_rot_hi<kPairs>(sm.rot_hi[it & 1][1], c.t + 1, a, lane);
@@ -1121,7 +1163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = nq & 1;
         if (nq >= 2 && !(ok = wait0(&sm.qempty[b], ((nq >> 1) - 1) & 1, kSiteQEmpty))) break;
         if (lane == 0) {
-          const int qt = c.t + i / a.G, hq = c.kvh * a.G + i % a.G;
+          const int qt = c.t + dt0(c) + i / a.G, hq = c.kvh * a.G + i % a.G;
           mbar_arrive_expect_tx(&sm.qfull[b], 2 * kTileBytes);
           tma_load_4d(sm.q[b], &tm_q, &sm.qfull[b], 0, hq, qt * kTile, c.b);
           tma_load_4d(sm.q[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, qt * kTile, c.b);
@@ -1152,8 +1194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return ok;
       };
       if (a.flags & SWA_FLAG_FORCE_TIMEOUT) W(&sm.never, 0, kSiteForced);  // for the tests
-      Cursor c = cursor_at(a, u0);
-      for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+      Cursor c = cursor_at_kv(a, u0);
+      for (int it = 0; it < n_tiles && ok; ++it, next_tile_kv(c, a)) {
         const int ni = n_iters(c);
         for (int i = 0; i < ni && ok; ++i, ++nq) {
           const int cg = nq & 1, ph = (nq >> 1) & 1;  // the pair's warpgroup, its phase
@@ -1223,8 +1265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = warp_wait(&sm.tables, 0, abort, a.err, kSiteTables);
     bool in_range = true;  // v within the fp16 staging range
     int nq = 0;
-    Cursor c = cursor_at(a, u0);
-    for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
+    Cursor c = cursor_at_kv(a, u0);
+    for (int it = 0; it < n_tiles && ok; ++it, next_tile_kv(c, a)) {
       const long long kpos = static_cast<long long>(c.t) * kTile + row;  // this thread's key
       // Common scale of this key tile's dV and dK accumulators: e_c, the
       // smallest dA exponent among the (query tile, head) pairs it meets, and
@@ -1232,18 +1274,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // j-1 .. j+1 bound every D_i the pairs bring).  Column i of P^T and dS^T
       // is scaled by 2^(e_c - e_i) <= 1 through its staged lse, so the
       // accumulators hold dV 2^e_c and dK 2^(e_c + k_c).
-      int ec = kExpLimit, kc;
+      int ec = kExpLimit, kc = kExpLimit;
       {
-        const bool next = c.t + 1 < a.tiles_per_chain;
+        const bool own = c.t >= 0, next = c.t + 1 < a.tiles_per_chain;
         const long long chain = static_cast<long long>(c.b) * a.Hkv + c.kvh;
-        kc = __ldg(a.ws_ek + chain * a.tiles_per_chain + c.t);
+        if (own) kc = min(kc, __ldg(a.ws_ek + chain * a.tiles_per_chain + c.t));
         if (next) kc = min(kc, __ldg(a.ws_ek + chain * a.tiles_per_chain + c.t + 1));
         for (int h2 = 0; h2 < a.G; ++h2) {
-          const int* e = a.ws_ee +
-                         (static_cast<long long>(c.b) * a.Hq + c.kvh * a.G + h2) * a.tiles_per_chain +
-                         c.t;
-          ec = min(ec, __ldg(e));
-          if (next) ec = min(ec, __ldg(e + 1));
+          const long long base =
+              (static_cast<long long>(c.b) * a.Hq + c.kvh * a.G + h2) * a.tiles_per_chain;
+          if (own) ec = min(ec, __ldg(a.ws_ee + base + c.t));
+          if (next) ec = min(ec, __ldg(a.ws_ee + base + c.t + 1));
         }
       }
       // ---- K'_j (cg 0) and V_j in fp16 (cg 1), published to the MMA by kvready
@@ -1261,7 +1302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < ni && ok; ++i, ++nq) {
         if ((nq & 1) != cg) continue;  // the other warpgroup's pair
         const int ph = (nq >> 1) & 1;   // phase of this warpgroup's barriers
-        const int dt = i / a.G;  // query tile j + dt
+        const int dt = dt0(c) + i / a.G;  // query tile j + dt
         const int hq = c.kvh * a.G + i % a.G;
         const long long qpos = static_cast<long long>(c.t + dt) * kTile + row;  // query row `row`
         // ---- Q'_i, and lse / D of its rows for the column-wise softmax (their
@@ -1344,11 +1385,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- dk (RoPE^-1, RMSNorm Jacobian) and dv of key tile j, over this
       // warpgroup's half of the row (the rotated dims are all in half 0)
       const long long krow = (static_cast<long long>(c.b) * a.T + kpos) * a.Hkv + c.kvh;
+      // the key's raw row: an own row, or (key tile -1) halo row `row - 1`;
+      // row 0 of the halo tile is the zero-filled row before the halo
+      const bool own_row = c.t >= 0 && kpos < a.T;
+      const long long hrow =
+          (static_cast<long long>(c.b) * (kWindow - 1) + (row - 1)) * a.Hkv + c.kvh;
+      const uint16_t* ksrc = own_row ? a.k + krow * kHeadDim
+                                     : (c.t < 0 && row >= 1 ? a.k_halo + hrow * kHeadDim : nullptr);
       uint32_t xk[32];  // this warpgroup's half of the raw k row, loaded while dK is computed
-      if (kpos < a.T) {
+      if (ksrc != nullptr) {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          ld32B(reinterpret_cast<const uint8_t*>(a.k + krow * kHeadDim) + 128 * cg + 32 * i,
+          ld32B(reinterpret_cast<const uint8_t*>(ksrc) + 128 * cg + 32 * i,
                 *reinterpret_cast<uint32_t(*)[8]>(xk + 8 * i));
       } else {
 #pragma unroll
@@ -1371,7 +1419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // partial gradients of the same keys from two calls (sequence
         // sharding) then rounds the sum once.
         float* edge = nullptr;
-        if (kpos < a.n_lo)
+        if (c.t < 0)  // the halo keys: this chunk's share, always in fp32
+          edge = row >= 1 ? a.dkv_halo + hrow * 2 * kHeadDim : nullptr;
+        else if (kpos < a.n_lo)
           edge = a.edge_lo +
                  ((static_cast<long long>(c.b) * a.n_lo + kpos) * a.Hkv + c.kvh) * 2 * kHeadDim;
         else if (kpos < a.T && kpos >= a.T - a.n_hi)
@@ -1408,7 +1458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&sm.tfree);  // dK and dV have been read from TMEM
-        if (kpos < a.T) {
+        if (own_row) {
           uint8_t* dvrow = reinterpret_cast<uint8_t*>(a.dv + krow * kHeadDim) + 128 * cg;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -1455,7 +1505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             y[2 * i] = cv.x;
             y[2 * i + 1] = cv.y;
           }
-          if (kpos < a.T) st32B(out + 32 * i4, o);
+          if (own_row) st32B(out + 32 * i4, o);
         }
         const float2 sw = warp_reduce_scatter64(y, lane);
         atomicAdd(sm.dw + 64 * cg + 2 * lane, sw.x * unk);
@@ -1476,7 +1526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int kPairs>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& tda, const BwdArgs& a, int num_sms, cudaStream_t stream) {
+                const CUtensorMap& tda, const CUtensorMap& tkh, const CUtensorMap& tvh,
+                const BwdArgs& a, int num_sms, cudaStream_t stream) {
   const size_t smem_q = sizeof(SmemQ) + 1024, smem_kv = sizeof(SmemKV) + 1024;
   static int configured_device = -1;
   int dev = 0;
@@ -1501,25 +1552,26 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
   }
   const long long grid = a.total_tiles < num_sms ? a.total_tiles : num_sms;
   int rc = launch_dependent(swa_bwd_q_kernel<kPairs>, static_cast<unsigned>(grid), kThreads,
-                            smem_q, stream, tq, tk, tv, a);
+                            smem_q, stream, tq, tk, tv, tkh, tvh, a);
   if (rc != SWA_OK) return rc;
-  return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid), kThreads, smem_kv,
-                          stream, tq, tk, tv, tda, a);
+  const long long grid_kv = a.kv_total_tiles < num_sms ? a.kv_total_tiles : num_sms;
+  return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid_kv), kThreads,
+                          smem_kv, stream, tq, tk, tv, tda, tkh, tvh, a);
 }
 
 }  // namespace bwd
 
 int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tda, const BwdArgs& a,
-               cudaStream_t stream) {
+               const CUtensorMap& tv, const CUtensorMap& tda, const CUtensorMap& tkh,
+               const CUtensorMap& tvh, const BwdArgs& a, cudaStream_t stream) {
   DeviceInfo di;
   int rc = current_device_info(&di);
   if (rc != SWA_OK) return rc;
   switch (p->rot_dim) {
-    case 0: return bwd::launch_impl<0>(tq, tk, tv, tda, a, di.num_sms, stream);
-    case 32: return bwd::launch_impl<16>(tq, tk, tv, tda, a, di.num_sms, stream);
-    case 42: return bwd::launch_impl<21>(tq, tk, tv, tda, a, di.num_sms, stream);
-    case 48: return bwd::launch_impl<24>(tq, tk, tv, tda, a, di.num_sms, stream);
+    case 0: return bwd::launch_impl<0>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
+    case 32: return bwd::launch_impl<16>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
+    case 42: return bwd::launch_impl<21>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
+    case 48: return bwd::launch_impl<24>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
     default: return SWA_ERR_UNSUPPORTED;
   }
 }

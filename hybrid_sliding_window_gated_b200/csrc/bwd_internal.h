@@ -39,6 +39,15 @@ struct BwdArgs {
   int n_lo, n_hi;
   float* edge_lo;
   float* edge_hi;
+  // A chunk with the previous chunk's halo: its W-1 keys precede row 0 (key
+  // tile -1 of each chain, the key-major pass's extra tile), and this chunk's
+  // share of their dk, dv goes to dkv_halo [B, W-1, Hkv, 2, D] fp32.
+  int halo;
+  long long pos0;            // position of row 0
+  int kv_tiles;              // key tiles per chain in the key-major pass: tiles + halo
+  long long kv_total_tiles;
+  const uint16_t* k_halo;    // [B, W-1, Hkv, D]
+  float* dkv_halo;
   int* err;
   double inv_freq[kMaxPairs];
 };
@@ -69,8 +78,9 @@ inline size_t bwd_ws_total_bytes(long long B, long long T, int Hq, int Hkv) {
          bwd_ws_ek_bytes(B, T, Hkv);
 }
 
+// tkh, tvh: the halo K and V (any valid map when a.halo is 0).
 int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tda, const BwdArgs& a,
-               cudaStream_t stream);
+               const CUtensorMap& tv, const CUtensorMap& tda, const CUtensorMap& tkh,
+               const CUtensorMap& tvh, const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace swa

@@ -8,43 +8,42 @@ Rank r holds tokens [s_r, s_r + T_r) of each of the B sequences, in rank order,
 with T_r >= W - 1 for every rank but the last.
 
 Forward: rank r receives the last W - 1 tokens of k and v from rank r - 1 and
-runs the single-GPU kernels on the chunk [halo, own tokens], whose halo query
-rows are zero and whose outputs there are dropped.  The chunk's RoPE positions
-start at 0, not at the global position: the rotation makes each score depend
-only on the difference of the two positions, so the attention is the same.
+runs swa_fwd_halo on its own tensors with that halo passed by pointer: the
+kernel loads it as the key tile before its first one.  Positions are
+chunk-relative (the first own token at W - 1, the halo before it): the
+rotation makes each score depend only on the difference of two positions, so
+the attention is the same.
 
-Backward: the same chunk, with dO = 0 on the halo rows and their lse set to
-log(i + 1), the exact normaliser of a zero query row over its i + 1 keys.  The
-halo keys' dk and dv (this rank's queries' share) go back to rank r - 1, which
-adds them to its own share of its last W - 1 rows; both shares come out of the
-kernel in fp32 (swa_bwd_edges), so the sum is rounded to bf16 once, as a
-single-GPU backward rounds it.  dq and dg need nothing from other ranks.  dwq
-and dwk are sums over tokens, so they are all-reduced over the group.
+Backward: swa_bwd_halo on the same chunk writes, in fp32, this rank's share of
+the halo keys' dk and dv; it goes back to rank r - 1, which asked its own
+call for its last W - 1 rows in fp32 as well, adds the two shares and rounds
+once, as a single-GPU backward rounds those rows.  dq and dg need nothing
+from other ranks.  dwq and dwk are sums over tokens, so they are all-reduced
+over the group.
 
 Exchanges are point-to-point sends to the next (forward) or previous
 (backward) rank through torch.distributed (NCCL between GPUs).  One rank's
 step, given the halo it received, is :func:`rank_fwd` / :func:`rank_bwd`, which
-need no process group.
-
-Cost: the kernels take one contiguous [B, T, H, D] tensor per input, so each
-rank assembles its chunk by copying q, k, v and g (and dO in the backward)
-behind the halo rows, and copies o, lse, dq, dk, dv and dg out of the chunk
-again.  Those copies move about as many bytes as the forward kernel itself;
-the halo rows' own compute (W - 1 query rows per rank) is small beside them.
-Needs eps > 0: the halo query rows are zero.
+need no process group.  No input or output is copied: the halo arrives in its
+own [B, W - 1, Hkv, D] buffer, and the per-rank traffic beyond the kernels'
+own is the halo (W - 1 rows of k and v in, their fp32 gradients back).
 """
 import torch
 import torch.distributed as dist
 
 from . import bwd as _kernel_bwd
 from . import bwd_edges as _kernel_bwd_edges
+from . import bwd_halo as _kernel_bwd_halo
 from . import fwd as _kernel_fwd
+from . import fwd_halo as _kernel_fwd_halo
 
 # The per-rank computation: the library's kernels.  (The CPU tests of the
 # exchange logic replace these with a host implementation.)
 _local_fwd = _kernel_fwd
+_local_fwd_halo = _kernel_fwd_halo
 _local_bwd = _kernel_bwd
 _local_bwd_edges = _kernel_bwd_edges
+_local_bwd_halo = _kernel_bwd_halo
 
 
 def _ranks(group):
@@ -73,41 +72,19 @@ def _exchange(send, recv_like, to_next, group):
     return got
 
 
-def _halo_in(k, v, halo, eps, group):
+def _halo_in(k, v, halo, group):
     rank, world, _ = _ranks(group)
     if world == 1:
         return None
-    # Both preconditions are agreed by every rank before any exchange, so
-    # that all of them raise together rather than one waiting on a send.
-    ok = torch.tensor([int(rank + 1 == world or k.shape[1] >= halo), int(eps > 0.0)],
-                      dtype=torch.int32, device=k.device)
+    # The precondition is agreed by every rank before any exchange, so that
+    # all of them raise together rather than one waiting on a send.
+    ok = torch.tensor([int(rank + 1 == world or k.shape[1] >= halo)], dtype=torch.int32,
+                      device=k.device)
     dist.all_reduce(ok, op=dist.ReduceOp.MIN, group=group)
-    if int(ok[0].item()) == 0:
+    if int(ok.item()) == 0:
         raise ValueError(f"every rank but the last must hold at least {halo} tokens")
-    _check_eps(eps if int(ok[1].item()) else 0.0)
     tails = [k[:, -halo:], v[:, -halo:]]
     return _exchange(tails, tails, True, group)
-
-
-def _with_halo(x, halo_rows):
-    """[B, T, H, D] -> [B, len + T, H, D] with `halo_rows` (or zeros) in front.
-    This copies x: the kernels take one contiguous [B, T, H, D] tensor per
-    input, so the chunk is assembled here."""
-    return torch.cat([halo_rows, x], dim=1)
-
-
-def halo_lse(B, Hq, n, device):
-    """lse of n zero query rows at chunk positions 0..n-1: log(i + 1)."""
-    lse = torch.log(torch.arange(1, n + 1, dtype=torch.float64)).to(torch.float32)
-    return lse.to(device).view(1, 1, n).expand(B, Hq, n).contiguous()
-
-
-def _check_eps(eps):
-    # The halo query rows are zero: with eps = 0 their RMSNorm divides 0 by 0,
-    # and the NaN would reach the halo keys' dk and dv and, through the
-    # all-reduce, dwq and dwk on every rank.
-    if not eps > 0.0:
-        raise ValueError("sequence sharding needs eps > 0 (its halo query rows are zero)")
 
 
 def rank_fwd(q, k, v, g, wq, wk, halo, *, window=128, rot_dim=42, rope_base=1e4, eps=1e-6,
@@ -117,14 +94,9 @@ def rank_fwd(q, k, v, g, wq, wk, halo, *, window=128, rot_dim=42, rope_base=1e4,
     kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
     if halo is None:
         return _local_fwd(q, k, v, g, wq, wk, want_lse=want_lse, **kw)
-    _check_eps(eps)
     hk, hv = halo
-    n = hk.shape[1]
-    zq = torch.zeros((q.shape[0], n) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
-    o, lse = _local_fwd(_with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv),
-                        _with_halo(g, zq), wq, wk, want_lse=True, **kw)
-    o = o[:, n:].contiguous()
-    return (o, lse[:, :, n:].contiguous()) if want_lse else o
+    return _local_fwd_halo(q, k, v, g, wq, wk, hk.contiguous(), hv.contiguous(), window - 1,
+                           want_lse=want_lse, **kw)
 
 
 def rank_bwd(q, k, v, g, wq, wk, lse, dO, halo, *, tail=0, window=128, rot_dim=42,
@@ -137,23 +109,15 @@ def rank_bwd(q, k, v, g, wq, wk, lse, dO, halo, *, tail=0, window=128, rot_dim=4
     form (None when tail is 0), to which the next rank's `back` is added by
     :func:`add_back`.  dwq and dwk are this rank's share."""
     kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
-    n = 0 if halo is None else halo[0].shape[1]
     if halo is None and tail == 0:
         return tuple(_local_bwd(q, k, v, g, wq, wk, lse, dO, **kw)) + (None, None)
     if halo is None:
         grads, _, own = _local_bwd_edges(q, k, v, g, wq, wk, lse, dO, 0, tail, **kw)
         return tuple(grads) + (None, own)
-    _check_eps(eps)
     hk, hv = halo
-    B, Hq = q.shape[0], q.shape[2]
-    zq = torch.zeros((B, n) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
-    lse_c = torch.cat([halo_lse(B, Hq, n, lse.device).to(lse.dtype), lse], dim=2)
-    grads, back, own = _local_bwd_edges(
-        _with_halo(q, zq), _with_halo(k, hk), _with_halo(v, hv), _with_halo(g, zq), wq, wk,
-        lse_c, _with_halo(dO, zq), n, tail, **kw)
-    dq, dk, dv, dg, dwq, dwk = grads
-    dq, dk, dv, dg = (x[:, n:].contiguous() for x in (dq, dk, dv, dg))
-    return dq, dk, dv, dg, dwq, dwk, back, own
+    grads, back, own = _local_bwd_halo(q, k, v, g, wq, wk, lse, dO, hk.contiguous(),
+                                       hv.contiguous(), window - 1, tail, **kw)
+    return tuple(grads) + (back, own)
 
 
 def add_back(dk, dv, own, back):
@@ -172,7 +136,7 @@ def fwd(q, k, v, g, wq, wk, *, group=None, window=128, rot_dim=42, rope_base=1e4
         scale=0.0, want_lse=False):
     """o (and lse [B, Hq, T_r]) for this rank's tokens.  q, g: [B, T_r, Hq, D];
     k, v: [B, T_r, Hkv, D]."""
-    halo = _halo_in(k, v, window - 1, eps, group)
+    halo = _halo_in(k, v, window - 1, group)
     return rank_fwd(q, k, v, g, wq, wk, halo, window=window, rot_dim=rot_dim,
                     rope_base=rope_base, eps=eps, scale=scale, want_lse=want_lse)
 
@@ -184,7 +148,7 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, group=None, window=128, rot_dim=42, rope
     ``reduce_weight_grads``, else this rank's share."""
     halo_n = window - 1
     rank, world, _ = _ranks(group)
-    halo = _halo_in(k, v, halo_n, eps, group)
+    halo = _halo_in(k, v, halo_n, group)
     tail = halo_n if rank + 1 < world else 0
     dq, dk, dv, dg, dwq, dwk, back, own = rank_bwd(q, k, v, g, wq, wk, lse, dO, halo, tail=tail,
                                                    window=window, rot_dim=rot_dim,
@@ -204,4 +168,4 @@ def bwd(q, k, v, g, wq, wk, lse, dO, *, group=None, window=128, rot_dim=42, rope
     return dq, dk, dv, dg, dwq, dwk
 
 
-__all__ = ["fwd", "bwd", "rank_fwd", "rank_bwd", "add_back", "halo_lse"]
+__all__ = ["fwd", "bwd", "rank_fwd", "rank_bwd", "add_back"]

@@ -183,6 +183,26 @@ int swa_bwd_edges(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* 
                   float* dkv_lo, int64_t n_hi, float* dkv_hi, void* workspace,
                   size_t workspace_bytes, void* stream);
 
+/*
+ * The backward of swa_fwd_halo: the chunk's own rows as in swa_bwd, with the
+ * halo k_halo, v_halo [B, 127, Hkv, D] and pos0 as given to the forward
+ * (both halos set, pos0 >= 127; k_halo 32-byte aligned, its rows move in
+ * 32-byte accesses).  Writes, in fp32, this chunk's share of the gradient
+ * of the halo keys to dkv_halo [B, 127, Hkv, 2, D] (dk, then dv; 8-byte
+ * aligned): the previous chunk adds it to its own share of its last 127 rows
+ * (the n_hi rows it asked for here in dkv_hi, as swa_bwd_edges does) and
+ * rounds the sum once.  dwq and dwk take this chunk's share, the halo keys'
+ * included (the weight gradients are linear in the incoming dk' and dq', so
+ * the chunks' shares sum).  Other arguments and results as swa_bwd_edges.
+ */
+int swa_bwd_halo(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t* k,
+                 const swa_bf16_t* v, const swa_bf16_t* g, const float* wq, const float* wk,
+                 const float* lse, const swa_bf16_t* dO, swa_bf16_t* dq, swa_bf16_t* dk,
+                 swa_bf16_t* dv, swa_bf16_t* dg, float* dwq, float* dwk,
+                 const swa_bf16_t* k_halo, const swa_bf16_t* v_halo, int64_t pos0,
+                 float* dkv_halo, int64_t n_hi, float* dkv_hi, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
 /* Bytes of scratch swa_bwd needs for these parameters (0 if unsupported). */
 size_t swa_bwd_workspace_size(const swa_params_t* p);
 

@@ -63,3 +63,42 @@ def test_forward_halo_argument_checks():
     hk = torch.zeros((1, W - 1, 1, 128), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(swa.SwaError):  # a halo needs pos0 >= 127
         swa.fwd_halo(d["q"], d["k"], d["v"], d["g"], d["wq"], d["wk"], hk, hk, 100)
+
+
+@pytest.mark.parametrize("B,L,s,Hq,Hkv", [(1, 500, 200, 4, 1), (2, 900, 300, 8, 2),
+                                          (1, 700, 127, 3, 1), (2, 1400, 1000, 32, 8)])
+def test_backward_two_chunks_with_halo_equal_the_whole(B, L, s, Hq, Hkv):
+    """A sequence split at s: the first chunk's backward gives its own rows
+    (its last 127 keys' dk, dv in fp32 too); the second chunk's halo backward
+    gives its rows and, in fp32, its share of those 127 keys.  The two shares
+    summed and rounded once, and every other row, against the oracle's
+    backward of the whole; the weight gradients as the sum of the shares."""
+    cfg = workloads.custom_prefill(B, L, Hq, Hkv, base=1e4, seed=97 + s, backward=True)
+    inp = workloads.prefill_inputs(cfg, with_grad_out=True)
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    a = {x: d[x][:, :s].contiguous() for x in ("q", "k", "v", "g", "dO")}
+    b = {x: d[x][:, s:].contiguous() for x in ("q", "k", "v", "g", "dO")}
+    hk, hv = a["k"][:, -(W - 1):].contiguous(), a["v"][:, -(W - 1):].contiguous()
+    oa, la = swa.fwd(a["q"], a["k"], a["v"], a["g"], d["wq"], d["wk"], want_lse=True)
+    ob, lb = swa.fwd_halo(b["q"], b["k"], b["v"], b["g"], d["wq"], d["wk"], hk, hv, W - 1,
+                          want_lse=True)
+    ga, _, tail = swa.bwd_edges(a["q"], a["k"], a["v"], a["g"], d["wq"], d["wk"], la, a["dO"],
+                                0, W - 1)
+    gb, back, _ = swa.bwd_halo(b["q"], b["k"], b["v"], b["g"], d["wq"], d["wk"], lb, b["dO"],
+                               hk, hv, W - 1)
+    torch.cuda.synchronize()
+    assert swa.get_last_device_error()[0] == swa.OK
+    tot = tail + back
+    dk = torch.cat([ga[1][:, :s - (W - 1)], tot[:, :, :, 0].bfloat16(), gb[1]], dim=1)
+    dv = torch.cat([ga[2][:, :s - (W - 1)], tot[:, :, :, 1].bfloat16(), gb[2]], dim=1)
+    dq = torch.cat([ga[0], gb[0]], dim=1)
+    dg = torch.cat([ga[3], gb[3]], dim=1)
+    ref = oracle.bwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]), f64(inp["wq"]),
+                     f64(inp["wk"]), f64(inp["dO"]), W=W, R=42, base=1e4, eps=1e-6)
+    for name, x, r in (("dq", dq, ref[0]), ("dk", dk, ref[1]), ("dv", dv, ref[2]),
+                       ("dg", dg, ref[3])):
+        assert_parity(to_f64(x), r, f"stitched {name}")
+    for name, i in (("dwq", 4), ("dwk", 5)):
+        got = to_f64(ga[i]) + to_f64(gb[i])
+        fro = np.sqrt(((got - ref[i]) ** 2).sum() / (ref[i] ** 2).sum())
+        assert fro <= 5e-3, (name, fro)

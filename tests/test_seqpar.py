@@ -55,9 +55,41 @@ def host_bwd_edges(q, k, v, g, wq, wk, lse, dO, n_lo, n_hi, **kw):
     return grads, (dkv[:, :n_lo] if n_lo else None), (dkv[:, T - n_hi:] if n_hi else None)
 
 
+def host_fwd_halo(q, k, v, g, wq, wk, hk, hv, pos0, *, window, rot_dim, rope_base, eps, scale,
+                  want_lse):
+    """The chunk's rows at positions pos0 .., its keys the halo then its own."""
+    n = lambda t: t.numpy()
+    kk, vv = torch.cat([hk, k], dim=1), torch.cat([hv, v], dim=1)
+    o, lse = oracle.fwd(n(q), n(kk), n(vv), n(g), n(wq), n(wk), W=window, R=rot_dim,
+                        base=rope_base, eps=eps, scale=scale, pos0=pos0 - (window - 1),
+                        q_begin=window - 1)
+    o, lse = torch.from_numpy(o), torch.from_numpy(lse).permute(0, 2, 1).contiguous()
+    return (o, lse) if want_lse else o
+
+
+def host_bwd_halo(q, k, v, g, wq, wk, lse, dO, hk, hv, pos0, n_hi, *, window, rot_dim, rope_base,
+                  eps, scale):
+    """The exact backward of host_fwd_halo: the oracle's backward over the
+    chunk with its halo rows in front (positions from 0, so pos0 = W - 1),
+    their query, gate and upstream-gradient rows zero, which adds nothing."""
+    assert pos0 == window - 1
+    n = window - 1
+    z = torch.zeros((q.shape[0], n) + tuple(q.shape[2:]), dtype=q.dtype)
+    cat = lambda a, b: torch.cat([a, b], dim=1)
+    kw = dict(window=window, rot_dim=rot_dim, rope_base=rope_base, eps=eps, scale=scale)
+    dq, dk, dv, dg, dwq, dwk = host_bwd(cat(z, q), cat(hk, k), cat(hv, v), cat(z, g), wq, wk,
+                                        None, cat(z, dO), **kw)
+    dkv = torch.stack([dk, dv], dim=3)
+    T = q.shape[1]
+    back = dkv[:, :n]
+    own = dkv[:, n + T - n_hi:] if n_hi else None
+    return (dq[:, n:], dk[:, n:], dv[:, n:], dg[:, n:], dwq, dwk), back, own
+
+
 def _use_host(seqpar):
     seqpar._local_fwd, seqpar._local_bwd = host_fwd, host_bwd
     seqpar._local_bwd_edges = host_bwd_edges
+    seqpar._local_fwd_halo, seqpar._local_bwd_halo = host_fwd_halo, host_bwd_halo
 
 
 def _rank_main(rank, world, port, out):
@@ -104,20 +136,6 @@ def test_three_ranks_equal_the_whole_sequence():
         np.testing.assert_allclose(r[7], g_ref[5], rtol=1e-9, atol=1e-9, err_msg="dwk")
 
 
-def test_halo_lse_is_the_normaliser_of_zero_query_rows():
-    """The lse the backward gives the halo rows: a zero query row scores 0
-    against each of its i + 1 keys, so its normaliser is log(i + 1)."""
-    from hybrid_sliding_window_gated_b200 import seqpar
-    x = {k: v.numpy() for k, v in _inputs().items()}
-    T = 300
-    q = x["q"][:, :T].copy()
-    q[:, :W - 1] = 0.0
-    _, lse = oracle.fwd(q, x["k"][:, :T], x["v"][:, :T], x["g"][:, :T], x["wq"], x["wk"],
-                        W=W, R=R, base=BASE, eps=EPS)
-    got = seqpar.halo_lse(B, HQ, W - 1, "cpu").double().numpy()
-    np.testing.assert_allclose(got, lse[:, :W - 1].transpose(0, 2, 1), rtol=0, atol=1e-6)
-
-
 def test_single_process_calls_the_kernels_directly(monkeypatch):
     from hybrid_sliding_window_gated_b200 import seqpar
     calls = []
@@ -156,35 +174,9 @@ def test_the_product_path_calls_the_kernel_wrappers():
     from hybrid_sliding_window_gated_b200 import seqpar
     assert seqpar._local_fwd is swa.fwd and seqpar._local_bwd is swa.bwd
     assert seqpar._local_bwd_edges is swa.bwd_edges
+    assert seqpar._local_fwd_halo is swa.fwd_halo and seqpar._local_bwd_halo is swa.bwd_halo
     src = open(seqpar.__file__).read()
     assert "oracle" not in src
-
-
-def _eps_rank_main(rank, world, port, out):
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
-    try:
-        from hybrid_sliding_window_gated_b200 import seqpar
-        seqpar._local_fwd = host_fwd
-        x = {k: (v[:, :150].contiguous() if v.dim() == 4 else v) for k, v in _inputs().items()}
-        try:
-            seqpar.fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=W, rot_dim=R,
-                       eps=0.0)
-            out[rank] = "returned"
-        except ValueError:
-            out[rank] = "raised"
-    finally:
-        dist.destroy_process_group()
-
-
-def test_eps_zero_is_refused_on_every_rank():
-    """The halo query rows are zero, so eps = 0 would make their RMSNorm NaN,
-    and the NaN would spread to dk, dv and the all-reduced weight gradients."""
-    with mp.get_context("spawn").Manager() as mgr:
-        out = mgr.dict()
-        mp.spawn(_eps_rank_main, args=(2, _free_port(), out), nprocs=2, join=True)
-        assert dict(out) == {0: "raised", 1: "raised"}
 
 
 def test_rank_steps_without_a_process_group():
@@ -192,7 +184,8 @@ def test_rank_steps_without_a_process_group():
     the oracle on the whole sequences (the host computation standing in for
     the kernels, as above)."""
     from hybrid_sliding_window_gated_b200 import seqpar
-    old = seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges
+    old = (seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges, seqpar._local_fwd_halo,
+           seqpar._local_bwd_halo)
     _use_host(seqpar)
     try:
         x = _inputs()
@@ -213,7 +206,8 @@ def test_rank_steps_without_a_process_group():
         for r in range(1, len(grads)):
             seqpar.add_back(grads[r - 1][1], grads[r - 1][2], grads[r - 1][7], grads[r][6])
     finally:
-        seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges = old
+        (seqpar._local_fwd, seqpar._local_bwd, seqpar._local_bwd_edges, seqpar._local_fwd_halo,
+         seqpar._local_bwd_halo) = old
     n = {k: v.numpy() for k, v in x.items()}
     o_ref, _ = oracle.fwd(n["q"], n["k"], n["v"], n["g"], n["wq"], n["wk"], W=W, R=R, base=BASE,
                           eps=EPS)
