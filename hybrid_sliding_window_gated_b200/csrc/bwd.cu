@@ -253,10 +253,10 @@ __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane
 }
 
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
-  return make_desc_sw128(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+  return desc_advance(make_desc_sw128(smem_u32(tile), 16, 1024), (kk >> 2) * kHalfBytes + (kk & 3) * 32);
 }
 __device__ __forceinline__ uint64_t desc_mn(const uint8_t* tile, int kk) {
-  return make_desc_sw128(smem_u32(tile) + kk * 2048, kHalfBytes, 1024);
+  return desc_advance(make_desc_sw128(smem_u32(tile), kHalfBytes, 1024), kk * 2048);
 }
 constexpr uint32_t kIdescKK = make_idesc_bf16(128, 128, false, false);  // A, B K-major
 constexpr uint32_t kIdescKM = make_idesc_bf16(128, 128, false, true);   // B MN-major

@@ -137,10 +137,10 @@ __device__ __forceinline__ float2 cmul(float2 x, float2 y) {
   return make_float2(x.x * y.x - x.y * y.y, x.x * y.y + x.y * y.x);
 }
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
-  return make_desc_sw128(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+  return desc_advance(make_desc_sw128(smem_u32(tile), 16, 1024), (kk >> 2) * kHalfBytes + (kk & 3) * 32);
 }
 __device__ __forceinline__ uint64_t desc_v(const uint8_t* tile, int kk) {
-  return make_desc_sw128(smem_u32(tile) + kk * 2048, kHalfBytes, 1024);
+  return desc_advance(make_desc_sw128(smem_u32(tile), kHalfBytes, 1024), kk * 2048);
 }
 constexpr uint32_t kIdescQK = make_idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 128, false, true);

@@ -309,6 +309,15 @@ __device__ __forceinline__ uint64_t make_desc_sw128(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// The same descriptor with its start address advanced by `bytes` (a multiple
+// of 16 that keeps the operand inside shared memory).  The address field is
+// the low 14 bits, which cannot carry, so only the low word changes: one add
+// per MMA instead of rebuilding the descriptor.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = static_cast<uint32_t>(d) + (bytes >> 4);
+  return (d & 0xFFFFFFFF00000000ull) | lo;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn_major,
                                                        bool b_mn_major) {
