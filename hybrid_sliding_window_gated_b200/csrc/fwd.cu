@@ -94,7 +94,9 @@ constexpr int kHalfBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = 16 KiB (one 
 constexpr int kTileBytes = 2 * kHalfBytes;  // a full 128 x 128 bf16 tile
 
 struct alignas(1024) Smem {
-  uint8_t k[2][kTileBytes];
+  // K ring, [half][slot]: per 64-dim half the two slots' 128 rows lie one
+  // after the other, so one N = 256 MMA per k-step reads both key tiles.
+  uint8_t k[2][2][kHalfBytes];
   uint8_t v[2][kTileBytes];
   uint8_t q[3][kTileBytes];  // head n uses slot n % 3: Q(n), then g(n), then o(n)
   float2 rot_tile[2][kMaxPairs];  // rot(128 j * w_p) of the K tile in each slot
@@ -280,10 +282,8 @@ __device__ __forceinline__ void scale_chunks(uint8_t* h0, uint8_t* h1, int row, 
 // K row: k'' = [RoPE(k / rms(k) * wk) on the rotated dims; k / rms(k) * wk * wq
 // elsewhere].
 template <int kPairs>
-__device__ __forceinline__ void transform_k_row(uint8_t* tile, int row, const Smem& sm, int kslot,
-                                                const RowRot<kPairs>& rr, float eps) {
-  uint8_t* h0 = tile;
-  uint8_t* h1 = tile + kHalfBytes;
+__device__ __forceinline__ void transform_k_row(uint8_t* h0, uint8_t* h1, int row, const Smem& sm,
+                                                int kslot, const RowRot<kPairs>& rr, float eps) {
   const float rinv = rsqrtf(row_sumsq(h0, h1, row) * (1.0f / kHeadDim) + eps);
   constexpr int kRopeChunks = (2 * kPairs + 7) / 8;
   if constexpr (kRopeChunks > 0)
@@ -329,10 +329,11 @@ __device__ __forceinline__ void e4m3x16_to_f32(const uint4& u, float (&x)[16]) {
   }
 }
 
-__device__ __forceinline__ void load_row_fp8(const uint8_t* tile, int row, uint4 (&u)[8]) {
+// The FP8 row as it landed: 128 bytes in the swizzled 16 KiB box at `src`.
+__device__ __forceinline__ void load_row_fp8(const uint8_t* src, int row, uint4 (&u)[8]) {
 #pragma unroll
   for (int c = 0; c < 8; ++c)
-    u[c] = *reinterpret_cast<const uint4*>(tile + kHalfBytes + sw_off(row, c));
+    u[c] = *reinterpret_cast<const uint4*>(src + sw_off(row, c));
 }
 
 __device__ __forceinline__ float row_sumsq_fp8(const uint4 (&u)[8]) {
@@ -351,9 +352,8 @@ __device__ __forceinline__ float row_sumsq_fp8(const uint4 (&u)[8]) {
   return s2.x + s2.y;
 }
 
-// Write dims [64 h, 64 h + 64) of a row, given as floats, as bf16 half h.
-__device__ __forceinline__ void store_half_bf16(uint8_t* tile, int row, int h, const float* x) {
-  uint8_t* hp = tile + h * kHalfBytes;
+// Write 64 dims of a row, given as floats, as bf16 into the half at `hp`.
+__device__ __forceinline__ void store_half_bf16(uint8_t* hp, int row, const float* x) {
 #pragma unroll
   for (int c = 0; c < 8; ++c)
     *reinterpret_cast<uint4*>(hp + sw_off(row, c)) = pack8(x + 8 * c);
@@ -367,11 +367,11 @@ __device__ __forceinline__ float fp8_row_factor(float sumsq8, float s, float eps
 
 // K row from FP8: k'' as transform_k_row writes it, from x8 and the factor.
 template <int kPairs>
-__device__ __forceinline__ void transform_k_row_fp8(uint8_t* tile, int row, const Smem& sm,
-                                                    int kslot, const RowRot<kPairs>& rr,
-                                                    float eps) {
+__device__ __forceinline__ void transform_k_row_fp8(uint8_t* h0, uint8_t* h1, int row,
+                                                    const Smem& sm, int kslot,
+                                                    const RowRot<kPairs>& rr, float eps) {
   uint4 u[8];
-  load_row_fp8(tile, row, u);
+  load_row_fp8(h1, row, u);  // the FP8 box lands in the second half's bytes
   const float f = fp8_row_factor(row_sumsq_fp8(u), sm.sc[1], eps);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -395,7 +395,7 @@ __device__ __forceinline__ void transform_k_row_fp8(uint8_t* tile, int row, cons
         x[p + kPairs] = b0 * t.x + a0 * t.y;
       }
     }
-    store_half_bf16(tile, row, h, x);
+    store_half_bf16(h == 0 ? h0 : h1, row, x);
   }
 }
 
@@ -407,7 +407,7 @@ __device__ __forceinline__ float transform_q_row_fp8(uint8_t* tile, int row, con
                                                      int kslot, const RowRot<kPairs>& rr,
                                                      float eps) {
   uint4 u[8];
-  load_row_fp8(tile, row, u);
+  load_row_fp8(tile + kHalfBytes, row, u);
   const float f = fp8_row_factor(row_sumsq_fp8(u), sm.sc[0], eps);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -431,7 +431,7 @@ __device__ __forceinline__ float transform_q_row_fp8(uint8_t* tile, int row, con
         x[p + kPairs] = b0 * t.x + a0 * t.y;
       }
     }
-    store_half_bf16(tile, row, h, x);
+    store_half_bf16(tile + h * kHalfBytes, row, x);
   }
   return f;
 }
@@ -439,7 +439,7 @@ __device__ __forceinline__ float transform_q_row_fp8(uint8_t* tile, int row, con
 // V row from FP8: x8 exactly as bf16 (the factor s_v enters with 1/l).
 __device__ __forceinline__ void expand_v_row_fp8(uint8_t* tile, int row) {
   uint4 u[8];
-  load_row_fp8(tile, row, u);
+  load_row_fp8(tile + kHalfBytes, row, u);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float x[64];
@@ -450,7 +450,7 @@ __device__ __forceinline__ void expand_v_row_fp8(uint8_t* tile, int row) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) x[16 * c + i] = y[i];
     }
-    store_half_bf16(tile, row, h, x);
+    store_half_bf16(tile + h * kHalfBytes, row, x);
   }
 }
 
@@ -463,7 +463,12 @@ __device__ __forceinline__ uint64_t desc_v(const uint8_t* tile, int kk) {
   return make_desc_sw128(smem_u32(tile) + kk * 2048, kHalfBytes, 1024);
 }
 
-constexpr uint32_t kIdescQK = make_idesc_bf16(128, 128, false, false);
+constexpr uint32_t kIdescQK = make_idesc_bf16(128, 256, false, false);  // both key tiles at once
+// K-major descriptor of k-step kk of the K ring: 256 rows (slot 0's keys,
+// then slot 1's) of one 64-dim half.
+__device__ __forceinline__ uint64_t desc_kring(const uint8_t (*khalf)[2][kHalfBytes], int kk) {
+  return make_desc_sw128(smem_u32(khalf[kk >> 2][0]) + (kk & 3) * 32, 16, 1024);
+}
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, 128, false, true);
 
 // Phase bookkeeping for a 2-slot ring: bit s of `par` is the parity of the
@@ -574,14 +579,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           if (kFp8) {  // one 16 KiB box of bytes, into the slot's upper half
             mbar_arrive_expect_tx(&sm.kfull[s], kHalfBytes);
-            tma_load_4d(sm.k[s] + kHalfBytes, &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
+            tma_load_4d(sm.k[1][s], &tm_k, &sm.kfull[s], 0, c.kvh, j * kTile, c.b);
           } else {
             // key tile -1: the halo's 127 rows, from row -1 (zero-filled, never in the band)
             const CUtensorMap* map = j < 0 ? &tm_kh : &tm_k;
             const int y = j < 0 ? -1 : j * kTile;
             mbar_arrive_expect_tx(&sm.kfull[s], kTileBytes);
-            tma_load_4d(sm.k[s], map, &sm.kfull[s], 0, c.kvh, y, c.b);
-            tma_load_4d(sm.k[s] + kHalfBytes, map, &sm.kfull[s], 64, c.kvh, y, c.b);
+            tma_load_4d(sm.k[0][s], map, &sm.kfull[s], 0, c.kvh, y, c.b);
+            tma_load_4d(sm.k[1][s], map, &sm.kfull[s], 64, c.kvh, y, c.b);
           }
         }
         // rot(128 j w_p) for this tile, then the second arrive on kfull.
@@ -688,17 +693,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cnt > 0 && !mbar_wait_inl(&sm.tfree[r], (cnt - 1) & 1, abort, a.err, kSiteTFree)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s_base = tmem + r * 256;
-          const bool hp = has_prev(cq, a);
-          for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
-            const uint8_t* kt = sm.k[blk == 0 ? sp : sc];
+          // S = Q' [K slot 0; K slot 1]^T: columns 0..127 hold the keys of the
+          // tile in slot 0, 128..255 those in slot 1 (key tile t-1 and t in
+          // either order; without a tile t-1 that half is never read).
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(s_base + blk * 128, desc_kmajor(sm.q[m % 3], kk), desc_kmajor(kt, kk), kIdescQK,
-                     kk > 0);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(s_base, desc_kmajor(sm.q[m % 3], kk), desc_kring(sm.k, kk), kIdescQK, kk > 0);
           mma_commit(&sm.sfull[r]);
           if (cq.h == a.G - 1) {
-            if (hp) mma_commit(&sm.kempty[sp]);
+            if (has_prev(cq, a)) mma_commit(&sm.kempty[sp]);
             if (seg_last(cq, a, n_tiles)) mma_commit(&sm.kempty[sc]);
           }
         }
@@ -722,10 +725,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool hp = has_prev(cp, a);
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
-            const uint8_t* vt = sm.v[blk == 0 ? sp : sc];
+            const int slot = blk == 0 ? sp : sc;  // P sits over the S columns of its slot
+            const uint8_t* vt = sm.v[slot];
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              mma_ts(p_base + 128, p_base + blk * 64 + kk * 8, desc_v(vt, kk), kIdescPV, acc);
+              mma_ts(p_base + 128, p_base + slot * 64 + kk * 8, desc_v(vt, kk), kIdescPV, acc);
               acc = 1;
             }
           }
@@ -787,9 +791,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (transform_last && acct == upto) {
             if (!mbar_wait_inl(&sm.kfull[s], kr.parity(s), abort, a.err, kSiteKFull)) return false;
             if constexpr (kFp8)
-              transform_k_row_fp8<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
+              transform_k_row_fp8<kPairs>(sm.k[0][s], sm.k[1][s], row, sm, s, rr, a.eps);
             else
-              transform_k_row<kPairs>(sm.k[s], row, sm, s, rr, a.eps);
+              transform_k_row<kPairs>(sm.k[0][s], sm.k[1][s], row, sm, s, rr, a.eps);
             fence_proxy_async_smem();
             mbar_arrive(&sm.kready[s]);
             if constexpr (kFp8) {  // V of the same tile (vfull has the K ring's phase)
@@ -856,6 +860,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The MMA saw unnormalised q rows; 1/rms(q) enters with the softmax scale.
       const float rs = sl2 * rinv;
       const bool hp = has_prev(c, a);
+      // Key tile t sits in K slot t & 1 and key tile t-1 (logical block 0) in
+      // the other: block b's S is in columns slot_of(b) * 128, its P goes over
+      // columns slot_of(b) * 64.
+      const int st = c.t & 1;
+      auto slot_of = [&](int blk) { return blk == 1 ? st : st ^ 1; };
       float ms = bound;
       if (exact) {
         // Row maximum over the band: key tile t-1 gives columns c > row, key
@@ -868,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool none = blk == 0 ? (pc < wq4) : (pc > wq4);
             if (none) continue;
             uint32_t v[32];
-            tmem_ld32(t_row + blk * 128 + pc * 32, v);
+            tmem_ld32(t_row + slot_of(blk) * 128 + pc * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -880,13 +889,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ms = m * rs;
       }
       // P = exp2(s * rs - ms), packed bf16 over the first 128 columns of the
-      // region; fp32 row sum.  Key tile t-1 (columns 0..127) keeps columns
-      // c > row, key tile t (128..255) columns c <= row.  For this warp's 32
-      // rows, 32-column chunk pc of key tile t-1 is empty for pc < wq4 and
-      // full for pc > wq4; of key tile t full for pc < wq4 and empty for
-      // pc > wq4; only pc == wq4 straddles the band edge.
+      // region; fp32 row sum.  Key tile t-1 keeps columns c > row, key tile t
+      // columns c <= row.  For this warp's 32 rows, 32-column chunk pc of key
+      // tile t-1 is empty for pc < wq4 and full for pc > wq4; of key tile t
+      // full for pc < wq4 and empty for pc > wq4; only pc == wq4 straddles
+      // the band edge.  The tile in slot 0 is taken first: the other tile's
+      // P lands over S columns 64..127 of slot 0, which must be read by then.
       const int na = hp ? 4 - wq4 : 0;  // chunks of key tile t-1 in the band
-      const int nch = na + wq4 + 1;     // plus those of key tile t
+      const int nt = wq4 + 1;           // chunks of key tile t
+      const int nch = na + nt;
+      const int b_first = st == 0 ? 1 : 0;  // the logical tile in slot 0
+      const int n_first = b_first == 0 ? na : nt;
       float2 l2 = make_float2(0.f, 0.f);
       const float2 rs2 = make_float2(rs, rs), nms2 = make_float2(-ms, -ms);
       {
@@ -894,10 +907,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Loops stay rolled (two chunk bodies per variant): the region code
         // is refetched by every head, so its size decides instruction-cache
         // hits.
-        auto chunk_col = [&](int i) { return i < na ? wq4 * 32 + i * 32 : 128 + (i - na) * 32; };
+        auto chunk_blk = [&](int i) { return i < n_first ? b_first : 1 - b_first; };
+        auto chunk_pc = [&](int i) {
+          const int k = i < n_first ? i : i - n_first;
+          return chunk_blk(i) == 0 ? wq4 + k : k;
+        };
+        auto chunk_col = [&](int i) { return slot_of(chunk_blk(i)) * 128 + chunk_pc(i) * 32; };
         auto chunk = [&](const uint32_t(&x)[32], int i) {
-          const int blk = i < na ? 0 : 1;
-          const int pc = blk == 0 ? wq4 + i : i - na;
+          const int blk = chunk_blk(i);
+          const int pc = chunk_pc(i);
           uint32_t pk[16];
           if (pc != wq4) {
 #pragma unroll
@@ -923,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[e] = pack_bf16x2(p.x, p.y);
             }
           }
-          tmem_st16(t_row + blk * 64 + pc * 16, pk);
+          tmem_st16(t_row + slot_of(blk) * 64 + pc * 16, pk);
         };
         // One register buffer: while a warp waits for its chunk, the SM runs
         // the other warps; the smaller loop keeps the region code in cache.
@@ -941,8 +959,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
                                      0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         for (int pc = 0; pc < 4; ++pc) {
-          if (hp && pc < wq4) tmem_st16(t_row + pc * 16, zero16);
-          if (pc > wq4) tmem_st16(t_row + 64 + pc * 16, zero16);
+          if (hp && pc < wq4) tmem_st16(t_row + slot_of(0) * 64 + pc * 16, zero16);
+          if (pc > wq4) tmem_st16(t_row + slot_of(1) * 64 + pc * 16, zero16);
         }
       }
       const float l = l2.x + l2.y;
