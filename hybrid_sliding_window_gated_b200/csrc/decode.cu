@@ -43,6 +43,7 @@ struct alignas(1024) Stage {
   uint16_t q[kDecMaxGroup][kHeadDim];  // the group's query rows
   uint16_t g[kDecMaxGroup][kHeadDim];  // gate logits
   uint16_t kn[kHeadDim], vn[kHeadDim];  // new token's k and v
+  float2 rot[kMaxPairs];                // rot(pos w_p): the position's rotation, per pair
   long long pos;
 };
 
@@ -114,7 +115,11 @@ __device__ __forceinline__ void process_unit(Stage& st, Group& gp, const DecArgs
 
   // ---- q' for heads lw, lw+4; k' and v_new on the owner warp
   float cs = 1.0f, sn = 0.0f;
-  if (lane < a.half_rot) rope_cos_sin(static_cast<double>(p), a.inv_freq[lane], &cs, &sn);
+  if (lane < a.half_rot) {  // from the producer, once per sequence
+    const float2 r = st.rot[lane];
+    cs = r.x;
+    sn = r.y;
+  }
   for (int h = lw; h < a.G; h += 4) {
     float x[4];
     load4(st.q[h] + 4 * lane, x);
@@ -285,23 +290,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Lane 0 issues the copies; the whole warp then writes the position and
+    // its rotation (computed once per sequence: a sequence's KV-head units
+    // are consecutive) into the stage before the position's arrive.
     if (lane == 0) {
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      const uint32_t row_bytes = kHeadDim * 2;
-      const uint32_t bytes = 4 * kHalfBytes + 2 * a.G * row_bytes + 2 * row_bytes;
-      int issued[kStages] = {0};
-      bool ok = true;
-      for (int i = 0; i < n_units; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages &&
-            !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1, abort, a.err, kSiteEmpty)) {
-          ok = false;
-          break;
-        }
-        const long long u = u0 + i;
-        const int n = static_cast<int>(u / a.Hkv), kvh = static_cast<int>(u - u / a.Hkv * a.Hkv);
-        Stage& st = sm.st[s];
+    }
+    const uint32_t row_bytes = kHeadDim * 2;
+    const uint32_t bytes = 4 * kHalfBytes + 2 * a.G * row_bytes + 2 * row_bytes;
+    int issued[kStages] = {0};
+    bool ok = true;
+    long long seq = -1, p = 0;  // the last sequence seen, its position
+    float2 rot = make_float2(1.0f, 0.0f);
+    for (int i = 0; i < n_units; ++i) {
+      const int s = i % kStages;
+      bool w = true;
+      if (lane == 0 && i >= kStages)
+        w = mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1, abort, a.err, kSiteEmpty);
+      if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) {
+        ok = false;
+        break;
+      }
+      const long long u = u0 + i;
+      const int n = static_cast<int>(u / a.Hkv), kvh = static_cast<int>(u - u / a.Hkv * a.Hkv);
+      Stage& st = sm.st[s];
+      if (lane == 0) {
         mbar_arrive_expect_tx(&sm.full[s], bytes);
         tma_load_4d(st.k[0], &tm_k, &sm.full[s], 0, 0, kvh, n);
         tma_load_4d(st.k[1], &tm_k, &sm.full[s], 64, 0, kvh, n);
@@ -313,15 +327,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(st.g, a.g + qrow, a.G * row_bytes, &sm.full[s]);
         bulk_load(st.kn, a.k_new + kvrow, row_bytes, &sm.full[s]);
         bulk_load(st.vn, a.v_new + kvrow, row_bytes, &sm.full[s]);
-        st.pos = a.pos[n];  // read while the copies fly
-        mbar_arrive(&sm.full[s]);  // releases the position written above
         ++issued[s];
       }
-      if (!ok) {
-        // Every copy issued lands before the CTA releases its shared memory.
-        for (int s = 0; s < kStages; ++s)
-          if (issued[s] > 0) mbar_wait_drain(&sm.full[s], (issued[s] - 1) & 1);
+      if (n != seq) {  // read while the copies fly
+        seq = n;
+        p = a.pos[n];
+        if (lane < a.half_rot)
+          rope_cos_sin(static_cast<double>(p), a.inv_freq[lane], &rot.x, &rot.y);
       }
+      if (lane == 0) st.pos = p;
+      if (lane < a.half_rot) st.rot[lane] = rot;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.full[s]);  // releases the position and rotation
+    }
+    if (!ok && lane == 0) {
+      // Every copy issued lands before the CTA releases its shared memory.
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&sm.full[s], (issued[s] - 1) & 1);
     }
     __syncwarp();
   } else {
