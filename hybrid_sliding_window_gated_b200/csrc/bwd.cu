@@ -1049,7 +1049,6 @@ struct alignas(1024) SmemKV {
   float xt[2][kTile];   // per-warpgroup halves of each dk row's Jacobian dot
   uint64_t kfull, vfull, kvempty, qfull[2], qempty[2], kvready, dkvfull, tfree, xtb;
   uint64_t qready[2], staged[2], sfull[2], pfull[2];  // per warpgroup: pair nq is warpgroup nq & 1's
-  uint64_t mmadone;  // dV/dK of the previous pair finished (their TMEM operands are free)
   uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
   uint32_t tmem_base;
   int abort;
@@ -1088,7 +1087,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.pfull[i], 128);
     }
     mbar_init(&sm.kvready, 256);
-    mbar_init(&sm.mmadone, 1);
     mbar_init(&sm.dkvfull, 1);
     mbar_init(&sm.tfree, 256);
     mbar_init(&sm.xtb, 256);
@@ -1204,9 +1202,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (it > 0 && !W(&sm.tfree, (it - 1) & 1, kSiteTFree)) break;
           }
           if (!W(&sm.qready[cg], ph, kSiteQReady)) break;
-          // S^T of this pair overwrites the columns dV of the previous pair
-          // reads as its A operand: start it only once that MMA is done.
-          if (nq > 0 && !W(&sm.mmadone, (nq - 1) & 1, kSiteMmaDone)) break;
+          // S^T and dP^T of this pair overwrite the columns that dV and dK of
+          // the previous pair read as their A operands (P^T, dS^T); the tensor
+          // core runs one thread's MMAs in issue order, so they go right
+          // behind them.
           tc_fence_after();
           // S^T = K' Q'^T (columns 256..383), dP^T = V dA^T (384..511)
 #pragma unroll
@@ -1230,7 +1229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tmem + 128, tmem + 384 + kk * 8, desc_mn(sm.q[nq & 1], kk), kIdescKM16,
                    (i > 0 || kk > 0));
           mma_commit(&sm.qempty[nq & 1]);
-          mma_commit(&sm.mmadone);
         }
         if (!ok) break;
         mma_commit(&sm.dkvfull);
