@@ -365,13 +365,11 @@ static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
   fill_inv_freq(p, a.inv_freq);
   if (a.total_tiles > (1ll << 30)) return SWA_ERR_UNSUPPORTED;
 
-  CUtensorMap tq, tk, tv, tda;
+  CUtensorMap tq, tk, tv;
   const uint64_t D = kHeadDim, T = p->T, B = p->B;
   if ((rc = encode_tmap_4d(&tq, q, D, p->Hq, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       (rc = encode_tmap_4d(&tk, k, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-      (rc = encode_tmap_4d(&tda, a.ws_da, D, p->Hq, T, B, 64, 1, kTile, 1,
-                           CU_TENSOR_MAP_SWIZZLE_128B)))
+      (rc = encode_tmap_4d(&tv, v, D, p->Hkv, T, B, 64, 1, kTile, 1, CU_TENSOR_MAP_SWIZZLE_128B)))
     return rc;
   CUtensorMap tkh = tk, tvh = tv;
   if (halo &&
@@ -380,7 +378,7 @@ static int bwd_impl(const swa_params_t* p, const swa_bf16_t* q, const swa_bf16_t
        (rc = encode_tmap_4d(&tvh, v_halo, D, p->Hkv, kWindow - 1, B, 64, 1, kTile, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B))))
     return rc;
-  return launch_bwd(p, tq, tk, tv, tda, tkh, tvh, a, static_cast<cudaStream_t>(stream));
+  return launch_bwd(p, tq, tk, tv, tkh, tvh, a, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace swa

@@ -258,6 +258,28 @@ __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t* tile, int kk) {
 __device__ __forceinline__ uint64_t desc_mn(const uint8_t* tile, int kk) {
   return desc_advance(make_desc_sw128(smem_u32(tile), kHalfBytes, 1024), kk * 2048);
 }
+// One dA tile of the workspace, which is tile-major: [B, Hq, tiles] tiles of
+// 128 rows x 128 fp16 in the swizzled MMA operand layout, 32 KiB each, so the
+// query-major pass stores and the key-major pass loads a tile in one copy.
+__device__ __forceinline__ uint16_t* da_tile(const BwdArgs& a, int b, int hq, int t) {
+  return a.ws_da + ((static_cast<long long>(b) * a.Hq + hq) * a.tiles_per_chain + t) *
+                       (kTileBytes / 2);
+}
+// 1-D bulk copies (16-byte aligned, sizes multiples of 16).
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(sdst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 constexpr uint32_t kIdescKK = make_idesc_bf16(128, 128, false, false);  // A, B K-major
 constexpr uint32_t kIdescKM = make_idesc_bf16(128, 128, false, true);   // B MN-major
 // The same shapes with fp16 A and B (format fields 0): Q', K' and dS operands.
@@ -567,14 +589,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         mma_commit(&sm.afull);
-        // dP = dA [V_{t-1} V_t]^T into columns 256..511
+        // dP = dA [V_{t-1} V_t]^T into columns 256..511.  The dA tile goes to
+        // the workspace (for the key-major pass) while the MMAs read it too;
+        // dS overwrites it after dpfull, which follows the store's read.
         if (!W(&sm.dafull, ph, kSiteDAFull)) break;
         tc_fence_after();
+        bulk_store(da_tile(a, c.b, c.kvh * a.G + h, c.t), sm.slot[n & 1], kTileBytes);
+        bulk_commit();
         for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tmem + 256 + blk * 128, desc_kmajor(sm.slot[n & 1], kk),
                    desc_kmajor(sm.v[blk ? sc : sp], kk), kIdescKK16, kk > 0);
+        bulk_wait_read<0>();
         mma_commit(&sm.dpfull);
         // dQ = sum over key tiles of dS K' into columns 128..255
         {
@@ -613,6 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&sm.drain);
         mbar_wait_drain(&sm.drain, 0);
       }
+      bulk_wait_all();  // every dA tile written before the CTA exits
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -824,7 +852,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 si2 = make_float2(pow2f(ei), pow2f(ei));  // dA is staged as dA 2^e
       {
         uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim) + 128 * cg;
-        uint8_t* darow = reinterpret_cast<uint8_t*>(a.ws_da + tok * kHeadDim) + 128 * cg;
 #pragma unroll 1
         for (int hc = 0; hc < 2; ++hc) {
           const int ch = 2 * cg + hc;  // 32-column chunk of the row
@@ -857,8 +884,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (valid_row) {
             st32B(dgrow + 64 * hc, *reinterpret_cast<const uint32_t(*)[8]>(dgo));
             st32B(dgrow + 64 * hc + 32, *reinterpret_cast<const uint32_t(*)[8]>(dgo + 8));
-            st32B(darow + 64 * hc, *reinterpret_cast<const uint32_t(*)[8]>(dao));
-            st32B(darow + 64 * hc + 32, *reinterpret_cast<const uint32_t(*)[8]>(dao + 8));
           }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {  // the second chunk's g and dO move down
@@ -1060,7 +1085,7 @@ static_assert(sizeof(SmemKV) + 1024 <= 232448, "pass 2 shared memory");
 template <int kPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     swa_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
+                      const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_kh,
                       const __grid_constant__ CUtensorMap tm_vh, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -1165,8 +1190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sm.qfull[b], 2 * kTileBytes);
           tma_load_4d(sm.q[b], &tm_q, &sm.qfull[b], 0, hq, qt * kTile, c.b);
           tma_load_4d(sm.q[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, qt * kTile, c.b);
-          tma_load_4d(sm.da[b], &tm_da, &sm.qfull[b], 0, hq, qt * kTile, c.b);
-          tma_load_4d(sm.da[b] + kHalfBytes, &tm_da, &sm.qfull[b], 64, hq, qt * kTile, c.b);
+          bulk_load(sm.da[b], da_tile(a, c.b, hq, qt), kTileBytes, &sm.qfull[b]);
         }
       }
     }
@@ -1524,7 +1548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int kPairs>
 int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& tda, const CUtensorMap& tkh, const CUtensorMap& tvh,
+                const CUtensorMap& tkh, const CUtensorMap& tvh,
                 const BwdArgs& a, int num_sms, cudaStream_t stream) {
   const size_t smem_q = sizeof(SmemQ) + 1024, smem_kv = sizeof(SmemKV) + 1024;
   static int configured_device = -1;
@@ -1554,22 +1578,22 @@ int launch_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap&
   if (rc != SWA_OK) return rc;
   const long long grid_kv = a.kv_total_tiles < num_sms ? a.kv_total_tiles : num_sms;
   return launch_dependent(swa_bwd_kv_kernel<kPairs>, static_cast<unsigned>(grid_kv), kThreads,
-                          smem_kv, stream, tq, tk, tv, tda, tkh, tvh, a);
+                          smem_kv, stream, tq, tk, tv, tkh, tvh, a);
 }
 
 }  // namespace bwd
 
 int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tda, const CUtensorMap& tkh,
-               const CUtensorMap& tvh, const BwdArgs& a, cudaStream_t stream) {
+               const CUtensorMap& tv, const CUtensorMap& tkh, const CUtensorMap& tvh,
+               const BwdArgs& a, cudaStream_t stream) {
   DeviceInfo di;
   int rc = current_device_info(&di);
   if (rc != SWA_OK) return rc;
   switch (p->rot_dim) {
-    case 0: return bwd::launch_impl<0>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
-    case 32: return bwd::launch_impl<16>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
-    case 42: return bwd::launch_impl<21>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
-    case 48: return bwd::launch_impl<24>(tq, tk, tv, tda, tkh, tvh, a, di.num_sms, stream);
+    case 0: return bwd::launch_impl<0>(tq, tk, tv, tkh, tvh, a, di.num_sms, stream);
+    case 32: return bwd::launch_impl<16>(tq, tk, tv, tkh, tvh, a, di.num_sms, stream);
+    case 42: return bwd::launch_impl<21>(tq, tk, tv, tkh, tvh, a, di.num_sms, stream);
+    case 48: return bwd::launch_impl<24>(tq, tk, tv, tkh, tvh, a, di.num_sms, stream);
     default: return SWA_ERR_UNSUPPORTED;
   }
 }

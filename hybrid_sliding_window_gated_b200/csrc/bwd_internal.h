@@ -28,7 +28,7 @@ struct BwdArgs {
   // Workspace.  Row i of dA is staged as dA_i 2^e_i, with e_i chosen from
   // max|dO_i| so the row's largest value lies in [1, 2) (fp16 keeps its full
   // precision there whatever the scale of the upstream gradient).
-  uint16_t* ws_da;  // dA_i 2^e_i, [B, T, Hq, D] fp16
+  uint16_t* ws_da;  // dA_i 2^e_i, fp16 tiles [B, Hq, tiles] of 128 x 128 (operand layout)
   float* ws_d;      // D_i 2^e_i = (dA_i 2^e_i) . A_i, [B, Hq, T] fp32
   float* ws_lse;    // log2 of the renormalised softmax normaliser, plus e_i, [B, Hq, T] fp32
   int* ws_ee;       // min of e_i over each query tile's rows, [B, Hq, tiles]
@@ -58,11 +58,11 @@ constexpr int kDevErrBadWeights = 0x201;
 // a finite |dO| >= 2^63 (beyond the per-row scaling's range).
 constexpr int kDevErrRange = 0x202;
 
-// Workspace layout, each part 256-byte aligned: dA rows, D, the renormalised
+// Workspace layout, each part 256-byte aligned: dA tiles, D, the renormalised
 // lse (D and lse share the size bwd_ws_d_bytes), then the two exponent records.
 inline size_t bwd_round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
-inline size_t bwd_ws_da_bytes(long long B, long long T, int Hq) {
-  return bwd_round256(static_cast<size_t>(B) * T * Hq * kHeadDim * 2);
+inline size_t bwd_ws_da_bytes(long long B, long long T, int Hq) {  // whole 128 x 128 tiles
+  return bwd_round256(static_cast<size_t>(B) * ((T + kTile - 1) / kTile) * Hq * kTile * kHeadDim * 2);
 }
 inline size_t bwd_ws_d_bytes(long long B, long long T, int Hq) {
   return bwd_round256(static_cast<size_t>(B) * T * Hq * 4);
@@ -80,7 +80,7 @@ inline size_t bwd_ws_total_bytes(long long B, long long T, int Hq, int Hkv) {
 
 // tkh, tvh: the halo K and V (any valid map when a.halo is 0).
 int launch_bwd(const swa_params_t* p, const CUtensorMap& tq, const CUtensorMap& tk,
-               const CUtensorMap& tv, const CUtensorMap& tda, const CUtensorMap& tkh,
-               const CUtensorMap& tvh, const BwdArgs& a, cudaStream_t stream);
+               const CUtensorMap& tv, const CUtensorMap& tkh, const CUtensorMap& tvh,
+               const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace swa
