@@ -749,9 +749,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // --------------------------------------------------------------- region
-    // Warpgroup r serves TMEM region r: heads n = r, r+2, ...  Per head:
-    // softmax S(n) once QK^T(n) is done, then the transform T(n+2) of the
-    // next Q (overlapping PV(n)), then the epilogue E(n).
+    // Warpgroup r serves TMEM region r: heads n = r, r+2, ...  Per head: the
+    // transform T(n) (the tile's K when this is its first head, then Q(n)),
+    // the softmax S(n) once QK^T(n) is done, then the epilogue E(n) once
+    // PV(n) is.
     regs_inc<kRegsRegion>();
     const int r = (warp - 4) >> 2;
     const int wq4 = warp & 3;  // TMEM lane quarter
