@@ -95,11 +95,13 @@ constexpr uint32_t kF16MaxBits = 0x477Fu;
 // fp16 in place: every backward contraction runs fp16 x fp16, three more
 // mantissa bits than bf16.  Returns the row's largest magnitude as bf16 bits
 // (NaN compares above every finite value).
-__device__ __forceinline__ uint32_t row_to_f16(uint8_t* tile, int row) {
+// `hs` is the distance between the tile's two halves (the query-major pass
+// keeps its two key tiles interleaved by half).
+__device__ __forceinline__ uint32_t row_to_f16(uint8_t* tile, int row, int hs = kHalfBytes) {
   uint32_t m = 0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint4* p = reinterpret_cast<uint4*>(tile + h * kHalfBytes + row * 128);
+    uint4* p = reinterpret_cast<uint4*>(tile + h * hs + row * 128);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const uint4 u = p[c];
@@ -168,13 +170,13 @@ __device__ __forceinline__ float2 rot_at(const float2 (*hi)[8], const RotTables&
   return cmul(hi[p][row >> 4], t.lo[p][row & 15]);
 }
 
-__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
+__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row, int hs = kHalfBytes) {
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                    make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 x = *reinterpret_cast<const uint4*>(tile + sw_off(row, c));
-    const uint4 y = *reinterpret_cast<const uint4*>(tile + kHalfBytes + sw_off(row, c));
+    const uint4 y = *reinterpret_cast<const uint4*>(tile + hs + sw_off(row, c));
     const uint32_t w[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -192,8 +194,8 @@ __device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
 template <int kPairs>
 __device__ __forceinline__ float norm_rope_row(uint8_t* tile, int row, const float* w,
                                                const float2 (*hi)[8], const RotTables& t,
-                                               float eps) {
-  const float rinv = rsqrtf(row_sumsq(tile, row) * (1.0f / kHeadDim) + eps);
+                                               float eps, int hs = kHalfBytes) {
+  const float rinv = rsqrtf(row_sumsq(tile, row, hs) * (1.0f / kHeadDim) + eps);
   float x[kHeadDim / 2];  // the first half (dims 0..63): it holds every rotated pair
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -221,7 +223,7 @@ __device__ __forceinline__ float norm_rope_row(uint8_t* tile, int row, const flo
     u.w = pack_f16x2(x[8 * c + 6], x[8 * c + 7]);
     *reinterpret_cast<uint4*>(tile + sw_off(row, c)) = u;
   }
-  uint8_t* h1 = tile + kHalfBytes;
+  uint8_t* h1 = tile + hs;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(h1 + sw_off(row, c));
@@ -280,12 +282,22 @@ __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t
       : "memory");
 }
 
+// K-major descriptor of k-step kk over both slots of a ring (256 rows).
+__device__ __forceinline__ uint64_t desc_ring(const uint8_t (*ring)[2][kHalfBytes], int kk) {
+  return desc_advance(make_desc_sw128(smem_u32(ring[kk >> 2][0]), 16, 1024), (kk & 3) * 32);
+}
+// MN-major descriptor of one slot of a ring for k-step kk (its halves 32 KiB apart).
+__device__ __forceinline__ uint64_t desc_mn_ring(const uint8_t (*ring)[2][kHalfBytes], int slot,
+                                                 int kk) {
+  return desc_advance(make_desc_sw128(smem_u32(ring[0][slot]), 2 * kHalfBytes, 1024), kk * 2048);
+}
 constexpr uint32_t kIdescKK = make_idesc_bf16(128, 128, false, false);  // A, B K-major
 constexpr uint32_t kIdescKM = make_idesc_bf16(128, 128, false, true);   // B MN-major
 // The same shapes with fp16 A and B (format fields 0): Q', K' and dS operands.
 constexpr uint32_t kF16 = ~((1u << 7) | (1u << 10));
 constexpr uint32_t kIdescKK16 = kIdescKK & kF16;
 constexpr uint32_t kIdescKM16 = kIdescKM & kF16;
+constexpr uint32_t kIdescKK16x256 = make_idesc_bf16(128, 256, false, false) & kF16;  // both key tiles
 // fp16 holds the normalised operands while max|w| * sqrt(head_dim) stays well
 // inside its range; larger weights are refused (device error code below).
 constexpr float kMaxWeight = 4096.0f;
@@ -345,11 +357,11 @@ __device__ __forceinline__ void next_tile_kv(Cursor& c, const BwdArgs& a) {
 // row zero-filled and never in the band).
 __device__ __forceinline__ void load_key_tile(uint8_t* dst, const CUtensorMap* map,
                                               const CUtensorMap* map_halo, uint64_t* bar, int j,
-                                              int kvh, int b) {
+                                              int kvh, int b, int hs = kHalfBytes) {
   const CUtensorMap* m = j < 0 ? map_halo : map;
   const int y = j < 0 ? -1 : j * kTile;
   tma_load_4d(dst, m, bar, 0, kvh, y, b);
-  tma_load_4d(dst + kHalfBytes, m, bar, 64, kvh, y, b);
+  tma_load_4d(dst + hs, m, bar, 64, kvh, y, b);
 }
 
 // Rotation table rot((128 j + 16 a) w_p), a = 0..7, computed by a warp.
@@ -367,8 +379,10 @@ __device__ __forceinline__ void fill_rot_hi(float2 (*hi)[8], int j, const BwdArg
 // ===================================================== pass 1: query-major
 
 struct alignas(1024) SmemQ {
-  uint8_t k[2][kTileBytes];
-  uint8_t v[2][kTileBytes];
+  // K and V rings, [half][slot]: per 64-dim half the two slots' 128 rows lie
+  // one after the other, so one N = 256 MMA reads both key tiles.
+  uint8_t k[2][2][kHalfBytes];
+  uint8_t v[2][2][kHalfBytes];
   // Head n works in slot n & 1: Q', then dA, then dS of each key tile, each
   // written once the MMA reading its predecessor is done; the other slot
   // receives Q of head n+1 meanwhile.
@@ -492,9 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           !wait0(empty, ((par >> s) & 1u) ^ 1u, is_k ? kSiteKEmpty : kSiteVEmpty))
         return false;
       if (lane == 0) {
-        uint8_t* dst = is_k ? sm.k[s] : sm.v[s];
+        uint8_t* dst = is_k ? sm.k[0][s] : sm.v[0][s];
         mbar_arrive_expect_tx(full, kTileBytes);
-        load_key_tile(dst, is_k ? &tm_k : &tm_v, is_k ? &tm_kh : &tm_vh, full, j, c.kvh, c.b);
+        load_key_tile(dst, is_k ? &tm_k : &tm_v, is_k ? &tm_kh : &tm_vh, full, j, c.kvh, c.b,
+                      2 * kHalfBytes);
       }
       if (is_k) {
         fill_rot_hi<kPairs>(sm.rot_hi[s], j, a, lane);
@@ -560,12 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!W(&sm.qready, ph, kSiteQReady)) break;
         if (n > 0 && !W(&sm.tfree, ph ^ 1u, kSiteTFree)) break;
         tc_fence_after();
-        // S = Q' [K'_{t-1} K'_t]^T into columns 0..255
-        for (int blk = hp ? 0 : 1; blk < 2; ++blk)
+        // S = Q' [K' slot 0; K' slot 1]^T into columns 0..255, one N = 256
+        // MMA per k-step: columns 128 s .. 128 s + 127 hold the key tile in
+        // slot s (t-1 and t in either order; without a tile t-1 that half is
+        // never read).
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + blk * 128, desc_kmajor(sm.slot[n & 1], kk),
-                   desc_kmajor(sm.k[blk ? sc : sp], kk), kIdescKK16, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.k, kk), kIdescKK16x256,
+                 kk > 0);
         mma_commit(&sm.sfull);
         if (h == 0) {
           if (need_prev(c, a)) {
@@ -582,8 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              mma_ts(tmem + 256, tmem + blk * 64 + kk * 8, desc_mn(sm.v[blk ? sc : sp], kk),
+            for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns 64 s ..
+              const int slot = blk ? sc : sp;
+              mma_ts(tmem + 256, tmem + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
                      kIdescKM16, acc);
               acc = 1;
             }
@@ -596,11 +614,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         bulk_store(da_tile(a, c.b, c.kvh * a.G + h, c.t), sm.slot[n & 1], kTileBytes);
         bulk_commit();
-        for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 256 + blk * 128, desc_kmajor(sm.slot[n & 1], kk),
-                   desc_kmajor(sm.v[blk ? sc : sp], kk), kIdescKK16, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)  // dP of the tile in slot s: columns 256 + 128 s ..
+          mma_ss(tmem + 256, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.v, kk), kIdescKK16x256,
+                 kk > 0);
         bulk_wait_read<0>();
         mma_commit(&sm.dpfull);
         // dQ = sum over key tiles of dS K' into columns 128..255
@@ -613,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               mma_ss(tmem + 128, desc_kmajor(sm.slot[n & 1], kk),
-                     desc_mn(sm.k[blk ? sc : sp], kk), kIdescKM16, acc);
+                     desc_mn_ring(sm.k, blk ? sc : sp, kk), kIdescKM16, acc);
               acc = 1;
             }
             mma_commit(blk == 0 ? &sm.dq0 : &sm.dqfull);
@@ -699,14 +716,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cg == 0) {
             ok = warp_wait(&sm.kfull[s], (kpar >> s) & 1u, abort, a.err, kSiteKFull);
             if (!ok) break;
-            norm_rope_row<kPairs>(sm.k[s], row, sm.wk, sm.rot_hi[s], sm.rot, a.eps);
+            norm_rope_row<kPairs>(sm.k[0][s], row, sm.wk, sm.rot_hi[s], sm.rot, a.eps,
+                                  2 * kHalfBytes);
             fence_proxy_async_smem();
             mbar_arrive(&sm.kready[s]);
             kpar ^= 1u << s;
           } else {
             ok = warp_wait(&sm.vfull[s], (vpar >> s) & 1u, abort, a.err, kSiteVFull);
             if (!ok) break;
-            const uint32_t m = row_to_f16(sm.v[s], row);
+            const uint32_t m = row_to_f16(sm.v[0][s], row, 2 * kHalfBytes);
             in_range &= m <= kF16MaxBits;
             const uint32_t wm = __reduce_max_sync(0xffffffffu, m);
             if (lane == 0) sm.vmax[s][wq4] = wm;
@@ -743,13 +761,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- P = exp(s - lse) on the band.  The in-band 32-column chunks are
       // key tile t-1's wq4..3 (when it exists), then key tile t's 0..wq4;
-      // this warpgroup takes every other one.  P is packed over S's first 128
-      // columns, which the other warpgroup may still be reading, so the
-      // stores wait for the exchange of the row sums.
+      // this warpgroup takes every other one.  A key tile's S sits at the
+      // columns of its ring slot (128 s ..), its P at 64 s ..: P is packed
+      // over S's first 128 columns, which the other warpgroup may still be
+      // reading, so the stores wait for the exchange of the row sums.
       if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
       tc_fence_after();
       const int na = hp ? 4 - wq4 : 0;  // chunks of key tile t-1 in the band
       const int nch = na + wq4 + 1;
+      const int sp = sc ^ 1;  // ring slot of key tile t-1
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
       float2 lsum2 = make_float2(0.f, 0.f);
       uint32_t pk[3][16];
@@ -760,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int blk = i < na ? 0 : 1;
           const int pc = blk == 0 ? wq4 + i : i - na;
           uint32_t x[32];
-          tmem_ld32(t_row + blk * 128 + pc * 32, x);
+          tmem_ld32(t_row + (blk ? sc : sp) * 128 + pc * 32, x);
           tmem_wait_ld();
           if (pc != wq4) {
 #pragma unroll
@@ -821,14 +841,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i < nch) {
             const int blk = i < na ? 0 : 1;
             const int pc = blk == 0 ? wq4 + i : i - na;
-            tmem_st16(t_row + blk * 64 + pc * 16, pk[k]);
+            tmem_st16(t_row + (blk ? sc : sp) * 64 + pc * 16, pk[k]);
           }
         }
         // chunks outside the band: key tile t-1's below wq4 (or all of it
         // when it does not exist) by cg 0, key tile t's above wq4 by cg 1
         for (int pc = 0; pc < 4; ++pc) {
-          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + pc * 16, zero16);
-          if (cg == 1 && pc > wq4) tmem_st16(t_row + 64 + pc * 16, zero16);
+          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + sp * 64 + pc * 16, zero16);
+          if (cg == 1 && pc > wq4) tmem_st16(t_row + sc * 64 + pc * 16, zero16);
         }
       }
       tmem_wait_st();
@@ -944,8 +964,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hc = 0; hc < 2; ++hc) {
           const int pc = 2 * cg + hc;
           uint32_t pkc[16], dp[32];
-          tmem_ld16(t_row + blk * 64 + pc * 16, pkc);
-          tmem_ld32(t_row + 256 + blk * 128 + pc * 32, dp);
+          tmem_ld16(t_row + (blk ? sc : sc ^ 1) * 64 + pc * 16, pkc);
+          tmem_ld32(t_row + 256 + (blk ? sc : sc ^ 1) * 128 + pc * 32, dp);
           tmem_wait_ld();
           uint32_t ds[16];
 #pragma unroll
