@@ -239,6 +239,55 @@ __device__ __forceinline__ float norm_rope_row(uint8_t* tile, int row, const flo
   return rinv;
 }
 
+// Dim d of row `row` in a [128 x 128] 16-bit tile (two halves, 128B swizzle).
+__device__ __forceinline__ uint16_t* tile_elem(uint8_t* tile, int row, int d) {
+  return reinterpret_cast<uint16_t*>(tile + (d >> 6) * kHalfBytes + sw_off(row, (d >> 3) & 7) +
+                                     (d & 7) * 2);
+}
+__device__ __forceinline__ uint16_t f16_bits(float x) {
+  return static_cast<uint16_t>(pack_f16x2(x, 0.f) & 0xFFFFu);
+}
+
+// norm_rope_row for warps with few registers: the same operand, with each
+// rotated pair (p, p + kPairs) taken on its own and the rest of the row by
+// 16-byte chunks.  Every value is read once before it is rewritten.
+template <int kPairs>
+__device__ __forceinline__ float norm_rope_row_lean(uint8_t* tile, int row, const float* w,
+                                                    const float2 (*hi)[8], const RotTables& t,
+                                                    float eps) {
+  const float rinv = rsqrtf(row_sumsq(tile, row) * (1.0f / kHeadDim) + eps);
+#pragma unroll 1
+  for (int p = 0; p < kPairs; ++p) {
+    uint16_t* pa = tile_elem(tile, row, p);
+    uint16_t* pb = tile_elem(tile, row, p + kPairs);
+    const float a = bf16_lo(*pa) * rinv * w[p];
+    const float b = bf16_lo(*pb) * rinv * w[p + kPairs];
+    const float2 r = rot_at(hi, t, p, row);
+    *pa = f16_bits(a * r.x - b * r.y);
+    *pb = f16_bits(b * r.x + a * r.y);
+  }
+  constexpr int kFirstChunk = (2 * kPairs + 7) / 8;  // the first chunk with no rotated dim
+#pragma unroll 1
+  for (int d = 2 * kPairs; d < 8 * kFirstChunk; ++d) {
+    uint16_t* pd = tile_elem(tile, row, d);
+    *pd = f16_bits(bf16_lo(*pd) * rinv * w[d]);
+  }
+#pragma unroll 1
+  for (int c = kFirstChunk; c < 16; ++c) {
+    uint4* pc = reinterpret_cast<uint4*>(tile + (c >> 3) * kHalfBytes + sw_off(row, c & 7));
+    const uint4 u = *pc;
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int d = 8 * c + 2 * e;
+      o4[e] = pack_f16x2(bf16_lo(w4[e]) * rinv * w[d], bf16_hi(w4[e]) * rinv * w[d + 1]);
+    }
+    *pc = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+  }
+  return rinv;
+}
+
 // Sum a 64-value per-thread vector over the warp; lane l gets dims 2l, 2l+1.
 __device__ __forceinline__ float2 warp_reduce_scatter64(float (&v)[64], int lane) {
 #pragma unroll
@@ -389,10 +438,12 @@ struct alignas(1024) SmemQ {
   uint8_t slot[2][kTileBytes];
   RotTables rot;
   float2 rot_hi[2][kMaxPairs][8];  // per K slot
+  float2 qrot_hi[kMaxPairs][8];    // the Q transform's (each of its warps fills its rows' entries)
   float wq[kHeadDim], wk[kHeadDim], dw[kHeadDim];
   uint64_t kfull[2], kready[2], kempty[2], vfull[2], vready[2], vempty[2];
   uint64_t qfull[2], qempty[2];
-  uint64_t qready, sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull, tfree;
+  uint64_t qready[2];  // per Q slot
+  uint64_t sfull, pfull, afull, dafull, dpfull, dsfull, dq0, dqfull;
   uint64_t tables, drain, never;  // never: completed by nothing (forced timeouts)
   // Row-sum exchanges between the two compute warpgroups (l with the dA row
   // exponent, D, the dq dot).
@@ -401,7 +452,7 @@ struct alignas(1024) SmemQ {
   int xe[2][kTile];     // each half row's dA exponent (exchanged with l)
   int xew[2][2][4];     // [head parity][warpgroup][warp]: minimum of those exponents
   uint32_t vmax[2][4];  // per V slot and converting warp: largest |v| (bf16 bits)
-  float rinvq[kTile];  // 1/rms of each Q row (cg 0 computes it; both use it)
+  float rinvq[3][kTile];  // 1/rms of each Q row, head n in n % 3
   uint32_t tmem_base;
   int abort;
 };
@@ -435,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.qfull[i], 1);
       mbar_init(&sm.qempty[i], 1);
     }
-    mbar_init(&sm.qready, 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.qready[i], 64);
     mbar_init(&sm.sfull, 1);
     mbar_init(&sm.pfull, 256);
     mbar_init(&sm.afull, 1);
@@ -444,7 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.dsfull, 256);
     mbar_init(&sm.dq0, 1);
     mbar_init(&sm.dqfull, 1);
-    mbar_init(&sm.tfree, 256);
     mbar_init(&sm.tables, 256);
     mbar_init(&sm.xlb, 256);
     mbar_init(&sm.xdb, 256);
@@ -520,21 +570,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       used |= 1u << s;
       return true;
     };
+    auto load_q = [&](const Cursor& c, int h) -> bool {
+      const int b = nq & 1;
+      if (nq >= 2 && !wait0(&sm.qempty[b], ((nq >> 1) - 1) & 1, kSiteQEmpty)) return false;
+      if (lane == 0) {
+        const int hq = c.kvh * a.G + h;
+        mbar_arrive_expect_tx(&sm.qfull[b], kTileBytes);
+        tma_load_4d(sm.slot[b], &tm_q, &sm.qfull[b], 0, hq, c.t * kTile, c.b);
+        tma_load_4d(sm.slot[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, c.t * kTile, c.b);
+      }
+      ++nq;
+      return true;
+    };
     Cursor c = cursor_at(a, u0);
     for (int it = 0; it < n_tiles && ok; ++it, next_tile(c, a)) {
-      if (need_prev(c, a))
+      // The tile's first Q goes ahead of its key tiles: its slot frees a head
+      // earlier than theirs, and its transform needs no key tile.
+      ok = load_q(c, 0);
+      if (ok && need_prev(c, a))
         ok = load_kv(true, c.t - 1, c) && load_kv(false, c.t - 1, c);
       ok = ok && load_kv(true, c.t, c) && load_kv(false, c.t, c);
-      for (int h = 0; h < a.G && ok; ++h, ++nq) {
-        const int b = nq & 1;
-        if (nq >= 2 && !wait0(&sm.qempty[b], ((nq >> 1) - 1) & 1, kSiteQEmpty)) { ok = false; break; }
-        if (lane == 0) {
-          const int hq = c.kvh * a.G + h;
-          mbar_arrive_expect_tx(&sm.qfull[b], kTileBytes);
-          tma_load_4d(sm.slot[b], &tm_q, &sm.qfull[b], 0, hq, c.t * kTile, c.b);
-          tma_load_4d(sm.slot[b] + kHalfBytes, &tm_q, &sm.qfull[b], 64, hq, c.t * kTile, c.b);
-        }
-      }
+      for (int h = 1; h < a.G && ok; ++h) ok = load_q(c, h);
     }
     if (!ok && lane == 0) {
       for (int s = 0; s < 2; ++s) {
@@ -572,16 +628,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!W(&sm.kready[sc], (kpar >> sc) & 1u, kSiteKReady)) break;
           kpar ^= 1u << sc;
         }
-        if (!W(&sm.qready, ph, kSiteQReady)) break;
-        if (n > 0 && !W(&sm.tfree, ph ^ 1u, kSiteTFree)) break;
+        if (!W(&sm.qready[n & 1], (n >> 1) & 1u, kSiteQReady)) break;
         tc_fence_after();
-        // S = Q' [K' slot 0; K' slot 1]^T into columns 0..255, one N = 256
-        // MMA per k-step: columns 128 s .. 128 s + 127 hold the key tile in
+        // Head n's S and dQ live in the TMEM half tb (0 or 256, by the
+        // parity of n), A and dP in the other one, tw.  This head's S
+        // overwrites only what the previous head's dS phase has read (its A
+        // and dP), not its dQ, so it goes right behind the previous dQ.
+        const uint32_t tb = (n & 1) * 256u, tw = 256u - tb;
+        // S = Q' [K' slot 0; K' slot 1]^T into columns tb .. tb + 255, one
+        // N = 256 MMA per k-step: columns tb + 128 s .. hold the key tile in
         // slot s (t-1 and t in either order; without a tile t-1 that half is
         // never read).
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.k, kk), kIdescKK16x256,
+          mma_ss(tmem + tb, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.k, kk), kIdescKK16x256,
                  kk > 0);
         mma_commit(&sm.sfull);
         if (h == 0) {
@@ -592,22 +652,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!W(&sm.vready[sc], (vpar >> sc) & 1u, kSiteVFull)) break;
           vpar ^= 1u << sc;
         }
-        // A = P V into columns 256..383 (P packed in columns 0..127)
+        // A = P V into columns tw .. tw + 127 (P packed in columns tb .. tb + 127)
         if (!W(&sm.pfull, ph, kSitePFull)) break;
         tc_fence_after();
         {
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns 64 s ..
+            for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns tb + 64 s ..
               const int slot = blk ? sc : sp;
-              mma_ts(tmem + 256, tmem + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
+              mma_ts(tmem + tw, tmem + tb + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
                      kIdescKM16, acc);
               acc = 1;
             }
         }
         mma_commit(&sm.afull);
-        // dP = dA [V_{t-1} V_t]^T into columns 256..511.  The dA tile goes to
+        // dP = dA [V_{t-1} V_t]^T into columns tw .. tw + 255.  The dA tile goes to
         // the workspace (for the key-major pass) while the MMAs read it too;
         // dS overwrites it after dpfull, which follows the store's read.
         if (!W(&sm.dafull, ph, kSiteDAFull)) break;
@@ -615,12 +675,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_store(da_tile(a, c.b, c.kvh * a.G + h, c.t), sm.slot[n & 1], kTileBytes);
         bulk_commit();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dP of the tile in slot s: columns 256 + 128 s ..
-          mma_ss(tmem + 256, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.v, kk), kIdescKK16x256,
+        for (int kk = 0; kk < 8; ++kk)  // dP of the tile in slot s: columns tw + 128 s ..
+          mma_ss(tmem + tw, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.v, kk), kIdescKK16x256,
                  kk > 0);
         bulk_wait_read<0>();
         mma_commit(&sm.dpfull);
-        // dQ = sum over key tiles of dS K' into columns 128..255
+        // dQ = sum over key tiles of dS K' into columns tb + 128 .. tb + 255
         {
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
@@ -629,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              mma_ss(tmem + 128, desc_kmajor(sm.slot[n & 1], kk),
+              mma_ss(tmem + tb + 128, desc_kmajor(sm.slot[n & 1], kk),
                      desc_mn_ring(sm.k, blk ? sc : sp, kk), kIdescKM16, acc);
               acc = 1;
             }
@@ -660,7 +720,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_wait_all();  // every dA tile written before the CTA exits
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ------------------------------------------------ Q transform (warps 2, 3)
+    // Q' of head n in place in its slot, two rows per thread, while the
+    // compute warpgroups still work on head n-1: head n's QK^T then follows
+    // head n-1's dQ on the tensor core.
+    bool ok = warp_wait(&sm.tables, 0, abort, a.err, kSiteTables);
+    const int wsel = warp - 2;  // rows 32 wsel + 64 i + (0..31): hi entries 2 wsel + 4 i + (0, 1)
+    Cursor c = cursor_at(a, u0);
+    int h = 0;
+    for (int n = 0; n < n_heads && ok; ++n) {
+      if (h == 0) {  // rotation of the query tile's positions, this warp's entries
+        for (int e = lane; e < kPairs * 4; e += 32) {
+          const int p = e >> 2, ai = 2 * wsel + (e & 1) + 4 * ((e >> 1) & 1);
+          float cv, sv;
+          rope_cos_sin(static_cast<double>(a.pos0 + static_cast<long long>(c.t) * kTile) +
+                           16.0 * ai, a.inv_freq[p], &cv, &sv);
+          sm.qrot_hi[p][ai] = make_float2(cv, sv);
+        }
+        __syncwarp();
+      }
+      if (!(ok = warp_wait(&sm.qfull[n & 1], (n >> 1) & 1, abort, a.err, kSiteQFull))) break;
+      for (int r = tid - 64; r < kTile; r += 64)
+        sm.rinvq[n % 3][r] = norm_rope_row_lean<kPairs>(sm.slot[n & 1], r, sm.wq, sm.qrot_hi,
+                                                        sm.rot, a.eps);
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.qready[n & 1]);
+      if (++h == a.G) {
+        h = 0;
+        next_tile(c, a);
+      }
+    }
+  } else {
     // --------------------------------------------------- compute warpgroups
     // Two warpgroups share every query row: thread r of each owns row r
     // (TMEM lane r).  Warpgroup cg takes
@@ -734,16 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
       }
-      // ---- Q' (cg 0)
       uint8_t* slot = sm.slot[n & 1];
       const uint8_t* grow = reinterpret_cast<const uint8_t*>(a.g + tok * kHeadDim) + 128 * cg;
       const uint8_t* dorow = reinterpret_cast<const uint8_t*>(a.dO + tok * kHeadDim) + 128 * cg;
-      if (cg == 0) {
-        if (!(ok = warp_wait(&sm.qfull[n & 1], (n >> 1) & 1, abort, a.err, kSiteQFull))) break;
-        sm.rinvq[row] = norm_rope_row<kPairs>(slot, row, sm.wq, sm.rot_hi[sc], sm.rot, a.eps);
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.qready);
-      }
       // Rows past T take lse = +inf: their P is exactly 0 with no mask.
       const float lse2 = valid_row ? a.lse[lrow] * kLog2e : INFINITY;
       // this warpgroup's 64 columns of g and dO, in flight during P
@@ -767,6 +851,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // reading, so the stores wait for the exchange of the row sums.
       if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
       tc_fence_after();
+      // Q' done.  Its 1/rms, read in the dq epilogue, stays until head n+3's
+      // transform, which waits (through its slot) for head n+1's dS.
+      if (!(ok = warp_wait(&sm.qready[n & 1], (n >> 1) & 1, abort, a.err, kSiteQReady))) break;
+      const uint32_t tb = (n & 1) * 256u, tw = 256u - tb;  // TMEM halves, as the MMA lane's
       const int na = hp ? 4 - wq4 : 0;  // chunks of key tile t-1 in the band
       const int nch = na + wq4 + 1;
       const int sp = sc ^ 1;  // ring slot of key tile t-1
@@ -780,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int blk = i < na ? 0 : 1;
           const int pc = blk == 0 ? wq4 + i : i - na;
           uint32_t x[32];
-          tmem_ld32(t_row + (blk ? sc : sp) * 128 + pc * 32, x);
+          tmem_ld32(t_row + tb + (blk ? sc : sp) * 128 + pc * 32, x);
           tmem_wait_ld();
           if (pc != wq4) {
 #pragma unroll
@@ -841,14 +929,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i < nch) {
             const int blk = i < na ? 0 : 1;
             const int pc = blk == 0 ? wq4 + i : i - na;
-            tmem_st16(t_row + (blk ? sc : sp) * 64 + pc * 16, pk[k]);
+            tmem_st16(t_row + tb + (blk ? sc : sp) * 64 + pc * 16, pk[k]);
           }
         }
         // chunks outside the band: key tile t-1's below wq4 (or all of it
         // when it does not exist) by cg 0, key tile t's above wq4 by cg 1
         for (int pc = 0; pc < 4; ++pc) {
-          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + sp * 64 + pc * 16, zero16);
-          if (cg == 1 && pc > wq4) tmem_st16(t_row + sc * 64 + pc * 16, zero16);
+          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + tb + sp * 64 + pc * 16, zero16);
+          if (cg == 1 && pc > wq4) tmem_st16(t_row + tb + sc * 64 + pc * 16, zero16);
         }
       }
       tmem_wait_st();
@@ -876,7 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hc = 0; hc < 2; ++hc) {
           const int ch = 2 * cg + hc;  // 32-column chunk of the row
           uint32_t x[32];
-          tmem_ld32(t_row + 256 + ch * 32, x);
+          tmem_ld32(t_row + tw + ch * 32, x);
           tmem_wait_ld();
           uint32_t dgo[16], dao[16];
 #pragma unroll
@@ -964,8 +1052,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hc = 0; hc < 2; ++hc) {
           const int pc = 2 * cg + hc;
           uint32_t pkc[16], dp[32];
-          tmem_ld16(t_row + (blk ? sc : sc ^ 1) * 64 + pc * 16, pkc);
-          tmem_ld32(t_row + 256 + (blk ? sc : sc ^ 1) * 128 + pc * 32, dp);
+          tmem_ld16(t_row + tb + (blk ? sc : sc ^ 1) * 64 + pc * 16, pkc);
+          tmem_ld32(t_row + tw + (blk ? sc : sc ^ 1) * 128 + pc * 32, dp);
           tmem_wait_ld();
           uint32_t ds[16];
 #pragma unroll
@@ -993,13 +1081,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(&sm.dqfull, ph, abort, a.err, kSiteDQFull))) break;
       tc_fence_after();
       {
-        const float rinv = sm.rinvq[row];  // written by cg 0 before the first exchange
+        const float rinv = sm.rinvq[n % 3][row];
         const float2 rinv2 = make_float2(rinv, rinv);
         float y[64];
         {
           uint32_t r[32], r2[32];
-          tmem_ld32(t_row + 128 + cg * 64, r);
-          tmem_ld32(t_row + 128 + cg * 64 + 32, r2);
+          tmem_ld32(t_row + tb + 128 + cg * 64, r);
+          tmem_ld32(t_row + tb + 128 + cg * 64 + 32, r2);
           tmem_wait_ld();
           const float2 un2 = make_float2(pow2f(-(ei + kt)), pow2f(-(ei + kt)));  // undo 2^(e+k)
 #pragma unroll
@@ -1023,8 +1111,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             y[p + kPairs] = b0 * rcp.x - a0 * rcp.y;
           }
         }
-        tc_fence_before();
-        mbar_arrive(&sm.tfree);  // dQ has been read from TMEM
         float2 dot2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
