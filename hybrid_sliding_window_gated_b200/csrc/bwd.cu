@@ -630,10 +630,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!W(&sm.qready[n & 1], (n >> 1) & 1u, kSiteQReady)) break;
         tc_fence_after();
-        // Head n's S and dQ live in the TMEM half tb (0 or 256, by the
-        // parity of n), A and dP in the other one, tw.  This head's S
-        // overwrites only what the previous head's dS phase has read (its A
-        // and dP), not its dQ, so it goes right behind the previous dQ.
+        // Head n's S, P, A and dQ live in the TMEM half tb (0 or 256, by the
+        // parity of n), its dP in the other one, tw.  This head's S
+        // overwrites only what the previous head's dS phase has read (its
+        // dP), not its dQ, so it goes right behind the previous dQ; this
+        // head's dP follows its dA, which the compute warps write only after
+        // the previous head's dq epilogue.
         const uint32_t tb = (n & 1) * 256u, tw = 256u - tb;
         // S = Q' [K' slot 0; K' slot 1]^T into columns tb .. tb + 255, one
         // N = 256 MMA per k-step: columns tb + 128 s .. hold the key tile in
@@ -652,7 +654,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!W(&sm.vready[sc], (vpar >> sc) & 1u, kSiteVFull)) break;
           vpar ^= 1u << sc;
         }
-        // A = P V into columns tw .. tw + 127 (P packed in columns tb .. tb + 127)
+        // A = P V into columns tb + 128 .. tb + 255, which S's second half held
+        // (P packed in columns tb .. tb + 127)
         if (!W(&sm.pfull, ph, kSitePFull)) break;
         tc_fence_after();
         {
@@ -661,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns tb + 64 s ..
               const int slot = blk ? sc : sp;
-              mma_ts(tmem + tw, tmem + tb + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
+              mma_ts(tmem + tb + 128, tmem + tb + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
                      kIdescKM16, acc);
               acc = 1;
             }
@@ -951,57 +954,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (cg == 0 && valid_row)
         a.ws_lse[lrow] = (a.lse[lrow] + __logf(lsum)) * kLog2e + static_cast<float>(ei);
 
-      // ---- A: dg, dA (smem and workspace) and D over this warpgroup's 64
-      // columns (TMEM chunks 2 cg, 2 cg + 1)
+      // ---- dA = dO sigma(g) 2^e over this warpgroup's 64 columns, into the
+      // Q slot (QK^T has read it): dA needs no A, so the dP MMAs start on it
+      // while A = P V is still on its way.  dO sigma'(g) waits for A in
+      // registers.
+      const float2 il2 = make_float2(inv_l, inv_l);
+      const float2 si2 = make_float2(pow2f(ei), pow2f(ei));  // dA is staged as dA 2^e
+      float2 dgf[32];    // dO sigma (1 - sigma) per column pair
+      uint32_t dao[32];  // dA 2^e as the MMAs see it (fp16)
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2 gg = bf2(gc[e]), dd = bf2(dc[e]);
+        float2 ds;                            // sigma (1 - sigma), without cancellation
+        const float2 sg = sigmoid2(gg, &ds);  // one MUFU op per element
+        dgf[e] = __fmul2_rn(dd, ds);
+        const float2 dav = __fmul2_rn(__fmul2_rn(dd, sg), si2);
+        dao[e] = pack_f16x2(dav.x, dav.y);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // dA into the MMA operand tile (row-major over dims, 128B swizzle)
+        const int c16 = 8 * cg + i;  // 16-byte piece of the row
+        *reinterpret_cast<uint4*>(slot + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) =
+            make_uint4(dao[4 * i], dao[4 * i + 1], dao[4 * i + 2], dao[4 * i + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.dafull);
+
+      // ---- dg and D = sum dA A over the same columns (TMEM chunks 2 cg,
+      // 2 cg + 1 of A)
       if (!(ok = warp_wait(&sm.afull, ph, abort, a.err, kSiteAFull))) break;
       tc_fence_after();
       float2 dsum2 = make_float2(0.f, 0.f);
-      const float2 il2 = make_float2(inv_l, inv_l);
-      const float2 si2 = make_float2(pow2f(ei), pow2f(ei));  // dA is staged as dA 2^e
       {
         uint8_t* dgrow = reinterpret_cast<uint8_t*>(a.dg + tok * kHeadDim) + 128 * cg;
-#pragma unroll 1
+#pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
-          const int ch = 2 * cg + hc;  // 32-column chunk of the row
           uint32_t x[32];
-          tmem_ld32(t_row + tw + ch * 32, x);
+          tmem_ld32(t_row + tb + 128 + (2 * cg + hc) * 32, x);
           tmem_wait_ld();
-          uint32_t dgo[16], dao[16];
+          uint32_t dgo[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const uint32_t gw = gc[e];
-            const uint32_t dw = dc[e];
-            const float2 gg = bf2(gw), dd = bf2(dw);
             const float2 av = __fmul2_rn(
                 make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), il2);  // A / l
-            float2 ds;                            // sigma (1 - sigma), without cancellation
-            const float2 sg = sigmoid2(gg, &ds);  // one MUFU op per element
-            const float2 dgv = __fmul2_rn(__fmul2_rn(dd, av), ds);
+            const float2 dgv = __fmul2_rn(dgf[16 * hc + e], av);
             dgo[e] = pack_bf16x2(dgv.x, dgv.y);
-            const float2 dav = __fmul2_rn(__fmul2_rn(dd, sg), si2);
-            dao[e] = pack_f16x2(dav.x, dav.y);
-            dsum2 = __ffma2_rn(f16x2(dao[e]), av, dsum2);  // D uses the rounded dA the MMAs see
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            // dA into the MMA operand tile (row-major over dims, 128B swizzle)
-            const int c16 = 4 * ch + i;  // 16-byte piece of the row
-            *reinterpret_cast<uint4*>(slot + (c16 >> 3) * kHalfBytes + sw_off(row, c16 & 7)) =
-                make_uint4(dao[4 * i], dao[4 * i + 1], dao[4 * i + 2], dao[4 * i + 3]);
+            dsum2 = __ffma2_rn(f16x2(dao[16 * hc + e]), av, dsum2);  // D uses the rounded dA
           }
           if (valid_row) {
             st32B(dgrow + 64 * hc, *reinterpret_cast<const uint32_t(*)[8]>(dgo));
             st32B(dgrow + 64 * hc + 32, *reinterpret_cast<const uint32_t(*)[8]>(dgo + 8));
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {  // the second chunk's g and dO move down
-            gc[e] = gc[16 + e];
-            dc[e] = dc[16 + e];
-          }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&sm.dafull);
       }
       float dsum;
       if (!(ok = exchange(&sm.xdb, sm.xd, dsum2.x + dsum2.y, ph, kSiteXchg, dsum))) break;
