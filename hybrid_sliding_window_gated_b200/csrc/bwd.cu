@@ -101,10 +101,13 @@ __device__ __forceinline__ uint32_t row_to_f16(uint8_t* tile, int row, int hs = 
   uint32_t m = 0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint4* p = reinterpret_cast<uint4*>(tile + h * hs + row * 128);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const uint4 u = p[c];
+      // chunk c of the row in its swizzled place: the 32 rows of a warp then
+      // spread over all banks (row-linear order would put every lane's access
+      // in the same four)
+      uint4* p = reinterpret_cast<uint4*>(tile + h * hs + sw_off(row, c));
+      const uint4 u = *p;
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       uint32_t o[4];
 #pragma unroll
@@ -113,7 +116,7 @@ __device__ __forceinline__ uint32_t row_to_f16(uint8_t* tile, int row, int hs = 
         const float2 f = bf2(w[e]);
         o[e] = pack_f16x2(f.x, f.y);
       }
-      p[c] = make_uint4(o[0], o[1], o[2], o[3]);
+      *p = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
   return max(m & 0xFFFFu, m >> 16);
