@@ -835,7 +835,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* grow = reinterpret_cast<const uint8_t*>(a.g + tok * kHeadDim) + 128 * cg;
       const uint8_t* dorow = reinterpret_cast<const uint8_t*>(a.dO + tok * kHeadDim) + 128 * cg;
       // Rows past T take lse = +inf: their P is exactly 0 with no mask.
-      const float lse2 = valid_row ? a.lse[lrow] * kLog2e : INFINITY;
+      const float lse_r = valid_row ? a.lse[lrow] : INFINITY;  // loaded once, used twice
+      const float lse2 = lse_r * kLog2e;
       // this warpgroup's 64 columns of g and dO, in flight during P
       uint32_t gc[32], dc[32];  // this warpgroup's 64 columns of g and dO
       if (valid_row) {
@@ -919,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = warp_wait(&sm.xlb, ph, abort, a.err, kSiteXchg))) break;
         lsum = lsum2.x + lsum2.y + sm.xl[cg ^ 1][row];
         ei = min(eh, sm.xe[cg ^ 1][row]);
-        if (cg == 0 && row == 0) {  // the key-major pass's common scale starts here
+        if (cg == 1 && row == 0) {  // the key-major pass's common scale starts here
           int mn = kExpLimit;
 #pragma unroll
           for (int w = 0; w < 8; ++w) mn = min(mn, sm.xew[ph][w >> 2][w & 3]);
@@ -954,8 +955,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = lsum > 0.f ? 1.0f / lsum : 0.f;
       // in log2 units, with the row's exponent added (the key-major pass
       // subtracts its common exponent and so scales P^T column by column)
-      if (cg == 0 && valid_row)
-        a.ws_lse[lrow] = (a.lse[lrow] + __logf(lsum)) * kLog2e + static_cast<float>(ei);
+      // (warpgroup 1 writes the row's workspace entries: it has the fewer P chunks)
+      if (cg == 1 && valid_row)
+        a.ws_lse[lrow] = (lse_r + __logf(lsum)) * kLog2e + static_cast<float>(ei);
 
       // ---- dA = dO sigma(g) 2^e over this warpgroup's 64 columns, into the
       // Q slot (QK^T has read it): dA needs no A, so the dP MMAs start on it
@@ -1014,7 +1016,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float dsum;
       if (!(ok = exchange(&sm.xdb, sm.xd, dsum2.x + dsum2.y, ph, kSiteXchg, dsum))) break;
-      if (cg == 0 && valid_row) a.ws_d[lrow] = dsum;
+      if (cg == 1 && valid_row) a.ws_d[lrow] = dsum;
 
       // ---- dS = scale P (dP - D) per key tile into the Q slot (this
       // warpgroup's 64 columns), then dQ
