@@ -1061,19 +1061,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = warp_wait(&sm.dq0, ndq0 & 1, abort, a.err, kSiteDQ0))) break;
           ++ndq0;
         }
-#pragma unroll 1
+        // both chunks' P and dP in flight at once, then one wait
+        uint32_t pkc[2][16], dp[2][32];
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          tmem_ld16(t_row + tb + (blk ? sc : sc ^ 1) * 64 + (2 * cg + hc) * 16, pkc[hc]);
+          tmem_ld32(t_row + tw + (blk ? sc : sc ^ 1) * 128 + (2 * cg + hc) * 32, dp[hc]);
+        }
+        tmem_wait_ld();
+#pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
           const int pc = 2 * cg + hc;
-          uint32_t pkc[16], dp[32];
-          tmem_ld16(t_row + tb + (blk ? sc : sc ^ 1) * 64 + pc * 16, pkc);
-          tmem_ld32(t_row + tw + (blk ? sc : sc ^ 1) * 128 + pc * 32, dp);
-          tmem_wait_ld();
           uint32_t ds[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float2 v = __fmul2_rn(
-                __fmul2_rn(f16x2(pkc[e]), sl2),
-                __fadd2_rn(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                __fmul2_rn(f16x2(pkc[hc][e]), sl2),
+                __fadd2_rn(make_float2(__uint_as_float(dp[hc][2 * e]),
+                                       __uint_as_float(dp[hc][2 * e + 1])),
                            nd2));
             ds[e] = pack_f16x2(v.x, v.y);
           }
