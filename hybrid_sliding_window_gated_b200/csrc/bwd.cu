@@ -340,6 +340,11 @@ __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t
 __device__ __forceinline__ uint64_t desc_ring(const uint8_t (*ring)[2][kHalfBytes], int kk) {
   return desc_advance(make_desc_sw128(smem_u32(ring[kk >> 2][0]), 16, 1024), (kk & 3) * 32);
 }
+// K-major descriptor of one slot of a ring (128 rows) for k-step kk.
+__device__ __forceinline__ uint64_t desc_ring_slot(const uint8_t (*ring)[2][kHalfBytes], int slot,
+                                                   int kk) {
+  return desc_advance(make_desc_sw128(smem_u32(ring[kk >> 2][slot]), 16, 1024), (kk & 3) * 32);
+}
 // MN-major descriptor of one slot of a ring for k-step kk (its halves 32 KiB apart).
 __device__ __forceinline__ uint64_t desc_mn_ring(const uint8_t (*ring)[2][kHalfBytes], int slot,
                                                  int kk) {
@@ -635,12 +640,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!W(&sm.qready[n & 1], (n >> 1) & 1u, kSiteQReady)) break;
         tc_fence_after();
-        // Head n's S, P, A and dQ live in the TMEM half tb (0 or 256, by the
-        // parity of n), its dP in the other one, tw.  This head's S
-        // overwrites only what the previous head's dS phase has read (its
-        // dP), not its dQ, so it goes right behind the previous dQ; this
-        // head's dP follows its dA, which the compute warps write only after
-        // the previous head's dq epilogue.
+        // TMEM of head n, with tb = 0 or 256 by the parity of n and tw the
+        // other half: S in tb .. tb + 255, then A and later dQ over its second
+        // half; P in tw .. tw + 127; dP of ring slot 0 in tb .. tb + 127 and of
+        // slot 1 in tw + 128 .. tw + 255.  This head's S overwrites only what
+        // the previous head's dS phase has read (its P and slot-1 dP), not its
+        // dQ, so it goes right behind the previous dQ; everything else of this
+        // head is written after the compute warps' previous dq epilogue.
         const uint32_t tb = (n & 1) * 256u, tw = 256u - tb;
         // S = Q' [K' slot 0; K' slot 1]^T into columns tb .. tb + 255, one
         // N = 256 MMA per k-step: columns tb + 128 s .. hold the key tile in
@@ -660,32 +666,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           vpar ^= 1u << sc;
         }
         // A = P V into columns tb + 128 .. tb + 255, which S's second half held
-        // (P packed in columns tb .. tb + 127)
+        // (P packed in columns tw .. tw + 127)
         if (!W(&sm.pfull, ph, kSitePFull)) break;
         tc_fence_after();
         {
           uint32_t acc = 0;
           for (int blk = hp ? 0 : 1; blk < 2; ++blk)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns tb + 64 s ..
+            for (int kk = 0; kk < 8; ++kk) {  // P of the tile in slot s: columns tw + 64 s ..
               const int slot = blk ? sc : sp;
-              mma_ts(tmem + tb + 128, tmem + tb + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
+              mma_ts(tmem + tb + 128, tmem + tw + slot * 64 + kk * 8, desc_mn_ring(sm.v, slot, kk),
                      kIdescKM16, acc);
               acc = 1;
             }
         }
         mma_commit(&sm.afull);
-        // dP = dA [V_{t-1} V_t]^T into columns tw .. tw + 255.  The dA tile goes to
-        // the workspace (for the key-major pass) while the MMAs read it too;
-        // dS overwrites it after dpfull, which follows the store's read.
+        // dP = dA V^T per key tile: ring slot 0's into columns tb .. tb + 127
+        // (S's first half), slot 1's into tw + 128 .. tw + 255, clear of P and
+        // A.  The dA tile goes to the workspace (for the key-major pass) while
+        // the MMAs read it too; dS overwrites it after dpfull, which follows
+        // the store's read.
         if (!W(&sm.dafull, ph, kSiteDAFull)) break;
         tc_fence_after();
         bulk_store(da_tile(a, c.b, c.kvh * a.G + h, c.t), sm.slot[n & 1], kTileBytes);
         bulk_commit();
+        for (int blk = hp ? 0 : 1; blk < 2; ++blk) {
+          const int s = blk ? sc : sp;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dP of the tile in slot s: columns tw + 128 s ..
-          mma_ss(tmem + tw, desc_kmajor(sm.slot[n & 1], kk), desc_ring(sm.v, kk), kIdescKK16x256,
-                 kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + (s == 0 ? tb : tw + 128), desc_kmajor(sm.slot[n & 1], kk),
+                   desc_ring_slot(sm.v, s, kk), kIdescKK16, kk > 0);
+        }
         bulk_wait_read<0>();
         mma_commit(&sm.dpfull);
         // dQ = sum over key tiles of dS K' into columns tb + 128 .. tb + 255
@@ -855,9 +866,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- P = exp(s - lse) on the band.  The in-band 32-column chunks are
       // key tile t-1's wq4..3 (when it exists), then key tile t's 0..wq4;
       // this warpgroup takes every other one.  A key tile's S sits at the
-      // columns of its ring slot (128 s ..), its P at 64 s ..: P is packed
-      // over S's first 128 columns, which the other warpgroup may still be
-      // reading, so the stores wait for the exchange of the row sums.
+      // columns of its ring slot (tb + 128 s ..), its P at tw + 64 s .., clear
+      // of S: each chunk's P is stored as soon as it is computed, and PV may
+      // start before the row sums are exchanged.
       if (!(ok = warp_wait(&sm.sfull, ph, abort, a.err, kSiteSFull))) break;
       tc_fence_after();
       // Q' done.  Its 1/rms, read in the dq epilogue, stays until head n+3's
@@ -869,14 +880,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sp = sc ^ 1;  // ring slot of key tile t-1
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
       float2 lsum2 = make_float2(0.f, 0.f);
-      uint32_t pk[3][16];
 #pragma unroll
       for (int k = 0; k < 3; ++k) {
         const int i = cg + 2 * k;
         if (i < nch) {
           const int blk = i < na ? 0 : 1;
           const int pc = blk == 0 ? wq4 + i : i - na;
-          uint32_t x[32];
+          uint32_t x[32], pk[16];
           tmem_ld32(t_row + tb + (blk ? sc : sp) * 128 + pc * 32, x);
           tmem_wait_ld();
           if (pc != wq4) {
@@ -884,8 +894,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 16; ++e) {
               const float2 z = __ffma2_rn(
                   make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
-              pk[k][e] = pack_f16x2(ex2_approx(z.x), ex2_approx(z.y));
-              lsum2 = __fadd2_rn(lsum2, f16x2(pk[k][e]));  // the values the MMAs see
+              pk[e] = pack_f16x2(ex2_approx(z.x), ex2_approx(z.y));
+              lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));  // the values the MMAs see
             }
           } else {
 #pragma unroll
@@ -895,12 +905,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               const bool in1 = blk == 0 ? c0 + 1 > row : c0 + 1 <= row;
               const float2 z = __ffma2_rn(
                   make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), sc2, nl2);
-              pk[k][e] = pack_f16x2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
-              lsum2 = __fadd2_rn(lsum2, f16x2(pk[k][e]));
+              pk[e] = pack_f16x2(in0 ? ex2_approx(z.x) : 0.f, in1 ? ex2_approx(z.y) : 0.f);
+              lsum2 = __fadd2_rn(lsum2, f16x2(pk[e]));
             }
           }
+          tmem_st16(t_row + tw + (blk ? sc : sp) * 64 + pc * 16, pk);
         }
       }
+      {
+        // chunks outside the band: key tile t-1's below wq4 (or all of it
+        // when it does not exist) by cg 0, key tile t's above wq4 by cg 1
+        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        for (int pc = 0; pc < 4; ++pc) {
+          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + tw + sp * 64 + pc * 16, zero16);
+          if (cg == 1 && pc > wq4) tmem_st16(t_row + tw + sc * 64 + pc * 16, zero16);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.pfull);
       // The row's dA exponent e: each warpgroup takes it from its 64 values of
       // dO and the two are exchanged with l (the row takes the smaller).  Each
       // warp's minimum goes to shared memory too, for the tile's minimum.
@@ -929,28 +953,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           a.ws_ee[(static_cast<long long>(c.b) * a.Hq + hq) * a.tiles_per_chain + c.t] = mn;
         }
       }
-      {
-        const uint32_t zero16[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
-                                     0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int i = cg + 2 * k;
-          if (i < nch) {
-            const int blk = i < na ? 0 : 1;
-            const int pc = blk == 0 ? wq4 + i : i - na;
-            tmem_st16(t_row + tb + (blk ? sc : sp) * 64 + pc * 16, pk[k]);
-          }
-        }
-        // chunks outside the band: key tile t-1's below wq4 (or all of it
-        // when it does not exist) by cg 0, key tile t's above wq4 by cg 1
-        for (int pc = 0; pc < 4; ++pc) {
-          if (cg == 0 && (!hp || pc < wq4)) tmem_st16(t_row + tb + sp * 64 + pc * 16, zero16);
-          if (cg == 1 && pc > wq4) tmem_st16(t_row + tb + sc * 64 + pc * 16, zero16);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.pfull);
       // The forward's lse came from its own rounding of the scores; these rows
       // are renormalised to sum to exactly 1 under this pass's scores, and the
       // corrected normaliser goes to the key-major pass.
@@ -1065,8 +1067,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pkc[2][16], dp[2][32];
 #pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
-          tmem_ld16(t_row + tb + (blk ? sc : sc ^ 1) * 64 + (2 * cg + hc) * 16, pkc[hc]);
-          tmem_ld32(t_row + tw + (blk ? sc : sc ^ 1) * 128 + (2 * cg + hc) * 32, dp[hc]);
+          const int s = blk ? sc : sc ^ 1;  // the key tile's ring slot
+          tmem_ld16(t_row + tw + s * 64 + (2 * cg + hc) * 16, pkc[hc]);
+          tmem_ld32(t_row + (s == 0 ? tb : tw + 128) + (2 * cg + hc) * 32, dp[hc]);
         }
         tmem_wait_ld();
 #pragma unroll
