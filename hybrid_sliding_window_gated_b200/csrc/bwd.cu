@@ -75,8 +75,9 @@ __device__ __forceinline__ float2 f16x2(uint32_t u) {
 }
 // 32 bytes of one row per thread in one access (rows are 32-byte aligned):
 // a warp's row-per-thread access then touches each 32-byte sector once.  The
-// rows stream through once, so they skip L1: with the shared memory these
-// kernels take, L1 keeps about 28 KB, which the register spills need.
+// rows stream through once, so loads and stores both skip L1: with the
+// shared memory these kernels take, L1 keeps about 28 KB, which the register
+// spills need.
 __device__ __forceinline__ void ld32B(const void* p, uint32_t (&r)[8]) {
   asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
@@ -84,7 +85,7 @@ __device__ __forceinline__ void ld32B(const void* p, uint32_t (&r)[8]) {
                : "l"(p));
 }
 __device__ __forceinline__ void st32B(void* p, const uint32_t (&r)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]),
+  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]),
                "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
 }
