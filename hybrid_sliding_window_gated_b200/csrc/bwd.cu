@@ -23,7 +23,8 @@
 // except the per-CTA sums of dwq and dwk.
 //
 // Roles: warp 0 TMA producer (its lanes also compute rotation tables), warp 1
-// TMEM allocator and MMA issuer; both passes run 384 threads with registers
+// TMEM allocator and MMA issuer, and in the query-major pass warps 2-3 the Q
+// transform, a head ahead; both passes run 384 threads with registers
 // rebalanced by setmaxnreg and two compute warpgroups, warps 4-7 and 8-11,
 // thread r of each on tile row r.  In the query-major pass they share every
 // row: each takes half of the row's columns and they exchange the row sums
